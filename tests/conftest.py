@@ -1,0 +1,33 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+GOLDEN = os.path.join(ROOT, "tests", "golden")
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a) and the built library")
+    config.addinivalue_line("markers", "slow: long-running CPU check")
+
+
+def read_golden(name):
+    """Parse ``key = v1 v2 ...`` lines of a golden fixture (``#`` starts a comment)."""
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            k, v = line.split("=", 1)
+            out[k.strip()] = v.split()
+    return out
+
+
+@pytest.fixture
+def golden():
+    return read_golden

@@ -1,0 +1,385 @@
+"""Benchmark of the FP8 delayed-scaling linear hot path on B200.
+
+One step = the whole hot path over one batch of the 1.2B-model linear
+workload (hidden 1536, FFN 4096) at M = 8192 tokens, for both linear shapes
+(W1 [1536,1536], W2 [4096,1536]):
+  quantize X [M,1536] dual E4M3, W dual E4M3, G [M,N] dual E5M2 (rings
+  carried across steps: delayed scaling), then
+  fwd  Y  = Xq . Wq^T * sx*sw + b      (M x N x 1536)
+  dX   = Gq . (W^T)q^T * sg*sw          (M x 1536 x N, A = E5M2)
+  dW   = (G^T)q . (X^T)q^T * sg*sx      (N x 1536 x M, A = E5M2)
+12 kernel launches per step (6 quantize, 6 GEMM).
+
+Printed JSON line (rank 0): value = GEMM TFLOP/s of the whole step (GEMM
+flops / step time, quantize time included), plus the GEMM-only TFLOP/s,
+quantize GB/s, the roofline of the dominant kernel (the GEMM), clocks sampled
+during the timed region, an end-to-end figure through the C ABI with host
+buffers, and the CPU oracle baseline.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--M 8192]
+Multi-GPU: one process per GPU under torch.distributed.run; the path has no
+exchange step, so ranks run independent replicas (weak scaling) and only the
+timing is reduced (max over ranks).
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+HIDDEN, FFN = 1536, 4096
+METRIC = "mm_fp8 TFLOP/s & quantize GB/s on 1 B200, % of FP8/HBM roofline"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--M", type=int, default=8192)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def gemm_flops(M):
+    return sum(3 * 2 * M * n * HIDDEN for n in (HIDDEN, FFN))
+
+
+def quant_bytes(M):
+    """Algorithmic bytes of the 6 dual quantizes of one step: n*2 (bf16 in) + n*2 (two fp8 outs) + ring."""
+    tot = 0
+    for n in (HIDDEN, FFN):
+        for elems in (M * HIDDEN, n * HIDDEN, M * n):
+            tot += elems * 4 + 96
+    return tot
+
+
+# ---------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits", "-lms", "200",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------- the workload ----
+
+class Linear:
+    """Device state of one FP8 linear: weights, bias, rings, output buffers, input sets."""
+
+    def __init__(self, M, n_out, w, bias, inputs, torch, ops):
+        self.M, self.N = M, n_out
+        dev = "cuda"
+        self.w = w.to(dev)
+        self.bias = bias.to(dev)
+        self.rx, self.rw, self.rg = ops.Ring(), ops.Ring(), ops.Ring()
+        u8 = torch.uint8
+        self.xq = torch.empty((M, HIDDEN), dtype=u8, device=dev)
+        self.xq_t = torch.empty((HIDDEN, M), dtype=u8, device=dev)
+        self.wq = torch.empty((n_out, HIDDEN), dtype=u8, device=dev)
+        self.wq_t = torch.empty((HIDDEN, n_out), dtype=u8, device=dev)
+        self.gq = torch.empty((M, n_out), dtype=u8, device=dev)
+        self.gq_t = torch.empty((n_out, M), dtype=u8, device=dev)
+        bf = torch.bfloat16
+        self.y = torch.empty((M, n_out), dtype=bf, device=dev)
+        self.dx = torch.empty((M, HIDDEN), dtype=bf, device=dev)
+        self.dw = torch.empty((n_out, HIDDEN), dtype=bf, device=dev)
+        self.inputs = [(x.to(dev), g.to(dev)) for x, g in inputs]
+
+    def quantize(self, ops, x, g, ev=None):
+        ops.quantize(x, ops.E4M3, ops.DUAL, self.rx, self.xq, self.xq_t)
+        ops.quantize(self.w, ops.E4M3, ops.DUAL, self.rw, self.wq, self.wq_t)
+        ops.quantize(g, ops.E5M2, ops.DUAL, self.rg, self.gq, self.gq_t)
+
+    def gemms(self, ops):
+        ops.mm(self.xq, self.wq, self.rx.scale_inv, self.rw.scale_inv, self.bias, out=self.y)
+        ops.mm(self.gq, self.wq_t, self.rg.scale_inv, self.rw.scale_inv, None, fmt_a=ops.E5M2, out=self.dx)
+        ops.mm(self.gq_t, self.xq_t, self.rg.scale_inv, self.rx.scale_inv, None, fmt_a=ops.E5M2, out=self.dw)
+
+
+def build_workload(M, torch, ops, S, n_sets=2):
+    (w1, b1), (w2, b2) = S.linear_1p2b_weights()
+    lins = []
+    for n_out, w, b in ((HIDDEN, w1, b1), (FFN, w2, b2)):
+        sets = [S.linear_1p2b_step(M, n_out, s) for s in range(n_sets)]
+        lins.append(Linear(M, n_out, w, b, sets, torch, ops))
+    return lins
+
+
+def run_step(lins, ops, i):
+    for L in lins:
+        x, g = L.inputs[i % len(L.inputs)]
+        L.quantize(ops, x, g)
+        L.gemms(ops)
+
+
+def time_split(lins, ops, torch, reps):
+    """Per-phase device time (quantize vs GEMM) with events on the launching stream."""
+    st = torch.cuda.current_stream()
+    q_ms, g_ms = 0.0, 0.0
+    for i in range(reps):
+        for L in lins:
+            x, g = L.inputs[i % len(L.inputs)]
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            e0.record(st)
+            L.quantize(ops, x, g)
+            e1.record(st)
+            L.gemms(ops)
+            e2.record(st)
+            e2.synchronize()
+            q_ms += e0.elapsed_time(e1)
+            g_ms += e1.elapsed_time(e2)
+    return q_ms / reps, g_ms / reps
+
+
+# ------------------------------------------------------------- CPU oracle ----
+
+def cpu_baseline(M_full, seconds=12.0):
+    """The oracle as it stands, on a row sample of the same step, timed on host cores."""
+    import numpy as np
+
+    from fp8_delayed_scaling_02_b200 import synthetic as S
+    from oracle import gemm as OG
+    from oracle import recipe as OR
+
+    Ms = 256
+    (w1, b1), (w2, b2) = S.linear_1p2b_weights()
+    flops = 0
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        for n_out, w, b in ((HIDDEN, w1, b1), (FFN, w2, b2)):
+            x, g = S.linear_1p2b_step(Ms, n_out, 0)
+            rx, rw, rg = OR.Ring(), OR.Ring(), OR.Ring()
+            xq, xq_t, _ = OR.quantize(x, 0, OR.DUAL, rx)
+            wq, wq_t, _ = OR.quantize(w, 0, OR.DUAL, rw)
+            gq, gq_t, _ = OR.quantize(g, 1, OR.DUAL, rg)
+            OG.mm_fp8(xq, wq, 0, 0, rx.scale_inv, rw.scale_inv, b.numpy())
+            OG.mm_fp8(gq, wq_t, 1, 0, rg.scale_inv, rw.scale_inv)
+            OG.mm_fp8(gq_t, xq_t, 1, 0, rg.scale_inv, rx.scale_inv)
+            flops += 3 * 2 * Ms * n_out * HIDDEN
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds or reps >= 50:
+            break
+    try:
+        import threadpoolctl
+
+        cores = max((p.get("num_threads", 1) for p in threadpoolctl.threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count()
+    return {"value": flops / el / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"the same step (both linears: 6 quantizes + 3 GEMMs each) on {Ms} of {M_full} rows/tokens, "
+                      f"{reps} repetitions in {el:.1f} s; numpy float64 oracle"}
+
+
+# -------------------------------------------------------------------- main ----
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        cb = cpu_baseline(args.M, seconds=8.0)
+        # Each "step" of the reference arm is one bounded sample of the workload.
+        line = {"impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "TFLOP/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": None, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic",
+                "config": {"workload": f"1.2B-model linears fwd+bwd (hidden 1536, FFN 4096), M={args.M}, "
+                                       "row sample on CPU"},
+                "cpu_baseline": cb,
+                "e2e": {"value": cb["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+
+    from fp8_delayed_scaling_02_b200 import build as B
+    from fp8_delayed_scaling_02_b200 import ops, synthetic as S
+
+    B.build()
+    torch.cuda.set_device(local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+
+    M = args.M
+    lins = build_workload(M, torch, ops, S)
+    for i in range(max(3, args.warmup)):
+        run_step(lins, ops, i)
+    torch.cuda.synchronize()
+    q_ms, g_ms = time_split(lins, ops, torch, 5)
+
+    st = torch.cuda.current_stream()
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(st)
+        for i in range(args.steps):
+            run_step(lins, ops, i)
+        e1.record(st)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    if pg:
+        t = torch.tensor([ms], device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+        pg.barrier()
+    flops = gemm_flops(M)
+    value = world * flops / (ms * 1e-3) / 1e12
+
+    # End to end through the C ABI: pinned host X and G copied in, Y, dX, dW copied out, every step.
+    e2e = None
+    if not args.no_e2e:
+        host_in = [[(x.cpu().pin_memory(), g.cpu().pin_memory()) for x, g in L.inputs] for L in lins]
+        host_out = [(torch.empty(L.y.shape, dtype=L.y.dtype).pin_memory(),
+                     torch.empty(L.dx.shape, dtype=L.dx.dtype).pin_memory(),
+                     torch.empty(L.dw.shape, dtype=L.dw.dtype).pin_memory()) for L in lins]
+        h2d = sum(x.numel() * x.element_size() + g.numel() * g.element_size() for x, g in (h[0] for h in host_in))
+        d2h = sum(sum(t.numel() * t.element_size() for t in ho) for ho in host_out)
+        steps_e2e = max(3, args.steps // 5)
+        if pg:
+            pg.barrier()
+        torch.cuda.synchronize()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(st)
+        for i in range(steps_e2e):
+            for L, hin, hout in zip(lins, host_in, host_out):
+                hx, hg = hin[i % len(hin)]
+                x, g = L.inputs[i % len(L.inputs)]
+                x.copy_(hx, non_blocking=True)
+                g.copy_(hg, non_blocking=True)
+                L.quantize(ops, x, g)
+                L.gemms(ops)
+                hout[0].copy_(L.y, non_blocking=True)
+                hout[1].copy_(L.dx, non_blocking=True)
+                hout[2].copy_(L.dw, non_blocking=True)
+        a1.record(st)
+        torch.cuda.synchronize()
+        ms_e2e = a0.elapsed_time(a1) / steps_e2e
+        if pg:
+            t = torch.tensor([ms_e2e], device="cuda")
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            ms_e2e = float(t.item())
+        e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except (OSError, ValueError):
+        pass
+    if "bf16_tflops_sustained" in peaks:
+        fp8_peak, peak_src = 2.0 * peaks["bf16_tflops_sustained"], "of measured (bf16 sustained x 2)"
+    else:
+        fp8_peak, peak_src = 2.0 * 1400.0, "of fallback (1.4 PF/s bf16 sustained x 2)"
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    gemm_tf = flops / (g_ms * 1e-3) / 1e12
+    qb = quant_bytes(M)
+    quant_gbs = qb / (q_ms * 1e-3) / 1e9
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3/e5m2->f32acc->bf16",
+            "data": "synthetic",
+            "config": {"workload": f"1.2B-model linears fwd+bwd (hidden 1536, FFN 4096), M={M} tokens, "
+                                   "X/W/G dual quantize + fwd/dX/dW mm_fp8 for both linear shapes",
+                       "M": M, "linears": [[HIDDEN, HIDDEN], [FFN, HIDDEN]],
+                       "l2": "no flush: 2 rotating input sets, ~320 MB per set pair > 126 MB L2",
+                       "parallelism": f"replicas x{world}"},
+            "mm_tflops": round(gemm_tf, 2), "quantize_gbs": round(quant_gbs, 1),
+            "quantize_ms_per_step": round(q_ms, 4), "mm_ms_per_step": round(g_ms, 4),
+            "roofline": {"bound": "tensor", "achieved": round(gemm_tf, 2), "peak": round(fp8_peak, 1),
+                         "unit": "TFLOP/s", "frac": round(gemm_tf / fp8_peak, 4), "traffic": None,
+                         "kernel": "mm_fp8_kernel (all 6 GEMM launches of the step)", "peak_source": peak_src},
+            "quantize_roofline": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
+                                  "frac": round(quant_gbs / hbm_peak, 4), "peak_source": "of measured hbm_gbs"},
+            "clocks": clk.summary(),
+            "gpu_launches": 12 * args.steps,
+            "e2e": e2e,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(M)
+        print(json.dumps(line))
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

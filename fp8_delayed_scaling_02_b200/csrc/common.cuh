@@ -1,0 +1,53 @@
+// Shared device/host helpers of the fp8ds library (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fp8ds.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "fp8ds is written for sm_100a (B200) only"
+#endif
+
+namespace fp8ds {
+
+constexpr int kHistoryLen = 16;
+constexpr float kE4M3Max = 448.0f;
+constexpr float kE5M2Max = 57344.0f;
+
+// Codes for the device error word: which bounded wait gave up.
+enum WaitSite : uint32_t {
+  kWaitNone = 0,
+  kWaitProducerEmpty = 1,
+  kWaitMmaFull = 2,
+  kWaitMmaTmemEmpty = 3,
+  kWaitEpilogueTmemFull = 4,
+  kWaitDrain = 5,
+};
+
+// Library-global device error word (defined in capi.cu, relocatable device code
+// is not used, so each translation unit that records errors gets the address
+// through error_word_ptr()).
+uint32_t* error_word_ptr();
+
+// Nanosecond budget of every bounded wait in a kernel.
+constexpr unsigned long long kWaitBudgetNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void record_device_error(uint32_t* word, uint32_t site) {
+  if (word != nullptr) atomicCAS(word, 0u, site);
+}
+
+}  // namespace fp8ds
+
+#define FP8DS_CUDA_CHECK(expr)                 \
+  do {                                         \
+    cudaError_t e_ = (expr);                   \
+    if (e_ != cudaSuccess) return FP8_ERR_CUDA; \
+  } while (0)

@@ -1,0 +1,560 @@
+// fp8_mm: scaled FP8 GEMM (NT, batched with stride-0 broadcast) for sm_100a.
+//
+// Computes Y[b,m,n] = bf16(sum_k A[b,m,k] B[b,n,k] * sinv_a * sinv_b + bias[n])
+// as the AstrAI pages describe it ("tests/extension": bias-fusion commit --
+// the fp32 bias is added before the single bf16 rounding, guarded N tails,
+// batch broadcast of the bias; 3D batched commit -- batch strides, size-1
+// batches broadcast at stride 0; grouped rasterisation keeps the shared
+// operand stripe hot in L2).
+//
+// B200 design (the pages' kernels are sm_89 register-fragment MMAs; none of
+// that carries over):
+//   * persistent kernel, one CTA per SM, 6 warps with fixed roles:
+//       warp 0      TMA producer: 128x128-byte A and BNx128-byte B tiles,
+//                   128B-swizzled, into a STAGES-deep shared-memory ring
+//                   guarded by full/empty mbarriers;
+//       warp 1      TMEM allocator and single-thread tcgen05.mma issuer
+//                   (kind::f8f6f4, M=128, N=BN, K=32 per instruction), fp32
+//                   accumulators in TMEM, double-buffered (2 x BN columns) so
+//                   the epilogue of tile i overlaps the mainloop of tile i+1;
+//       warps 2..5  epilogue: tcgen05.ld 32 columns at a time, one fmaf per
+//                   element (acc * sinv_a*sinv_b + bias), one bf16 rounding,
+//                   16-byte stores with guarded tails.
+//   * every mbarrier wait is bounded by a %globaltimer budget; a wait that
+//     runs out records the site in the library error word, raises a shared
+//     abort flag so the other roles leave their loops, waits (bounded) for
+//     the copies and MMAs it issued, frees TMEM and returns.
+//   * no TMA multicast anywhere: the kernel stays legal when several GPUs
+//     run replicas.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace fp8ds {
+namespace {
+
+constexpr int kBM = 128;      // rows of A per tile (UMMA M)
+constexpr int kBK = 128;      // K bytes (= fp8 elements) per stage: one 128B swizzle atom row
+constexpr int kUmmaK = 32;    // K per tcgen05.mma for 8-bit operands
+constexpr int kThreadsMM = 192;
+
+template <int BN>
+struct Cfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = kBM * kBK;
+  static constexpr int kBBytes = BN * kBK;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = 2 * BN;  // two accumulators
+  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
+};
+
+struct MmParams {
+  int M, N, K;
+  int m_tiles, n_tiles, k_blocks, tiles_per_batch, tiles_total, group_m;
+  int a_bcast, b_bcast;
+  int64_t c_stride;  // elements between output batches
+  const float* sinv_a;
+  const float* sinv_b;
+  const float* bias;
+  uint16_t* out;
+  int out_vec;       // 16-byte stores are legal for full 8-column groups
+  int bias_vec;      // bias is 16-byte aligned
+  uint32_t idesc;
+  uint32_t* err;
+};
+
+// ---- PTX wrappers (written from the PTX ISA description) -----------------------
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// Bounded wait for the phase of parity `parity` to complete.  Returns false if
+// the budget ran out (error recorded, abort raised) or another role aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* err,
+                                          uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > kWaitBudgetNs) {
+        record_device_error(err, site);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// 32 lanes x 32 consecutive 32-bit columns; lane t of the warp receives row
+// (32 * (warp % 4) + t) of the accumulator.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile written by TMA with the
+// 128-byte swizzle: 8-row x 128-byte atoms stacked along M/N every 1024 bytes
+// (stride byte offset), leading byte offset unused for this layout, version 1,
+// layout type 2 (128B swizzle).  The tile base is 1024-byte aligned.
+__device__ __forceinline__ uint64_t sdesc_k128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t(1) << 16;
+  d |= uint64_t(1024 >> 4) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
+__device__ __forceinline__ void decode_tile(const MmParams& p, int t, int& b, int& mt, int& nt) {
+  b = t / p.tiles_per_batch;
+  const int r = t - b * p.tiles_per_batch;
+  const int span = p.group_m * p.n_tiles;
+  const int g = r / span;
+  const int first_m = g * p.group_m;
+  const int gm = min(p.m_tiles - first_m, p.group_m);
+  const int rr = r - g * span;
+  mt = first_m + rr % gm;
+  nt = rr / gm;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreadsMM, 1)
+    mm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const MmParams p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled tiles.
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  const uint32_t sbase = smem_u32(smem);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOffset);
+  // bars[0, S) full, [S, 2S) empty, [2S, 2S+2) tmem_full, [2S+2, 2S+4) tmem_empty, [2S+4] mma_done
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 5);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::kStages + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::kStages + 2 + a); };
+  const uint32_t done_bar = bar0 + 8u * (2 * C::kStages + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 4);
+    }
+    mbar_init(done_bar, 1);
+    *abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;  // bit s: stage s armed; its parity
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.tiles_total; t += gridDim.x) {
+        int b, mt, nt;
+        decode_tile(p, t, b, mt, nt);
+        const int ba = p.a_bcast ? 0 : b;
+        const int bb = p.b_bcast ? 0 : b;
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort, p.err, kWaitProducerEmpty)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+          const uint32_t sa = sbase + stage * C::kABytes;
+          const uint32_t sb = sbase + C::kStages * C::kABytes + stage * C::kBBytes;
+          tma_load_3d(sa, &tmA, kb * kBK, mt * kBM, ba, full_bar(stage));
+          tma_load_3d(sb, &tmB, kb * kBK, nt * BN, bb, full_bar(stage));
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // Let every copy this thread issued land before shared memory is released.
+        for (int s = 0; s < C::kStages; ++s)
+          if (armed & (1u << s)) {
+            const unsigned long long t0 = globaltimer_ns();
+            while (!mbar_try_wait(full_bar(s), (armed_par >> s) & 1u) && globaltimer_ns() - t0 < kWaitBudgetNs) {
+            }
+          }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int i = 0;
+      bool ok = true;
+      const uint32_t sa0 = sbase;
+      const uint32_t sb0 = sbase + C::kStages * C::kABytes;
+      for (int t = blockIdx.x; ok && t < p.tiles_total; t += gridDim.x, ++i) {
+        const int acc = i & 1;
+        const uint32_t acc_par = (i >> 1) & 1;
+        if (!mbar_wait(tempty_bar(acc), acc_par ^ 1u, abort, p.err, kWaitMmaTmemEmpty)) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + uint32_t(acc * BN);
+        for (int kb = 0; kb < p.k_blocks; ++kb) {
+          if (!mbar_wait(full_bar(stage), phase, abort, p.err, kWaitMmaFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t ad = sdesc_k128(sa0 + stage * C::kABytes);
+          const uint64_t bd = sdesc_k128(sb0 + stage * C::kBBytes);
+#pragma unroll
+          for (int k = 0; k < kBK / kUmmaK; ++k) {
+            // +32 bytes along K inside the swizzle atom = +2 in the address field.
+            umma_f8(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), p.idesc, (kb | k) != 0 ? 1u : 0u);
+          }
+          umma_commit(empty_bar(stage));
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (p.k_blocks > 0) umma_commit(tfull_bar(acc));
+        else mbar_arrive(tfull_bar(acc));
+      }
+      // All MMAs this thread issued are complete before TMEM is released.
+      umma_commit(done_bar);
+      const unsigned long long t0 = globaltimer_ns();
+      while (!mbar_try_wait(done_bar, 0) && globaltimer_ns() - t0 < kWaitBudgetNs) {
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quad = warp & 3;
+    const float sab = __fmul_rn(*p.sinv_a, *p.sinv_b);
+    int i = 0;
+    for (int t = blockIdx.x; t < p.tiles_total; t += gridDim.x, ++i) {
+      const int acc = i & 1;
+      const uint32_t acc_par = (i >> 1) & 1;
+      if (!mbar_wait(tfull_bar(acc), acc_par, abort, p.err, kWaitEpilogueTmemFull)) break;
+      tc_fence_after();
+      int b, mt, nt;
+      decode_tile(p, t, b, mt, nt);
+      const int row = mt * kBM + quad * 32 + lane;
+      uint16_t* orow = p.out + int64_t(b) * p.c_stride + int64_t(row) * p.N;
+      for (int c = 0; c < BN / 32; ++c) {
+        const int n0 = nt * BN + c * 32;
+        if (n0 >= p.N) break;  // warp-uniform
+        uint32_t r[32];
+        if (p.k_blocks > 0) {
+          tmem_ld32(tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + c * 32), r);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) r[j] = 0u;
+        }
+        float bv[32];
+        const bool full = n0 + 32 <= p.N;
+        if (p.bias != nullptr) {
+          if (full && p.bias_vec) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 f = __ldg(reinterpret_cast<const float4*>(p.bias + n0) + j);
+              bv[4 * j] = f.x; bv[4 * j + 1] = f.y; bv[4 * j + 2] = f.z; bv[4 * j + 3] = f.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) bv[j] = (n0 + j < p.N) ? __ldg(p.bias + n0 + j) : 0.0f;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) bv[j] = 0.0f;
+        }
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float y0 = fmaf(__uint_as_float(r[2 * j]), sab, bv[2 * j]);
+          const float y1 = fmaf(__uint_as_float(r[2 * j + 1]), sab, bv[2 * j + 1]);
+          const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
+          packed[j] = *reinterpret_cast<const uint32_t*>(&h);
+        }
+        if (row < p.M) {
+          if (full && p.out_vec) {
+            uint4* o = reinterpret_cast<uint4*>(orow + n0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              o[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (n0 + j < p.N) orow[n0 + j] = uint16_t(packed[j >> 1] >> (16 * (j & 1)));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(acc));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// K == 0: Y = bf16(bias) or 0.
+__global__ void mm_bias_only_kernel(uint16_t* out, const float* bias, int64_t M, int64_t N, int64_t batch,
+                                    int64_t c_stride) {
+  const int64_t total = batch * M * N;
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t b = i / (M * N), r = i - b * M * N, n = r % N;
+    const __nv_bfloat16 h = __float2bfloat16_rn(bias ? bias[n] : 0.0f);
+    out[b * c_stride + r] = *reinterpret_cast<const uint16_t*>(&h);
+  }
+}
+
+// ---- host side -----------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 3-D map over uint8 [batch, rows, K] with a box of [1, box_rows, 128].
+bool make_map(CUtensorMap* m, const uint8_t* base, int64_t K, int64_t rows, int64_t batch, int64_t bstride,
+              int box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {cuuint64_t(K), cuuint64_t(rows), cuuint64_t(batch)};
+  const cuuint64_t strides[2] = {cuuint64_t(K), cuuint64_t(batch > 1 ? bstride : K * rows)};
+  const cuuint32_t box[3] = {cuuint32_t(kBK), cuuint32_t(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int BN>
+bool ensure_smem_attr() {
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(mm_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes) !=
+        cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+template <int BN>
+int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+              const int64_t* strides, MmParams p, int sms, cudaStream_t st) {
+  CUtensorMap ta, tb;
+  const int64_t ba = (batch > 1 && strides[0] != 0) ? batch : 1;
+  const int64_t bb = (batch > 1 && strides[1] != 0) ? batch : 1;
+  if (!make_map(&ta, A, K, M, ba, ba > 1 ? strides[0] : 0, kBM)) return FP8_ERR_CUDA;
+  if (!make_map(&tb, B, K, N, bb, bb > 1 ? strides[1] : 0, BN)) return FP8_ERR_CUDA;
+  p.a_bcast = ba == 1;
+  p.b_bcast = bb == 1;
+  p.m_tiles = int((M + kBM - 1) / kBM);
+  p.n_tiles = int((N + BN - 1) / BN);
+  p.tiles_per_batch = p.m_tiles * p.n_tiles;
+  p.tiles_total = int(p.tiles_per_batch * batch);
+  p.group_m = 8;
+  p.idesc |= uint32_t(BN >> 3) << 17;
+  if (!ensure_smem_attr<BN>()) return FP8_ERR_CUDA;
+  const int grid = std::max(1, std::min(p.tiles_total, sms));
+  mm_fp8_kernel<BN><<<grid, kThreadsMM, Cfg<BN>::kSmemBytes, st>>>(ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fp8ds
+
+using namespace fp8ds;
+
+extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+                      const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b,
+                      const float* bias, uint16_t* out_bf16, fp8_stream_t stream) {
+  if (M < 0 || N < 0 || K < 0 || batch < 1) return FP8_ERR_INVALID_ARG;
+  if ((layout & ~(FP8_MM_A_E5M2 | FP8_MM_B_E5M2)) != FP8_MM_NT) return FP8_ERR_INVALID_ARG;
+  if (batch > 1 && strides == nullptr) return FP8_ERR_INVALID_ARG;
+  if (batch > 1 && (strides[0] < 0 || strides[1] < 0 || strides[2] < 0)) return FP8_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return FP8_OK;
+  if (out_bf16 == nullptr || sinv_a == nullptr || sinv_b == nullptr) return FP8_ERR_INVALID_ARG;
+  if (K > 0 && (A == nullptr || B == nullptr)) return FP8_ERR_INVALID_ARG;
+  if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2 || batch > 65535) return FP8_ERR_UNSUPPORTED;
+  if (K % 16 != 0) return FP8_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(out_bf16) % 2 != 0) return FP8_ERR_UNSUPPORTED;
+  const int64_t c_stride = batch > 1 ? strides[2] : M * N;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+
+  if (K == 0) {
+    const int64_t total = batch * M * N;
+    const int grid = int(std::min<int64_t>((total + 255) / 256, 4096));
+    mm_bias_only_kernel<<<grid, 256, 0, st>>>(out_bf16, bias, M, N, batch, c_stride);
+    return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+  }
+  if (reinterpret_cast<uintptr_t>(A) % 16 != 0 || reinterpret_cast<uintptr_t>(B) % 16 != 0) return FP8_ERR_UNSUPPORTED;
+  if (batch > 1 && ((strides[0] % 16) != 0 || (strides[1] % 16) != 0)) return FP8_ERR_UNSUPPORTED;
+
+  const int sms = sm_count();
+  if (sms <= 0) return FP8_ERR_CUDA;
+
+  MmParams p{};
+  p.M = int(M);
+  p.N = int(N);
+  p.K = int(K);
+  p.k_blocks = int((K + kBK - 1) / kBK);
+  p.c_stride = c_stride;
+  p.sinv_a = sinv_a;
+  p.sinv_b = sinv_b;
+  p.bias = bias;
+  p.out = out_bf16;
+  p.out_vec = (reinterpret_cast<uintptr_t>(out_bf16) % 16 == 0) && (N % 8 == 0) && (c_stride % 8 == 0);
+  p.bias_vec = bias != nullptr && (reinterpret_cast<uintptr_t>(bias) % 16 == 0);
+  const uint32_t fa = (layout & FP8_MM_A_E5M2) ? 1u : 0u;
+  const uint32_t fb = (layout & FP8_MM_B_E5M2) ? 1u : 0u;
+  // Instruction descriptor: fp32 accumulator (bits 4-5 = 1), A format bits 7-9,
+  // B format bits 10-12 (0 = E4M3, 1 = E5M2), both K-major, M/16 at bits 24-28;
+  // N/8 (bits 17-22) is added by the launcher for its tile width.
+  p.idesc = (1u << 4) | (fa << 7) | (fb << 10) | (uint32_t(kBM >> 4) << 24);
+  p.err = error_word_ptr();
+
+  const int64_t tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256) * batch;
+  if (N > 128 && tiles256 >= sms) return launch_mm<256>(A, B, M, N, K, batch, strides, p, sms, st);
+  return launch_mm<128>(A, B, M, N, K, batch, strides, p, sms, st);
+}

@@ -1,0 +1,467 @@
+// fp8_quantize: delayed-scaling cast of bf16/fp16/fp32 to E4M3/E5M2 on sm_100a.
+//
+// What is computed follows the AstrAI pages: "tests/extension" (ring commit:
+// the last block folds amax into the history window and publishes the next
+// scale with an atomic ticket and fences; quantize bindings commit: row /
+// transposed / dual QuantLayout), "csrc/kernels/fp8/quantize.cuh" (one tiled
+// transpose kernel with vector loads and a scalar fallback for ragged or
+// unaligned rows) and "csrc/kernels/fp8_mm.cu" (amax of the raw values).
+//
+// B200 design (not the pages' sm_89 one):
+//   * ROW layout is a flat stream: each thread converts 16 elements per step
+//     and writes one 16-byte store; loads are 16-byte vectors, realigned with
+//     funnel shifts when the input base is only element-aligned (a 2-byte
+//     offset for bf16), so the misaligned case reads HBM at full width too.
+//     Grid = a multiple of the SM count, grid-stride, two chunks in flight
+//     per thread.
+//   * T / DUAL use a 128x64 tile per 256-thread block: each lane converts a
+//     4-row x 8-column patch, packs the 4 rows of each column into one 32-bit
+//     word, writes it to a padded shared tile (pitch 33 words: conflict-free
+//     writes and reads) and the block streams 128-byte rows of out_t.
+//   * amax: fmaxf over |x| (NaN ignored) -> warp shuffle -> block -> one
+//     atomicMax on the float bits per block (non-negative floats order as
+//     unsigned integers).  The ticket is an atomicAdd after __threadfence;
+//     the block that draws the last ticket folds the ring, publishes the
+//     scale and resets the scratch words to zero for the next call (no
+//     memset launch, no host involvement).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace fp8ds {
+namespace {
+
+constexpr int kThreads = 256;
+
+struct RingArgs {
+  float* history;
+  int32_t* idx;
+  float* scale;
+  float* scale_inv;
+  uint32_t* scratch;
+};
+
+// ---- element loads -----------------------------------------------------------
+
+template <int DT> struct In;
+template <> struct In<FP8_IN_BF16> { static constexpr int kBytes = 2; };
+template <> struct In<FP8_IN_FP16> { static constexpr int kBytes = 2; };
+template <> struct In<FP8_IN_FP32> { static constexpr int kBytes = 4; };
+
+template <int DT>
+__device__ __forceinline__ float load_one(const uint8_t* p) {
+  if constexpr (DT == FP8_IN_BF16) {
+    return __uint_as_float(uint32_t(*reinterpret_cast<const uint16_t*>(p)) << 16);
+  } else if constexpr (DT == FP8_IN_FP16) {
+    return __half2float(__ushort_as_half(*reinterpret_cast<const uint16_t*>(p)));
+  } else {
+    return *reinterpret_cast<const float*>(p);
+  }
+}
+
+// Two 16-bit elements packed in one word -> floats (low half first).
+template <int DT>
+__device__ __forceinline__ void unpack2(uint32_t w, float& lo, float& hi) {
+  if constexpr (DT == FP8_IN_BF16) {
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xFFFF0000u);
+  } else {
+    __half2 h = *reinterpret_cast<__half2*>(&w);
+    float2 f = __half22float2(h);
+    lo = f.x;
+    hi = f.y;
+  }
+}
+
+__device__ __forceinline__ uint4 ldg16(const uint8_t* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// Words [0, NW) of the byte stream that starts `ph` bytes past the 16-byte
+// aligned address `q`, given the aligned words W[0, NW + 4).  ph is a multiple
+// of the element size; the word shift is selected without dynamic register
+// indexing and the half-word remainder (16-bit types only) is a funnel shift.
+template <int NW>
+__device__ __forceinline__ void realign(const uint32_t (&W)[NW + 4], int ph, uint32_t (&D)[NW]) {
+  const int ws = ph >> 2;
+  uint32_t X[NW + 1];
+#pragma unroll
+  for (int i = 0; i <= NW; ++i) {
+    uint32_t a = W[i], b = W[i + 1], c = W[i + 2], d = W[i + 3];
+    X[i] = ws == 0 ? a : (ws == 1 ? b : (ws == 2 ? c : d));
+  }
+  const bool half = (ph & 2) != 0;
+#pragma unroll
+  for (int i = 0; i < NW; ++i) D[i] = half ? __funnelshift_r(X[i], X[i + 1], 16) : X[i];
+}
+
+// Load N (8 or 16) consecutive elements starting at element address p into v.
+// Only 16-byte granules that hold at least one of the N elements are read.
+template <int DT, int N>
+__device__ __forceinline__ void load_vec(const uint8_t* p, float (&v)[N]) {
+  constexpr int kB = In<DT>::kBytes;
+  constexpr int NW = N * kB / 4;      // useful words
+  constexpr int NG = NW / 4;          // useful granules when aligned
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  const int ph = int(a & 15);
+  const uint8_t* q = p - ph;
+  uint32_t W[NW + 4];
+#pragma unroll
+  for (int g = 0; g < NG; ++g) {
+    uint4 t = ldg16(q + 16 * g);
+    W[4 * g] = t.x; W[4 * g + 1] = t.y; W[4 * g + 2] = t.z; W[4 * g + 3] = t.w;
+  }
+  if (ph != 0) {
+    uint4 t = ldg16(q + 16 * NG);
+    W[4 * NG] = t.x; W[4 * NG + 1] = t.y; W[4 * NG + 2] = t.z; W[4 * NG + 3] = t.w;
+  } else {
+    W[4 * NG] = W[4 * NG + 1] = W[4 * NG + 2] = W[4 * NG + 3] = 0u;
+  }
+  uint32_t D[NW];
+  realign<NW>(W, ph, D);
+  if constexpr (kB == 2) {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) unpack2<DT>(D[i], v[2 * i], v[2 * i + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < NW; ++i) v[i] = __uint_as_float(D[i]);
+  }
+}
+
+// Aligned fast path (p is 16-byte aligned).
+template <int DT, int N>
+__device__ __forceinline__ void load_vec_aligned(const uint8_t* p, float (&v)[N]) {
+  constexpr int kB = In<DT>::kBytes;
+  constexpr int NW = N * kB / 4;
+#pragma unroll
+  for (int g = 0; g < NW / 4; ++g) {
+    uint4 t = ldg16(p + 16 * g);
+    uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if constexpr (kB == 2) {
+        unpack2<DT>(w[i], v[8 * g + 2 * i], v[8 * g + 2 * i + 1]);
+      } else {
+        v[4 * g + i] = __uint_as_float(w[i]);
+      }
+    }
+  }
+}
+
+// ---- conversion ------------------------------------------------------------
+
+// fp8 codes of (lo*s, hi*s) packed low byte first: one fp32 multiply each (no
+// contraction), then the hardware round-to-nearest-even conversion with
+// saturation to the largest finite value.
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt_pair(float lo, float hi, float s) {
+  float2 f = make_float2(__fmul_rn(lo, s), __fmul_rn(hi, s));
+  return uint32_t(__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, FMT == FP8_E4M3 ? __NV_E4M3 : __NV_E5M2));
+}
+
+template <int FMT>
+__device__ __forceinline__ uint8_t cvt_one(float x, float s) {
+  return uint8_t(__nv_cvt_float_to_fp8(__fmul_rn(x, s), __NV_SATFINITE,
+                                       FMT == FP8_E4M3 ? __NV_E4M3 : __NV_E5M2));
+}
+
+// ---- amax + ring fold --------------------------------------------------------
+
+// Block-reduce the per-thread amax, publish it with one atomicMax, draw a
+// ticket; the last block folds the ring.  Must be called by every thread.
+template <int FMT>
+__device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& ring, float s_used) {
+  __shared__ float warp_max[kThreads / 32];
+  __shared__ int last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if (lane == 0) warp_max[warp] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, warp_max[w]);
+    if (m > 0.0f) atomicMax(&ring.scratch[0], __float_as_uint(m));
+    __threadfence();  // release: our amax is visible before our ticket
+    const unsigned t = atomicAdd(&ring.scratch[1], 1u);
+    last = (t == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (last && threadIdx.x == 0) {
+    __threadfence();  // acquire: every block's amax is visible now
+    const float a = __uint_as_float(atomicExch(&ring.scratch[0], 0u));
+    int idx = *ring.idx;
+    idx = ((idx % kHistoryLen) + kHistoryLen) % kHistoryLen;
+    ring.history[idx] = a;
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kHistoryLen; ++i) m = fmaxf(m, ring.history[i]);
+    *ring.idx = (idx + 1) % kHistoryLen;
+    const float fmax = FMT == FP8_E4M3 ? kE4M3Max : kE5M2Max;
+    if (m > 0.0f && isfinite(m)) {
+      const float c = __fdiv_rn(fmax, m);
+      if (isfinite(c) && c > 0.0f) *ring.scale = c;
+    }
+    *ring.scale_inv = __frcp_rn(s_used);
+    atomicExch(&ring.scratch[1], 0u);
+  }
+}
+
+// ---- ROW layout --------------------------------------------------------------
+
+struct RowArgs {
+  const uint8_t* in;   // element 0
+  uint8_t* out;
+  int64_t n;           // elements
+  int64_t head;        // scalar elements before the first 16-byte aligned output byte
+  int64_t nchunks;     // 16-element chunks after the head
+  RingArgs ring;
+};
+
+template <int DT, int FMT, bool kAligned>
+__device__ __forceinline__ void row_chunk(const RowArgs& a, int64_t j, float s, float& amax) {
+  constexpr int kB = In<DT>::kBytes;
+  const int64_t e = a.head + 16 * j;
+  float v[16];
+  if constexpr (kAligned) load_vec_aligned<DT, 16>(a.in + e * kB, v);
+  else load_vec<DT, 16>(a.in + e * kB, v);
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t p0 = cvt_pair<FMT>(v[4 * i], v[4 * i + 1], s);
+    uint32_t p1 = cvt_pair<FMT>(v[4 * i + 2], v[4 * i + 3], s);
+    w[i] = p0 | (p1 << 16);
+  }
+#pragma unroll
+  for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  *reinterpret_cast<uint4*>(a.out + e) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+template <int DT, int FMT, bool kAligned>
+__global__ void __launch_bounds__(kThreads) quantize_row_kernel(const RowArgs a) {
+  constexpr int kB = In<DT>::kBytes;
+  const float s = *a.ring.scale;
+  float amax = 0.0f;
+  const int64_t tid = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+  const int64_t nthr = int64_t(gridDim.x) * kThreads;
+
+  // Head and tail (fewer than 16 elements each): one element per thread.
+  const int64_t tail0 = a.head + 16 * a.nchunks;
+  if (tid < a.head) {
+    const float x = load_one<DT>(a.in + tid * kB);
+    amax = fmaxf(amax, fabsf(x));
+    a.out[tid] = cvt_one<FMT>(x, s);
+  }
+  if (tid < a.n - tail0) {
+    const int64_t e = tail0 + tid;
+    const float x = load_one<DT>(a.in + e * kB);
+    amax = fmaxf(amax, fabsf(x));
+    a.out[e] = cvt_one<FMT>(x, s);
+  }
+
+  for (int64_t j = tid; j < a.nchunks; j += 2 * nthr) {
+    row_chunk<DT, FMT, kAligned>(a, j, s, amax);
+    if (j + nthr < a.nchunks) row_chunk<DT, FMT, kAligned>(a, j + nthr, s, amax);
+  }
+  amax_ticket_fold<FMT>(amax, a.ring, s);
+}
+
+// ---- T / DUAL layouts --------------------------------------------------------
+
+constexpr int kTileR = 128;  // input rows per tile
+constexpr int kTileC = 64;   // input columns per tile
+constexpr int kPitchW = kTileR / 4 + 1;  // shared tile pitch in words (33)
+
+struct TileArgs {
+  const uint8_t* in;
+  uint8_t* out;     // [rows, cols] (DUAL only)
+  uint8_t* out_t;   // [cols, rows]
+  int64_t rows, cols;
+  int64_t tiles_c, ntiles;
+  int out8;         // out rows start 8-byte aligned (base and cols % 8)
+  int outt4;        // out_t rows start 4-byte aligned (base and rows % 4)
+  RingArgs ring;
+};
+
+template <int DT, int FMT, bool kDual>
+__global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs a) {
+  constexpr int kB = In<DT>::kBytes;
+  __shared__ uint32_t sT[kTileC * kPitchW];
+  const float s = *a.ring.scale;
+  float amax = 0.0f;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lr0 = 32 * (warp & 3) + 4 * (lane & 7);  // first of this lane's 4 rows
+  const int lc0 = 32 * (warp >> 2) + 8 * (lane >> 3);  // first of its 8 columns
+
+  for (int64_t t = blockIdx.x; t < a.ntiles; t += gridDim.x) {
+    const int64_t r0 = (t / a.tiles_c) * kTileR;
+    const int64_t c0 = (t % a.tiles_c) * kTileC;
+    const bool interior = (r0 + kTileR <= a.rows) && (c0 + kTileC <= a.cols);
+    uint32_t q[4][2];  // 4 rows x 8 codes
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int64_t r = r0 + lr0 + i;
+      const int64_t c = c0 + lc0;
+      float v[8];
+      if (interior) {
+        load_vec<DT, 8>(a.in + (r * a.cols + c) * kB, v);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          v[j] = (r < a.rows && c + j < a.cols) ? load_one<DT>(a.in + (r * a.cols + c + j) * kB) : 0.0f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+      q[i][0] = cvt_pair<FMT>(v[0], v[1], s) | (cvt_pair<FMT>(v[2], v[3], s) << 16);
+      q[i][1] = cvt_pair<FMT>(v[4], v[5], s) | (cvt_pair<FMT>(v[6], v[7], s) << 16);
+      if constexpr (kDual) {
+        uint8_t* o = a.out + r * a.cols + c;
+        if (interior && a.out8) {
+          *reinterpret_cast<uint2*>(o) = make_uint2(q[i][0], q[i][1]);
+        } else if (r < a.rows) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c + j < a.cols) o[j] = uint8_t(q[i][j >> 2] >> (8 * (j & 3)));
+        }
+      }
+    }
+    __syncthreads();  // previous tile's readers are done with sT
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int sh = 8 * (j & 3);
+      const uint32_t w = ((q[0][j >> 2] >> sh) & 0xFFu) | (((q[1][j >> 2] >> sh) & 0xFFu) << 8) |
+                         (((q[2][j >> 2] >> sh) & 0xFFu) << 16) | (((q[3][j >> 2] >> sh) & 0xFFu) << 24);
+      sT[(lc0 + j) * kPitchW + (lr0 >> 2)] = w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kTileC / 8; ++k) {
+      const int cl = 8 * warp + k;
+      const int64_t c = c0 + cl;
+      const int64_t r = r0 + 4 * lane;
+      const uint32_t w = sT[cl * kPitchW + lane];
+      if (c < a.cols) {
+        uint8_t* o = a.out_t + c * a.rows + r;
+        if (a.outt4 && r + 4 <= a.rows) {
+          *reinterpret_cast<uint32_t*>(o) = w;
+        } else {
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            if (r + b < a.rows) o[b] = uint8_t(w >> (8 * b));
+        }
+      }
+    }
+  }
+  amax_ticket_fold<FMT>(amax, a.ring, s);
+}
+
+// ---- host side ---------------------------------------------------------------
+
+int sm_count_current() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  if (dev < 0 || dev >= 64) return -1;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int DT, int FMT>
+int launch_row(const RowArgs& a, int grid, cudaStream_t st, bool aligned) {
+  if (aligned) quantize_row_kernel<DT, FMT, true><<<grid, kThreads, 0, st>>>(a);
+  else quantize_row_kernel<DT, FMT, false><<<grid, kThreads, 0, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+template <int DT, int FMT>
+int launch_tile(const TileArgs& a, int grid, cudaStream_t st, bool dual) {
+  if (dual) quantize_tile_kernel<DT, FMT, true><<<grid, kThreads, 0, st>>>(a);
+  else quantize_tile_kernel<DT, FMT, false><<<grid, kThreads, 0, st>>>(a);
+  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+template <int DT>
+int dispatch_fmt_row(int fmt, const RowArgs& a, int grid, cudaStream_t st, bool aligned) {
+  return fmt == FP8_E4M3 ? launch_row<DT, FP8_E4M3>(a, grid, st, aligned)
+                         : launch_row<DT, FP8_E5M2>(a, grid, st, aligned);
+}
+
+template <int DT>
+int dispatch_fmt_tile(int fmt, const TileArgs& a, int grid, cudaStream_t st, bool dual) {
+  return fmt == FP8_E4M3 ? launch_tile<DT, FP8_E4M3>(a, grid, st, dual)
+                         : launch_tile<DT, FP8_E5M2>(a, grid, st, dual);
+}
+
+}  // namespace
+}  // namespace fp8ds
+
+using namespace fp8ds;
+
+extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
+                            fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream) {
+  if (dtype < FP8_IN_BF16 || dtype > FP8_IN_FP32) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (layout < FP8_LAYOUT_ROW || layout > FP8_LAYOUT_DUAL) return FP8_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0) return FP8_ERR_INVALID_ARG;
+  if (cols > 0 && rows > INT64_MAX / cols) return FP8_ERR_INVALID_ARG;
+  if (!ring.history || !ring.idx || !ring.scale || !ring.scale_inv || !ring.scratch) return FP8_ERR_INVALID_ARG;
+  const int64_t n = rows * cols;
+  if (n > 0 && in == nullptr) return FP8_ERR_INVALID_ARG;
+  if ((layout == FP8_LAYOUT_ROW || layout == FP8_LAYOUT_DUAL) && n > 0 && out == nullptr) return FP8_ERR_INVALID_ARG;
+  if ((layout == FP8_LAYOUT_T || layout == FP8_LAYOUT_DUAL) && n > 0 && out_t == nullptr) return FP8_ERR_INVALID_ARG;
+  const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
+  if (reinterpret_cast<uintptr_t>(in) % eb != 0) return FP8_ERR_UNSUPPORTED;
+
+  const int sms = sm_count_current();
+  if (sms <= 0) return FP8_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const RingArgs r{ring.history, ring.idx, ring.scale, ring.scale_inv, ring.scratch};
+  const int max_grid = sms * (2048 / kThreads);
+
+  if (layout == FP8_LAYOUT_ROW) {
+    RowArgs a{};
+    a.in = static_cast<const uint8_t*>(in);
+    a.out = out;
+    a.n = n;
+    const uintptr_t oa = reinterpret_cast<uintptr_t>(out);
+    a.head = std::min<int64_t>(n, int64_t((16 - (oa & 15)) & 15));
+    a.nchunks = (n - a.head) / 16;
+    a.ring = r;
+    const bool aligned = ((reinterpret_cast<uintptr_t>(in) + uintptr_t(a.head * eb)) & 15) == 0;
+    const int64_t want = (a.nchunks + 2 * kThreads - 1) / (2 * kThreads);
+    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(want, max_grid)));
+    switch (dtype) {
+      case FP8_IN_BF16: return dispatch_fmt_row<FP8_IN_BF16>(fmt, a, grid, st, aligned);
+      case FP8_IN_FP16: return dispatch_fmt_row<FP8_IN_FP16>(fmt, a, grid, st, aligned);
+      default: return dispatch_fmt_row<FP8_IN_FP32>(fmt, a, grid, st, aligned);
+    }
+  }
+
+  TileArgs a{};
+  a.in = static_cast<const uint8_t*>(in);
+  a.out = out;
+  a.out_t = out_t;
+  a.rows = rows;
+  a.cols = cols;
+  a.tiles_c = (cols + kTileC - 1) / kTileC;
+  a.ntiles = ((rows + kTileR - 1) / kTileR) * a.tiles_c;
+  a.out8 = (layout == FP8_LAYOUT_DUAL) && (reinterpret_cast<uintptr_t>(out) % 8 == 0) && (cols % 8 == 0);
+  a.outt4 = (reinterpret_cast<uintptr_t>(out_t) % 4 == 0) && (rows % 4 == 0);
+  a.ring = r;
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(a.ntiles, max_grid)));
+  const bool dual = layout == FP8_LAYOUT_DUAL;
+  switch (dtype) {
+    case FP8_IN_BF16: return dispatch_fmt_tile<FP8_IN_BF16>(fmt, a, grid, st, dual);
+    case FP8_IN_FP16: return dispatch_fmt_tile<FP8_IN_FP16>(fmt, a, grid, st, dual);
+    default: return dispatch_fmt_tile<FP8_IN_FP32>(fmt, a, grid, st, dual);
+  }
+}

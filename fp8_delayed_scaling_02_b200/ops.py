@@ -1,0 +1,197 @@
+"""Thin ctypes binding of the fp8ds C ABI (``include/fp8ds.h``).
+
+Argument marshalling only: every step of quantize_fp8 and mm_fp8 runs in the
+CUDA kernels of ``libfp8ds.so``.  There is no CPU fallback -- if the library
+is missing or no CUDA device is present the calls raise.  torch provides the
+device memory and the current stream.
+"""
+
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+E4M3, E5M2 = 0, 1
+ROW, TRANSPOSED, DUAL = 0, 1, 2
+IN_DTYPE = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
+MM_NT = 0
+MM_A_E5M2 = 1 << 8
+MM_B_E5M2 = 1 << 9
+HISTORY_LEN = 16
+
+FP8_OK = 0
+FP8_ERR_INVALID_ARG = -1
+FP8_ERR_UNSUPPORTED = -2
+FP8_ERR_CUDA = -3
+FP8_ERR_DEVICE_TIMEOUT = -4
+
+
+class CRing(ctypes.Structure):
+    """Mirror of ``fp8_ring``: five device pointers."""
+
+    _fields_ = [
+        ("history", ctypes.c_void_p),
+        ("idx", ctypes.c_void_p),
+        ("scale", ctypes.c_void_p),
+        ("scale_inv", ctypes.c_void_p),
+        ("scratch", ctypes.c_void_p),
+    ]
+
+
+_LIB = None
+
+
+def lib_path():
+    return _build.LIB
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        path = lib_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m fp8_delayed_scaling_02_b200.build` "
+                "(there is no CPU fallback)")
+        L = ctypes.CDLL(path)
+        vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+        L.fp8_quantize.argtypes = [vp, i32, i64, i64, i32, i32, CRing, vp, vp, vp]
+        L.fp8_quantize.restype = i32
+        L.fp8_mm.argtypes = [vp, vp, i64, i64, i64, i64, vp, i32, vp, vp, vp, vp, vp]
+        L.fp8_mm.restype = i32
+        L.fp8_status_string.argtypes = [i32]
+        L.fp8_status_string.restype = ctypes.c_char_p
+        L.fp8_device_error.argtypes = [i32, ctypes.POINTER(ctypes.c_uint32)]
+        L.fp8_device_error.restype = i32
+        L.fp8_device_info.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_char_p)]
+        L.fp8_device_info.restype = i32
+        _LIB = L
+    return _LIB
+
+
+class Fp8Error(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {lib().fp8_status_string(status).decode()} ({status})")
+
+
+def _check(rc, what):
+    if rc != FP8_OK:
+        raise Fp8Error(rc, what)
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+class Ring:
+    """One tensor's delayed-scaling state in a single device buffer.
+
+    Layout (32-bit words): history[0:16] | idx[16] | scale[17] | scale_inv[18] | scratch[19:21].
+    """
+
+    WORDS = 24
+
+    def __init__(self, device="cuda", scale=1.0):
+        self.buf = torch.zeros(self.WORDS, dtype=torch.int32, device=device)
+        f = self.buf.view(torch.float32)
+        f[17] = float(scale)
+        f[18] = 1.0
+
+    @property
+    def history(self):
+        return self.buf[0:HISTORY_LEN].view(torch.float32)
+
+    @property
+    def idx(self):
+        return self.buf[16:17]
+
+    @property
+    def scale(self):
+        return self.buf[17:18].view(torch.float32)
+
+    @property
+    def scale_inv(self):
+        return self.buf[18:19].view(torch.float32)
+
+    @property
+    def scratch(self):
+        return self.buf[19:21]
+
+    def c(self):
+        base = self.buf.data_ptr()
+        return CRing(base, base + 16 * 4, base + 17 * 4, base + 18 * 4, base + 19 * 4)
+
+    def state(self):
+        """Host copy: (history float32[16], idx, scale, scale_inv, scratch[2])."""
+        h = self.buf.cpu()
+        f = h.view(torch.float32)
+        return f[:16].clone(), int(h[16]), float(f[17]), float(f[18]), h[19:21].clone()
+
+
+def quantize(x, fmt, layout, ring, out=None, out_t=None, stream=None):
+    """fp8_quantize on a 2-D CUDA tensor ``x`` (bf16/fp16/fp32, contiguous).
+
+    Returns (out, out_t) as uint8 tensors (None where the layout has none).
+    """
+    if x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D tensor")
+    rows, cols = x.shape
+    if layout in (ROW, DUAL) and out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if layout in (TRANSPOSED, DUAL) and out_t is None:
+        out_t = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+    rc = lib().fp8_quantize(_ptr(x), IN_DTYPE[x.dtype], rows, cols, layout, fmt, ring.c(),
+                            _ptr(out if layout in (ROW, DUAL) else None),
+                            _ptr(out_t if layout in (TRANSPOSED, DUAL) else None), _stream(stream))
+    _check(rc, "fp8_quantize")
+    return (out if layout in (ROW, DUAL) else None), (out_t if layout in (TRANSPOSED, DUAL) else None)
+
+
+def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream=None):
+    """fp8_mm: Y = bf16(a . b^T * sinv_a * sinv_b + bias).
+
+    a: uint8 [M, K] or [Ba, M, K]; b: uint8 [N, K] or [Bb, N, K] (K contiguous);
+    a size-1 (or 2-D) operand broadcasts over the batch at stride 0.
+    sinv_a / sinv_b: one-element float32 CUDA tensors.  bias: float32 [N] or None.
+    """
+    if a.dtype != torch.uint8 or b.dtype != torch.uint8:
+        raise ValueError("a and b hold FP8 codes as uint8")
+    a3 = a if a.dim() == 3 else a.unsqueeze(0)
+    b3 = b if b.dim() == 3 else b.unsqueeze(0)
+    batch = max(a3.shape[0], b3.shape[0])
+    M, K = a3.shape[1], a3.shape[2]
+    N = b3.shape[1]
+    if b3.shape[2] != K:
+        raise ValueError("K mismatch")
+    for t, n in ((a3, M * K), (b3, N * K)):
+        if t.shape[0] not in (1, batch) or (K > 0 and t.shape[1] > 1 and (t.stride(2) != 1 or t.stride(1) != K)):
+            raise ValueError("operands must be K-contiguous with matching batch")
+    sa = 0 if a3.shape[0] == 1 else a3.stride(0)
+    sb = 0 if b3.shape[0] == 1 else b3.stride(0)
+    squeeze = a.dim() == 2 and b.dim() == 2
+    if out is None:
+        out = torch.empty((batch, M, N), dtype=torch.bfloat16, device=a.device)
+    out3 = out if out.dim() == 3 else out.unsqueeze(0)
+    strides = (ctypes.c_int64 * 3)(sa, sb, out3.stride(0) if batch > 1 else M * N)
+    layout = MM_NT | (MM_A_E5M2 if fmt_a == E5M2 else 0) | (MM_B_E5M2 if fmt_b == E5M2 else 0)
+    rc = lib().fp8_mm(_ptr(a3), _ptr(b3), M, N, K, batch, strides, layout, _ptr(sinv_a), _ptr(sinv_b),
+                      _ptr(bias), _ptr(out3), _stream(stream))
+    _check(rc, "fp8_mm")
+    return out3[0] if squeeze and out.dim() == 3 else out
+
+
+def device_error(clear=True):
+    """(status, site) of the library's device error word; synchronises the device."""
+    where = ctypes.c_uint32(0)
+    rc = lib().fp8_device_error(1 if clear else 0, ctypes.byref(where))
+    return rc, where.value

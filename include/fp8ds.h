@@ -1,0 +1,163 @@
+/*
+ * fp8ds.h -- C ABI of the B200 (sm_100a) FP8 per-tensor delayed-scaling linear.
+ *
+ * Two operations, both asynchronous on the caller's CUDA stream:
+ *
+ *   fp8_quantize  cast a bf16/fp16/fp32 tensor to E4M3 or E5M2 with the scale
+ *                 held in a delayed-scaling ring, reduce amax over the raw
+ *                 values, and fold that amax into the ring in the same kernel.
+ *   fp8_mm        Y = bf16(sinv_a * sinv_b * A.B^T + bias), A and B FP8 with K
+ *                 contiguous ("NT"), fp32 accumulation, optional fp32 bias,
+ *                 optional batch with stride-0 broadcast.
+ *
+ * Sources: the AstrAI commit-log pages "AstrAI commits, branch main,
+ * tests/extension" (ring commit, quantize split commit, snapshot commit,
+ * bias-fusion commit, 3D batched commit), "AstrAI commit 05463316
+ * csrc/kernels/fp8/quantize.cuh" (transposed/dual quantize), and "AstrAI
+ * commit 0d0dc648 csrc/kernels/fp8_mm.cu" (amax over raw values, te-style
+ * 16-step history ring).
+ *
+ * Conventions for every entry point:
+ *   - Every pointer argument is device memory owned by the caller, unless the
+ *     comment says "host".  The library allocates no device memory, never
+ *     synchronises the device, and returns as soon as the work is enqueued.
+ *   - The return value is FP8_OK (0) or a negative fp8_status.  On an error
+ *     nothing was launched unless the status is FP8_ERR_CUDA.
+ *   - Kernel-side faults are never raised on purpose: every wait in a kernel
+ *     is bounded; a wait that runs out records FP8_ERR_DEVICE_TIMEOUT in a
+ *     library-global error word that fp8_device_error() reads.
+ */
+#ifndef FP8DS_H_
+#define FP8DS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle as cudaStream_t; 0 is the legacy default stream. */
+typedef struct CUstream_st* fp8_stream_t;
+
+typedef enum {
+  FP8_OK = 0,
+  FP8_ERR_INVALID_ARG = -1,    /* bad enum, negative size, missing pointer      */
+  FP8_ERR_UNSUPPORTED = -2,    /* valid request outside what the kernels take  */
+  FP8_ERR_CUDA = -3,           /* a CUDA runtime/driver call failed             */
+  FP8_ERR_DEVICE_TIMEOUT = -4  /* a bounded in-kernel wait ran out              */
+} fp8_status;
+
+/* Input element type of fp8_quantize. */
+typedef enum { FP8_IN_BF16 = 0, FP8_IN_FP16 = 1, FP8_IN_FP32 = 2 } fp8_in_dtype;
+
+/* FP8 format: E4M3 (largest finite 448) for activations and weights, E5M2
+ * (largest finite 57344) for gradients -- the te-style recipe of the
+ * "AstrAI commit 5244f1a8" entry on the fp8_mm.cu page. */
+typedef enum { FP8_E4M3 = 0, FP8_E5M2 = 1 } fp8_fmt;
+
+/* QuantLayout of the quantize bindings commit ("tests/extension" page):
+ * ROW writes out[r*cols + c]; T writes out_t[c*rows + r] (the [cols, rows]
+ * transpose); DUAL writes both from a single read of the input. */
+typedef enum { FP8_LAYOUT_ROW = 0, FP8_LAYOUT_T = 1, FP8_LAYOUT_DUAL = 2 } fp8_qlayout;
+
+/* History ring of one tensor (x, w or g each own one), the "[hist | scale |
+ * counter]" buffer of the ring commit.  All five pointers are device memory,
+ * usually slices of one caller-owned buffer.  Before the first call the
+ * caller sets history to 0, idx to 0, scale to the initial scale (1.0),
+ * scale_inv to 1.0 and scratch to 0; the kernel keeps them consistent after
+ * that.  A ring must not be used by two quantize calls that may run at the
+ * same time. */
+typedef struct {
+  float* history;     /* [16] amax of the last 16 calls, float32               */
+  int32_t* idx;       /* [1]  slot the next amax is written to, 0..15          */
+  float* scale;       /* [1]  scale the NEXT call multiplies by (published     */
+                      /*      by the last block of each call)                  */
+  float* scale_inv;   /* [1]  1/scale that the MOST RECENT call used: the      */
+                      /*      dequantisation factor to hand to fp8_mm          */
+  uint32_t* scratch;  /* [2]  amax bits and block ticket; zero between calls   */
+} fp8_ring;
+
+/*
+ * fp8_quantize -- delayed-scaling cast to FP8 with in-kernel ring fold.
+ *
+ * Computes, with s = *ring.scale read at launch:
+ *   q[r,c]  = saturate_rne_fp8(fp32(x[r,c]) * s)       (one fp32 multiply)
+ *   amax    = max |x[r,c]| over the raw values (NaN ignored), the fix of
+ *             "AstrAI commit 69f35c46" (amax of raw, not scaled, values)
+ *   then, in the last block to finish (atomic ticket + fences, ring commit):
+ *   history[idx] = amax; idx = (idx + 1) % 16; m = max(history);
+ *   *scale = FP8_MAX / m (fp32, round-to-nearest) when m > 0 and finite and
+ *            the quotient is finite, otherwise unchanged;
+ *   *scale_inv = 1 / s  (the inverse of the scale this call used, as the
+ *            snapshot commit requires for the GEMM's dequantisation).
+ *
+ * in      [rows, cols] row-major, contiguous, element type `dtype`; any
+ *         address aligned to the element size (e.g. a 2-byte offset for bf16).
+ * layout  fp8_qlayout; out is [rows, cols] uint8 (ROW, DUAL), out_t is
+ *         [cols, rows] uint8 (T, DUAL); the unused one may be NULL.
+ * rows, cols >= 0; rows*cols == 0 still folds amax = 0 into the ring.
+ * Errors: FP8_ERR_INVALID_ARG for a bad enum, a negative size, a NULL ring
+ *         field, a NULL in with rows*cols > 0, or a NULL out/out_t the
+ *         layout needs; FP8_ERR_UNSUPPORTED for an input address not aligned
+ *         to its element size; FP8_ERR_CUDA if the launch fails.
+ */
+int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
+                 fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);
+
+/* fp8_mm layout word: FP8_MM_NT plus the operand format bits.  NT means A is
+ * [M, K] and B is [N, K], both with K contiguous. */
+#define FP8_MM_NT 0
+#define FP8_MM_A_E5M2 (1 << 8) /* A holds E5M2 codes (default E4M3) */
+#define FP8_MM_B_E5M2 (1 << 9) /* B holds E5M2 codes (default E4M3) */
+
+/*
+ * fp8_mm -- scaled FP8 GEMM with fused scale, bias and bf16 rounding.
+ *
+ * For b in [0, batch), m in [0, M), n in [0, N):
+ *   Y[b,m,n] = bf16_rne( fp32_acc(sum_k A[b,m,k] * B[b,n,k]) * (sinv_a*sinv_b)
+ *                        + bias[n] )
+ * (bias-fusion commit: the fp32 bias is added before the single bf16
+ * rounding; 3D batched commit: size-1 batches broadcast with stride 0).
+ *
+ * A       uint8 FP8 codes, element (b,m,k) at A[b*strides[0] + m*K + k].
+ * B       uint8 FP8 codes, element (b,n,k) at B[b*strides[1] + n*K + k].
+ * out_bf16 bfloat16 (uint16 storage), element (b,m,n) at
+ *         out_bf16[b*strides[2] + m*N + n].
+ * strides host array of 3 int64 batch strides in elements; may be NULL when
+ *         batch == 1.  0 broadcasts that operand over the batch.
+ * sinv_a, sinv_b  device pointers to one float each (typically a ring's
+ *         scale_inv), read on the device so the scale chain never visits
+ *         the host.
+ * bias    device pointer to N floats, or NULL for no bias.
+ * M, N >= 0, batch >= 1; M*N == 0 is a no-op.  K >= 0 and K % 16 == 0
+ *         (the TMA row pitch must be a multiple of 16 bytes); K == 0 gives
+ *         Y = bf16(bias) (or 0).
+ * Errors: FP8_ERR_INVALID_ARG (negative size, batch < 1, NULL A/B/out/sinv,
+ *         unknown layout bits, NULL strides with batch > 1);
+ *         FP8_ERR_UNSUPPORTED (K % 16 != 0, A/B/stride not 16-byte aligned,
+ *         out_bf16 not 2-byte aligned, a dimension beyond 2^31);
+ *         FP8_ERR_CUDA (descriptor encoding or launch failed).
+ */
+int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+           const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b,
+           const float* bias, uint16_t* out_bf16, fp8_stream_t stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fp8_status_string(int status);
+
+/* Reads, and with clear != 0 resets, the library's device error word on the
+ * current device.  Synchronises the device.  Returns FP8_OK when no bounded
+ * wait has run out since the last clear, FP8_ERR_DEVICE_TIMEOUT when one has
+ * (then *where_out, if not NULL, receives a code naming the wait), or
+ * FP8_ERR_CUDA. */
+int fp8_device_error(int clear, uint32_t* where_out);
+
+/* Number of SMs and the library's build architecture string, for reports. */
+int fp8_device_info(int* sm_count, const char** arch);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8DS_H_ */

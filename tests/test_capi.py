@@ -1,0 +1,90 @@
+"""CPU checks of the C ABI: the library loads, exports every declared symbol,
+and rejects bad arguments on the host before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp8_delayed_scaling_02_b200 import build, ops
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fp8ds.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return ops.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp8_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    assert declared_functions() == sorted(
+        ["fp8_quantize", "fp8_mm", "fp8_status_string", "fp8_device_error", "fp8_device_info"])
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code in (0, -1, -2, -3, -4, 7):
+        s = L.fp8_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+    assert L.fp8_status_string(-4).startswith(b"FP8_ERR_DEVICE_TIMEOUT")
+
+
+def _ring(addr=0x1000):
+    return ops.CRing(addr, addr + 64, addr + 68, addr + 72, addr + 76)
+
+
+def _q(L, dtype=0, rows=4, cols=4, layout=0, fmt=0, ring=None, out=0x2000, out_t=0x3000, inp=0x4000):
+    return L.fp8_quantize(ctypes.c_void_p(inp), dtype, rows, cols, layout, fmt, ring or _ring(),
+                          ctypes.c_void_p(out), ctypes.c_void_p(out_t), None)
+
+
+def test_quantize_rejects_bad_arguments_without_cuda(L):
+    assert _q(L, dtype=3) == ops.FP8_ERR_INVALID_ARG
+    assert _q(L, fmt=2) == ops.FP8_ERR_INVALID_ARG
+    assert _q(L, layout=3) == ops.FP8_ERR_INVALID_ARG
+    assert _q(L, rows=-1) == ops.FP8_ERR_INVALID_ARG
+    assert _q(L, ring=ops.CRing(0, 0, 0, 0, 0)) == ops.FP8_ERR_INVALID_ARG
+    assert _q(L, inp=0) == ops.FP8_ERR_INVALID_ARG
+    assert _q(L, layout=0, out=0) == ops.FP8_ERR_INVALID_ARG
+    assert _q(L, layout=1, out_t=0) == ops.FP8_ERR_INVALID_ARG
+    assert _q(L, layout=2, out_t=0) == ops.FP8_ERR_INVALID_ARG
+    assert _q(L, dtype=2, inp=0x4002) == ops.FP8_ERR_UNSUPPORTED   # fp32 needs 4-byte alignment
+    assert _q(L, dtype=0, inp=0x4001) == ops.FP8_ERR_UNSUPPORTED   # bf16 needs 2-byte alignment
+
+
+def _mm(L, M=128, N=128, K=128, batch=1, strides=None, layout=0, A=0x10000, B=0x20000, out=0x30000,
+        sa=0x40000, sb=0x40010):
+    st = (ctypes.c_int64 * 3)(*strides) if strides is not None else None
+    return L.fp8_mm(ctypes.c_void_p(A), ctypes.c_void_p(B), M, N, K, batch, st, layout, ctypes.c_void_p(sa),
+                    ctypes.c_void_p(sb), None, ctypes.c_void_p(out), None)
+
+
+def test_mm_rejects_bad_arguments_without_cuda(L):
+    assert _mm(L, M=-1) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, batch=0) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, layout=1) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, layout=1 << 10) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, batch=2, strides=None) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, batch=2, strides=(-16, 0, 0)) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, out=0) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, sa=0) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, A=0) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, K=24) == ops.FP8_ERR_UNSUPPORTED
+    assert _mm(L, out=0x30001) == ops.FP8_ERR_UNSUPPORTED
+    assert _mm(L, A=0x10008) == ops.FP8_ERR_UNSUPPORTED
+    assert _mm(L, batch=2, strides=(8, 0, 0)) == ops.FP8_ERR_UNSUPPORTED
+    # Empty products are a no-op that needs no device.
+    assert _mm(L, M=0) == ops.FP8_OK
+    assert _mm(L, N=0, A=0, B=0) == ops.FP8_OK

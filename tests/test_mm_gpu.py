@@ -1,0 +1,134 @@
+"""GPU parity of fp8_mm against the float64 oracle: |y - ref| <= ulp_bf16(ref) + 2^-20 sum|ab| sinv_a sinv_b."""
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_delayed_scaling_02_b200 import ops, synthetic as S
+from gpu_helpers import OG, OR, mm_check, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _scalar(v):
+    return torch.tensor([v], dtype=torch.float32, device="cuda")
+
+
+def _run(M, N, K, fmt_a=ops.E4M3, fmt_b=ops.E4M3, sa=1.0, sb=1.0, with_bias=False, seed=0, rows=None):
+    a = S.fp8_codes((M, K), seed=seed, fmt=fmt_a)
+    b = S.fp8_codes((N, K), seed=seed + 1, fmt=fmt_b)
+    bias = S.uniform((N,), seed=seed + 2) if with_bias else None
+    y = ops.mm(a.cuda(), b.cuda(), _scalar(sa), _scalar(sb), bias.cuda() if bias is not None else None,
+               fmt_a=fmt_a, fmt_b=fmt_b)
+    torch.cuda.synchronize()
+    assert y.shape == (M, N) and y.dtype == torch.bfloat16
+    return mm_check(y, a.numpy(), b.numpy(), fmt_a, fmt_b, np.float32(sa), np.float32(sb),
+                    bias.numpy() if bias is not None else None, rows)
+
+
+# Ragged and tiny shapes: M/N tails inside a 128 x BN tile, K tails inside a
+# 128-byte stage, several tiles in every dimension.
+@pytest.mark.parametrize("M,N,K", [(1, 1, 16), (5, 7, 48), (128, 128, 128), (200, 300, 160), (130, 129, 4096),
+                                   (257, 513, 272), (384, 1024, 640)])
+@pytest.mark.parametrize("with_bias", [False, True])
+def test_small_and_ragged(M, N, K, with_bias):
+    _run(M, N, K, with_bias=with_bias, sa=0.37, sb=0.125, seed=M + N + K)
+
+
+@pytest.mark.parametrize("fa,fb", [(ops.E5M2, ops.E4M3), (ops.E4M3, ops.E5M2), (ops.E5M2, ops.E5M2)])
+def test_mixed_formats(fa, fb):
+    _run(256, 384, 512, fmt_a=fa, fmt_b=fb, with_bias=True, sa=2.0 ** -10, sb=3.5)
+
+
+# Square sweep; full comparison up to 2048^3, sampled rows above.
+@pytest.mark.parametrize("n", [512, 1024, 1152, 2048, 3072, 4096, 8192])
+def test_square_sweep(n):
+    rows = None if n <= 2048 else np.unique(np.random.default_rng(n).integers(0, n, 24))
+    _run(n, n, n, with_bias=(n % 3 == 0 or n == 1024), seed=n, rows=rows)
+
+
+def test_square_8192_scaled_with_bias():
+    rows = np.array([0, 1, 127, 128, 4095, 8191])
+    _run(8192, 8192, 8192, sa=0.37, sb=0.125, with_bias=True, seed=5, rows=rows)
+
+
+def test_skinny_and_odd():
+    _run(64, 8192, 2048, seed=11)
+    _run(1024, 1536, 2048, seed=12)
+    _run(1000, 1537, 2048, with_bias=True, seed=13)
+
+
+def _quantized_normal(shape, seed):
+    """N(0,1) fp32 quantized E4M3 per tensor through fp8_quantize (second call uses 448/amax)."""
+    x = S.normal_with_outliers(shape, seed=seed, dtype="fp32").cuda()
+    ring = ops.Ring()
+    flat = x.reshape(-1, shape[-1])
+    ops.quantize(flat, ops.E4M3, ops.ROW, ring)
+    q, _ = ops.quantize(flat, ops.E4M3, ops.ROW, ring)
+    return q.view(shape), ring.scale_inv.clone()
+
+
+def test_batched_and_broadcast():
+    # 64 x (512^3), both operands batched.
+    a, sa = _quantized_normal((64, 512, 512), 21)
+    b, sb = _quantized_normal((64, 512, 512), 22)
+    y = ops.mm(a, b, sa, sb)
+    torch.cuda.synchronize()
+    assert y.shape == (64, 512, 512)
+    ref, Ssum = OG.mm_fp8(a.cpu().numpy(), b.cpu().numpy(), 0, 0, sa.item(), sb.item())
+    ok, ratio = OG.check(y.float().cpu().numpy(), ref, Ssum)
+    assert ok, ratio
+    # 8 x (1024 x 2048 x 2048) with a size-1 B batch broadcast at stride 0, bias.
+    a, sa = _quantized_normal((8, 1024, 2048), 23)
+    b, sb = _quantized_normal((1, 2048, 2048), 24)
+    bias = S.uniform((2048,), seed=25)
+    y = ops.mm(a, b, sa, sb, bias.cuda())
+    torch.cuda.synchronize()
+    assert y.shape == (8, 1024, 2048)
+    rows = np.array([0, 5, 511, 1023])
+    for z in (0, 3, 7):
+        ref, Ssum = OG.mm_fp8_rows(a[z].cpu().numpy(), b[0].cpu().numpy(), 0, 0, sa.item(), sb.item(),
+                                   bias.numpy(), rows)
+        ok, ratio = OG.check(y[z].float().cpu().numpy()[rows], ref, Ssum)
+        assert ok, (z, ratio)
+
+
+def test_k_zero_gives_bias_and_empty_is_noop():
+    bias = S.uniform((37,), seed=3).cuda()
+    a = torch.zeros((5, 0), dtype=torch.uint8, device="cuda")
+    b = torch.zeros((37, 0), dtype=torch.uint8, device="cuda")
+    y = ops.mm(a, b, _scalar(1.0), _scalar(1.0), bias)
+    torch.cuda.synchronize()
+    assert torch.equal(y.float().cpu(), bias.cpu().to(torch.bfloat16).float().expand(5, 37))
+    e = ops.mm(torch.zeros((0, 32), dtype=torch.uint8, device="cuda"),
+               torch.zeros((4, 32), dtype=torch.uint8, device="cuda"), _scalar(1.0), _scalar(1.0))
+    assert e.shape == (0, 4)
+
+
+def test_pr1_linear_end_to_end():
+    """Quantize X (row) and W (dual) through their rings for 3 steps, then
+    Y = Xq . Wq^T * sinv_x * sinv_w + bias with the scale_inv the quantize used."""
+    rx, rw = ops.Ring(), ops.Ring()
+    ox, ow = OR.Ring(), OR.Ring()
+    for step in range(3):
+        x, w, bias = S.linear_pr1_step(step)
+        xq, _ = ops.quantize(x.cuda(), ops.E4M3, ops.ROW, rx)
+        wq, wq_t = ops.quantize(w.cuda(), ops.E4M3, ops.DUAL, rw)
+        y = ops.mm(xq, wq, rx.scale_inv, rw.scale_inv, bias.cuda())
+        torch.cuda.synchronize()
+        rxq, _, _ = OR.quantize(x, 0, OR.ROW, ox)
+        rwq, _, _ = OR.quantize(w, 0, OR.DUAL, ow)
+        assert np.array_equal(xq.cpu().numpy(), rxq) and np.array_equal(wq.cpu().numpy(), rwq)
+        ref, Ssum = OG.mm_fp8(rxq, rwq, 0, 0, ox.scale_inv, ow.scale_inv, bias.numpy())
+        ok, ratio = OG.check(y.float().cpu().numpy(), ref, Ssum)
+        assert ok, (step, ratio)
+
+
+def test_device_error_word_clear():
+    rc, where = ops.device_error(clear=True)
+    assert rc == ops.FP8_OK and where == 0

@@ -1,0 +1,122 @@
+"""GPU parity of fp8_quantize against the CPU oracle: bytes, amax, ring and scales bit-exact."""
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_delayed_scaling_02_b200 import ops, synthetic as S
+from gpu_helpers import OR, assert_bytes_equal, assert_ring_equal, quantize_both, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+DTYPES = ["bf16", "fp16", "fp32"]
+FMTS = [ops.E4M3, ops.E5M2]
+LAYOUTS = [ops.ROW, ops.TRANSPOSED, ops.DUAL]
+
+
+@pytest.fixture(autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _run_and_compare(x, fmt, layout, ring, misalign=False):
+    out, out_t, r_out, r_out_t, r_ring = quantize_both(x, fmt, layout, ring, misalign)
+    if layout in (ops.ROW, ops.DUAL):
+        assert_bytes_equal(out, r_out, "out")
+    if layout in (ops.TRANSPOSED, ops.DUAL):
+        assert_bytes_equal(out_t, r_out_t, "out_t")
+    assert_ring_equal(ring, r_ring)
+
+
+# Small shapes that span several 128x64 tiles and 16-element chunks and leave
+# ragged tails in both dimensions, plus rows not a multiple of 4.
+SMALL = [(1, 1), (3, 5), (7, 33), (130, 70), (301, 1537)]
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("layout", LAYOUTS)
+@pytest.mark.parametrize("misalign", [False, True])
+def test_small_shapes_two_calls(dtype, fmt, layout, misalign):
+    for i, (r, c) in enumerate(SMALL):
+        vs = [1.0, 1e-3, 1e3][i % 3]
+        ring = ops.Ring()
+        for step in range(2):  # second call uses the delayed scale published by the first
+            x = S.quant_sweep_input(r, c, dtype, vs, seed=31 * i + step)
+            _run_and_compare(x, fmt, layout, ring, misalign)
+
+
+def test_pr1_linear_three_delayed_steps():
+    """X [128,512] row and W [256,512] dual, E4M3, rings carried over 3 steps."""
+    rx, rw = ops.Ring(), ops.Ring()
+    for step in range(3):
+        x, w, _ = S.linear_pr1_step(step)
+        _run_and_compare(x, ops.E4M3, ops.ROW, rx)
+        _run_and_compare(w, ops.E4M3, ops.DUAL, rw)
+    assert ops.Ring().state()[2] == 1.0
+
+
+def test_seventeen_steps_wrap_the_ring():
+    ring = ops.Ring()
+    for step in range(17):
+        x = S.quant_sweep_input(64, 48, "bf16", 10.0 ** ((step % 5) - 2), seed=step)
+        _run_and_compare(x, ops.E5M2, ops.ROW, ring)
+
+
+def test_empty_and_zero_inputs_fold_the_ring():
+    ring = ops.Ring(scale=0.5)
+    for layout in LAYOUTS:
+        x = torch.zeros((0, 9), dtype=torch.bfloat16)
+        _run_and_compare(x, ops.E4M3, layout, ring)
+    x = torch.zeros((5, 9), dtype=torch.float32)
+    _run_and_compare(x, ops.E4M3, ops.DUAL, ring)
+    assert ring.state()[2] == 0.5  # zero history keeps the scale
+
+
+def test_saturation_and_specials():
+    vals = torch.tensor([[0.0, -0.0, 1e-30, -1e-30, 480.0, -1e6, 65504.0, 3e38, float("inf"), -float("inf")]],
+                        dtype=torch.float32)
+    for fmt in FMTS:
+        for layout in LAYOUTS:
+            ring = ops.Ring()
+            _run_and_compare(vals, fmt, layout, ring)
+
+
+# Full sizes of the quantize bandwidth sweep, in the launch configuration the
+# bench times; bytes compared on sampled rows, amax / ring / scales in full.
+FULL = [(128, 1536), (2048, 1536), (8192, 1536), (16384, 4096), (2048, 1537), (8192, 1537)]
+
+
+@pytest.mark.parametrize("shape", FULL)
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_full_size_sampled(shape, layout):
+    rows, cols = shape
+    rng = np.random.default_rng(rows + cols + layout)
+    sample = np.unique(np.concatenate([rng.integers(0, rows, 24), [0, rows - 1]]))
+    for dtype, fmt, misalign, vs in (("bf16", ops.E4M3, False, 1.0), ("fp32", ops.E5M2, True, 1e3),
+                                     ("fp16", ops.E4M3, True, 1e-3)):
+        x = S.quant_sweep_input(rows, cols, dtype, vs, seed=rows ^ cols)
+        ring = ops.Ring()
+        for step in range(2):
+            ref_ring = OR.Ring()
+            hist, idx, sc, si, _ = ring.state()
+            ref_ring.history, ref_ring.idx = hist.numpy().astype(np.float32), idx
+            ref_ring.scale, ref_ring.scale_inv = np.float32(sc), np.float32(si)
+            if misalign:
+                flat = torch.empty(x.numel() + 1, dtype=x.dtype, device="cuda")
+                flat[1:].copy_(x.reshape(-1))
+                xd = flat[1:].view(x.shape)
+            else:
+                xd = x.cuda()
+            out, out_t = ops.quantize(xd, fmt, layout, ring)
+            torch.cuda.synchronize()
+            xf = OR.to_float32(x)
+            s_used = np.float32(ref_ring.scale)
+            ref_rows = OR.scaled_codes(xf[sample], s_used, fmt)
+            OR.fold(ref_ring, OR.amax(xf), fmt)
+            if out is not None:
+                assert_bytes_equal(out[torch.as_tensor(sample, device="cuda")], ref_rows, "out rows")
+            if out_t is not None:
+                assert_bytes_equal(out_t[:, torch.as_tensor(sample, device="cuda")].t().contiguous(), ref_rows,
+                                   "out_t columns")
+            assert_ring_equal(ring, ref_ring)

@@ -465,3 +465,64 @@ extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t col
     default: return dispatch_fmt_tile<FP8_IN_FP32>(fmt, a, grid, st, dual);
   }
 }
+
+// ---- variant for callers that cannot allocate --------------------------------
+//
+// Some callers cannot allocate device memory when they call us: operator or
+// plugin interfaces that hand over only input and output pointers, and
+// deployments that reserve all device memory at start-up (a cudaMalloc at run
+// time can also synchronise the device and stall other streams).  For them
+// fp8_quantize_static_scratch keeps the two scratch words that fp8_quantize
+// takes from ring.scratch (the amax bits and the block ticket) in the
+// library-owned array below instead.  Each GPU that loads the library holds
+// these 256 bytes until the process exits.  All calls on a device share the
+// array, so calls that overlap on the GPU race with each other.
+
+#include <mutex>
+
+static __device__ __align__(256) uint32_t g_quantize_static_scratch[64];
+
+namespace {
+constexpr int kStaticScratchWords = 64;    // capacity of g_quantize_static_scratch
+constexpr int kQuantizeScratchWords = 2;   // what one quantize call needs, whatever its size
+
+std::mutex g_static_scratch_mu;
+uint32_t* g_static_scratch_ptr[64] = {nullptr};
+
+// Device address of the static array on the current device, looked up once per
+// device with that device current.  Host code must not use the symbol itself:
+// on the host it is only a stand-in, not a device address.
+uint32_t* static_scratch_on_current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+  if (g_static_scratch_ptr[dev] == nullptr) {
+    uint32_t* p = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&p), g_quantize_static_scratch) != cudaSuccess) return nullptr;
+    g_static_scratch_ptr[dev] = p;
+  }
+  return g_static_scratch_ptr[dev];
+}
+}  // namespace
+
+extern "C" int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t cols, int layout,
+                                           int fmt, fp8_ring ring, uint8_t* out, uint8_t* out_t,
+                                           fp8_stream_t stream) {
+  if (kQuantizeScratchWords > kStaticScratchWords) return FP8_ERR_UNSUPPORTED;
+  // The argument checks that need no device run first, so a rejected call
+  // enqueues nothing.
+  if (dtype < FP8_IN_BF16 || dtype > FP8_IN_FP32) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (layout < FP8_LAYOUT_ROW || layout > FP8_LAYOUT_DUAL) return FP8_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0) return FP8_ERR_INVALID_ARG;
+  if (!ring.history || !ring.idx || !ring.scale || !ring.scale_inv) return FP8_ERR_INVALID_ARG;
+  uint32_t* scratch = static_scratch_on_current_device();
+  if (scratch == nullptr) return FP8_ERR_CUDA;
+  // The kernel leaves both words at zero when it finishes; clearing them here
+  // as well means a call never depends on what an earlier call left behind.
+  if (cudaMemsetAsync(scratch, 0, kQuantizeScratchWords * sizeof(uint32_t),
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FP8_ERR_CUDA;
+  ring.scratch = scratch;
+  return fp8_quantize(in, dtype, rows, cols, layout, fmt, ring, out, out_t, stream);
+}

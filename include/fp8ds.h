@@ -105,6 +105,35 @@ typedef struct {
 int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
                  fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);
 
+/*
+ * fp8_quantize_static_scratch -- fp8_quantize for callers that cannot allocate.
+ *
+ * The paper has no counterpart; this entry point exists for callers that
+ * cannot allocate device memory at call time, such as operator or plugin
+ * interfaces that receive only input and output pointers, or deployments that
+ * reserve all device memory at start-up.  It computes exactly what
+ * fp8_quantize computes, with the same arguments, except that ring.scratch is
+ * ignored (it may be NULL): the two scratch words (amax bits and block
+ * ticket) live in a 256-byte array owned by the library, which every GPU that
+ * loads the library holds until the process exits.  The call itself allocates
+ * nothing.
+ *
+ *   - The array holds 64 words; a call needs 2, whatever rows*cols is, so no
+ *     tensor is refused for lack of scratch.  A request needing more than the
+ *     array holds would return FP8_ERR_UNSUPPORTED.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.
+ *   - All calls on a device share the array.  Each call clears the two words
+ *     on `stream` before its kernel, and the kernel leaves them at zero, but
+ *     two calls that overlap on the GPU (different streams, no ordering
+ *     between them) race on the array and give wrong amax and scales.
+ *   - Errors are those of fp8_quantize, plus FP8_ERR_CUDA if the array's
+ *     address cannot be obtained or the clearing memset fails.
+ */
+int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
+                                fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);
+
 /* fp8_mm layout word: FP8_MM_NT plus the operand format bits.  NT means A is
  * [M, K] and B is [N, K], both with K contiguous. */
 #define FP8_MM_NT 0

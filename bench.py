@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--M", type=int, default=8192)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", choices=["gemm", "quantize"], default=None,
+                    help="per-shape kernel rows instead of the step line")
+    ap.add_argument("--iters", type=int, default=50)
+    ap.add_argument("--shapes", default=None, help="sweep subset, e.g. 8192x8192x8192,64x8192x2048")
     return ap.parse_args()
 
 
@@ -232,10 +236,82 @@ def cpu_baseline(M_full, seconds=12.0):
                       f"{reps} repetitions in {el:.1f} s; numpy float64 oracle"}
 
 
+# ------------------------------------------------------------------ sweeps ----
+
+GEMM_SHAPES = [(1, n, n, n) for n in (512, 1024, 1152, 2048, 3072, 4096, 8192)] + [
+    (1, 64, 8192, 2048), (1, 1024, 1536, 2048), (1, 1000, 1537, 2048), (64, 512, 512, 512), (8, 1024, 2048, 2048)]
+QUANT_SHAPES = [(128, 1536), (2048, 1536), (8192, 1536), (16384, 4096), (2048, 1537), (8192, 1537)]
+
+
+def _median_ms(fn, torch, iters, flush=None):
+    st = torch.cuda.current_stream()
+    times = []
+    for _ in range(iters):
+        if flush is not None:
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        fn()
+        b.record(st)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+def sweep(args):
+    import torch
+
+    from fp8_delayed_scaling_02_b200 import build as B
+    from fp8_delayed_scaling_02_b200 import ops, synthetic as S
+
+    B.build()
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    want = None
+    if args.shapes:
+        want = [tuple(int(v) for v in s.split("x")) for s in args.shapes.split(",")]
+    if args.sweep == "gemm":
+        shapes = GEMM_SHAPES if not want else [w if len(w) == 4 else (1,) + w for w in want]
+        for bt, M, N, K in shapes:
+            a = S.fp8_codes((bt, M, K), seed=1).cuda()
+            b = S.fp8_codes((1, N, K), seed=2).cuda() if bt == 8 else S.fp8_codes((bt, N, K), seed=2).cuda()
+            one = torch.ones(1, device="cuda")
+            bias = S.uniform((N,), seed=3).cuda()
+            out = torch.empty((bt, M, N), dtype=torch.bfloat16, device="cuda")
+            for with_bias in (False, True):
+                fn = lambda: ops.mm(a, b, one, one, bias if with_bias else None, out=out)  # noqa: E731
+                for _ in range(3):
+                    fn()
+                ms = _median_ms(fn, torch, args.iters)
+                fl = 2.0 * bt * M * N * K
+                print(json.dumps({"kernel": "mm_fp8", "batch": bt, "M": M, "N": N, "K": K, "bias": with_bias,
+                                  "us": round(ms * 1e3, 2), "tflops": round(fl / ms / 1e9, 1)}))
+    else:
+        for rows, cols in (QUANT_SHAPES if not want else want):
+            for dt in ("bf16", "fp32"):
+                x = S.quant_sweep_input(rows, cols, dt, 1.0).cuda()
+                eb = x.element_size()
+                for layout, name in ((ops.ROW, "row"), (ops.TRANSPOSED, "T"), (ops.DUAL, "dual")):
+                    ring = ops.Ring()
+                    out = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
+                    out_t = torch.empty((cols, rows), dtype=torch.uint8, device="cuda")
+                    fn = lambda: ops.quantize(x, ops.E4M3, layout, ring, out, out_t)  # noqa: E731
+                    for _ in range(3):
+                        fn()
+                    ms = _median_ms(fn, torch, args.iters, flush)
+                    nbytes = rows * cols * (eb + (2 if layout == ops.DUAL else 1)) + 96
+                    print(json.dumps({"kernel": "quantize", "dtype": dt, "layout": name, "rows": rows,
+                                      "cols": cols, "us": round(ms * 1e3, 2),
+                                      "gbs": round(nbytes / ms / 1e6, 1)}))
+    return 0
+
+
 # -------------------------------------------------------------------- main ----
 
 def main():
     args = parse()
+    if args.sweep:
+        return sweep(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -42,7 +42,7 @@ L2_BYTES = 126 * 1024 * 1024
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--M", type=int, default=8192)
@@ -95,7 +95,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -106,10 +106,13 @@ class ClockSampler:
                 self.proc.kill()
             self.t.join(timeout=2)
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
+        """Median SM clock and active throttle reasons of the samples read between t0 and t1."""
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ts, ln in self.lines:
+            if (t0 is not None and ts < t0) or (t1 is not None and ts > t1 + 0.25):
+                continue
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -361,11 +364,14 @@ def main():
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(local) as clk:
+        time.sleep(0.6)  # let nvidia-smi start sampling before the timed region
+        t_clk0 = time.monotonic()
         e0.record(st)
         for i in range(args.steps):
             run_step(lins, ops, i)
         e1.record(st)
         torch.cuda.synchronize()
+        t_clk1 = time.monotonic()
     ms = e0.elapsed_time(e1) / args.steps
     if pg:
         t = torch.tensor([ms], device="cuda")
@@ -384,7 +390,7 @@ def main():
                      torch.empty(L.dw.shape, dtype=L.dw.dtype).pin_memory()) for L in lins]
         h2d = sum(x.numel() * x.element_size() + g.numel() * g.element_size() for x, g in (h[0] for h in host_in))
         d2h = sum(sum(t.numel() * t.element_size() for t in ho) for ho in host_out)
-        steps_e2e = max(3, args.steps // 5)
+        steps_e2e = max(3, min(200, args.steps // 5))
         if pg:
             pg.barrier()
         torch.cuda.synchronize()
@@ -444,7 +450,7 @@ def main():
                          "kernel": "mm_fp8_kernel (all 6 GEMM launches of the step)", "peak_source": peak_src},
             "quantize_roofline": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                                   "frac": round(quant_gbs / hbm_peak, 4), "peak_source": "of measured hbm_gbs"},
-            "clocks": clk.summary(),
+            "clocks": clk.summary(t_clk0, t_clk1),
             "gpu_launches": 12 * args.steps,
             "e2e": e2e,
         }

@@ -1,6 +1,8 @@
 // Status strings, the device error word and device info of the fp8ds C ABI.
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "common.cuh"
 
 namespace {
@@ -21,6 +23,20 @@ uint32_t* error_word_ptr() {
     g_error_ptr[dev] = static_cast<uint32_t*>(p);
   }
   return g_error_ptr[dev];
+}
+
+void* tensor_map_encoder() {
+  static void* fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = p;
+  });
+  return fn;
 }
 }  // namespace fp8ds
 

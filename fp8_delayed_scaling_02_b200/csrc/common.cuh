@@ -24,12 +24,17 @@ enum WaitSite : uint32_t {
   kWaitMmaTmemEmpty = 3,
   kWaitEpilogueTmemFull = 4,
   kWaitDrain = 5,
+  kWaitQuantizeTma = 6,
 };
 
 // Library-global device error word (defined in capi.cu, relocatable device code
 // is not used, so each translation unit that records errors gets the address
 // through error_word_ptr()).
 uint32_t* error_word_ptr();
+
+// cuTensorMapEncodeTiled, fetched once through the runtime's driver entry
+// point (no link-time dependency on libcuda).  Returns nullptr if unavailable.
+void* tensor_map_encoder();
 
 // Nanosecond budget of every bounded wait in a kernel.
 constexpr unsigned long long kWaitBudgetNs = 2000000000ull;  // 2 s

@@ -9,7 +9,7 @@
 //
 // B200 design (the pages' kernels are sm_89 register-fragment MMAs; none of
 // that carries over):
-//   * persistent kernel, one CTA per SM, 6 warps with fixed roles:
+//   * persistent kernel, one CTA per SM, 10 warps with fixed roles:
 //       warp 0      TMA producer: 128x128-byte A and BNx128-byte B tiles,
 //                   128B-swizzled, into a STAGES-deep shared-memory ring
 //                   guarded by full/empty mbarriers;
@@ -17,9 +17,11 @@
 //                   (kind::f8f6f4, M=128, N=BN, K=32 per instruction), fp32
 //                   accumulators in TMEM, double-buffered (2 x BN columns) so
 //                   the epilogue of tile i overlaps the mainloop of tile i+1;
-//       warps 2..5  epilogue: tcgen05.ld 32 columns at a time, one fmaf per
-//                   element (acc * sinv_a*sinv_b + bias), one bf16 rounding,
-//                   16-byte stores with guarded tails.
+//       warps 2..9  epilogue: two warps per TMEM lane quadrant, each on half
+//                   the columns; tcgen05.ld 2x32 columns per wait, one fmaf
+//                   per element (acc * sinv_a*sinv_b + bias), one bf16
+//                   rounding, 32x32 TMA stores from swizzled staging buffers
+//                   (guarded plain stores when output rows are unaligned).
 //   * every mbarrier wait is bounded by a %globaltimer budget; a wait that
 //     runs out records the site in the library error word, raises a shared
 //     abort flag so the other roles leave their loops, waits (bounded) for
@@ -31,6 +33,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -41,7 +44,9 @@ namespace {
 constexpr int kBM = 128;      // rows of A per tile (UMMA M)
 constexpr int kBK = 128;      // K bytes (= fp8 elements) per stage: one 128B swizzle atom row
 constexpr int kUmmaK = 32;    // K per tcgen05.mma for 8-bit operands
-constexpr int kThreadsMM = 192;
+constexpr int kEpiWarps = 8;      // two warps per TMEM lane quadrant, each owning half the columns
+constexpr int kThreadsMM = 32 * (2 + kEpiWarps);
+constexpr int kStagingBytes = 2048;  // one 32x32 bf16 box per staging buffer
 
 template <int BN>
 struct Cfg {
@@ -50,8 +55,10 @@ struct Cfg {
   static constexpr int kBBytes = BN * kBK;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;  // two accumulators
-  static constexpr int kBarOffset = kStages * kStageBytes;
+  static constexpr int kStagingOffset = kStages * kStageBytes;  // 2 buffers per epilogue warp
+  static constexpr int kBarOffset = kStagingOffset + kEpiWarps * 2 * kStagingBytes;
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
 struct MmParams {
@@ -64,6 +71,7 @@ struct MmParams {
   const float* bias;
   uint16_t* out;
   int out_vec;       // 16-byte stores are legal for full 8-column groups
+  int tma_store;     // output leaves through TMA stores (tmC valid)
   int bias_vec;      // bias is 16-byte aligned
   uint32_t idesc;
   uint32_t* err;
@@ -127,6 +135,18 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm,
       : "memory");
 }
 
+// Bulk tensor store of a shared-memory box; clipped to the tensor bounds.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(tm)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tm)) : "memory");
 }
@@ -157,9 +177,11 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
 }
 
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 // 32 lanes x 32 consecutive 32-bit columns; lane t of the warp receives row
 // (32 * (warp % 4) + t) of the accumulator.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -170,7 +192,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr)
       : "memory");
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
 // Shared-memory matrix descriptor of a K-major tile written by TMA with the
@@ -202,7 +223,7 @@ __device__ __forceinline__ void decode_tile(const MmParams& p, int t, int& b, in
 template <int BN>
 __global__ void __launch_bounds__(kThreadsMM, 1)
     mm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const MmParams p) {
+                  const __grid_constant__ CUtensorMap tmC, const MmParams p) {
   using C = Cfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles.
@@ -230,7 +251,7 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), 4);
+      mbar_init(tempty_bar(a), kEpiWarps);
     }
     mbar_init(done_bar, 1);
     *abort = 0;
@@ -240,6 +261,7 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&tmA);
     prefetch_tmap(&tmB);
+    if (p.tma_store) prefetch_tmap(&tmC);
   }
   if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
   tc_fence_before();
@@ -334,9 +356,21 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..9) ----------------
+    // Warp w reads TMEM lane quadrant w % 4 (rows 32*(w%4) .. +31 of the tile)
+    // and half (w-2)/4 of the columns.  Two 32-column chunks are loaded per
+    // tcgen05.wait::ld; the accumulator is released to the MMA warp as soon
+    // as its last chunk is in registers.  Results leave through 32x32 bf16
+    // TMA stores from two 64B-swizzled staging buffers per warp (rows of
+    // 64 bytes, 16-byte unit j of row r at unit j ^ ((r >> 1) & 3)), or,
+    // when the output rows are not 16-byte aligned, through guarded stores.
+    const int ew = warp - 2;
     const int quad = warp & 3;
+    const int half = ew >> 2;
+    constexpr int kHalfCols = BN / 2;
     const float sab = __fmul_rn(*p.sinv_a, *p.sinv_b);
+    const uint32_t stage0 = sbase + C::kStagingOffset + uint32_t(ew) * 2u * kStagingBytes;
+    int buf = 0;
     int i = 0;
     for (int t = blockIdx.x; t < p.tiles_total; t += gridDim.x, ++i) {
       const int acc = i & 1;
@@ -345,60 +379,97 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
       tc_fence_after();
       int b, mt, nt;
       decode_tile(p, t, b, mt, nt);
-      const int row = mt * kBM + quad * 32 + lane;
+      const int m0 = mt * kBM + quad * 32;
+      const int row = m0 + lane;
       uint16_t* orow = p.out + int64_t(b) * p.c_stride + int64_t(row) * p.N;
-      for (int c = 0; c < BN / 32; ++c) {
-        const int n0 = nt * BN + c * 32;
-        if (n0 >= p.N) break;  // warp-uniform
-        uint32_t r[32];
-        if (p.k_blocks > 0) {
-          tmem_ld32(tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + c * 32), r);
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) r[j] = 0u;
+      const uint32_t tbase = tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + half * kHalfCols);
+      const int nbase = nt * BN + half * kHalfCols;
+      bool released = false;
+#pragma unroll 1
+      for (int c = 0; c < kHalfCols / 32; c += 2) {
+        if (nbase + c * 32 >= p.N) break;  // warp-uniform: the rest of this half is beyond N
+        uint32_t r[2][32];
+        tmem_ld32_nowait(tbase + uint32_t(c * 32), r[0]);
+        if (nbase + (c + 1) * 32 < p.N) tmem_ld32_nowait(tbase + uint32_t((c + 1) * 32), r[1]);
+        tmem_wait_ld();
+        if (c + 2 >= kHalfCols / 32 || nbase + (c + 2) * 32 >= p.N) {
+          // Last TMEM read of this tile for this warp: hand the accumulator back.
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(tempty_bar(acc));
+          released = true;
         }
-        float bv[32];
-        const bool full = n0 + 32 <= p.N;
-        if (p.bias != nullptr) {
-          if (full && p.bias_vec) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 f = __ldg(reinterpret_cast<const float4*>(p.bias + n0) + j);
-              bv[4 * j] = f.x; bv[4 * j + 1] = f.y; bv[4 * j + 2] = f.z; bv[4 * j + 3] = f.w;
+        for (int h = 0; h < 2; ++h) {
+          const int n0 = nbase + (c + h) * 32;
+          if (n0 >= p.N) break;  // warp-uniform
+          uint32_t packed[16];
+          const bool full = n0 + 32 <= p.N;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (p.bias != nullptr) {
+              if (full && p.bias_vec) {
+                bv = __ldg(reinterpret_cast<const float4*>(p.bias + n0) + j);
+              } else {
+                const int nn = n0 + 4 * j;
+                bv.x = nn < p.N ? __ldg(p.bias + nn) : 0.f;
+                bv.y = nn + 1 < p.N ? __ldg(p.bias + nn + 1) : 0.f;
+                bv.z = nn + 2 < p.N ? __ldg(p.bias + nn + 2) : 0.f;
+                bv.w = nn + 3 < p.N ? __ldg(p.bias + nn + 3) : 0.f;
+              }
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) bv[j] = (n0 + j < p.N) ? __ldg(p.bias + n0 + j) : 0.0f;
+            const float y0 = fmaf(__uint_as_float(r[h][4 * j + 0]), sab, bv.x);
+            const float y1 = fmaf(__uint_as_float(r[h][4 * j + 1]), sab, bv.y);
+            const float y2 = fmaf(__uint_as_float(r[h][4 * j + 2]), sab, bv.z);
+            const float y3 = fmaf(__uint_as_float(r[h][4 * j + 3]), sab, bv.w);
+            const __nv_bfloat162 h01 = __floats2bfloat162_rn(y0, y1);
+            const __nv_bfloat162 h23 = __floats2bfloat162_rn(y2, y3);
+            packed[2 * j] = *reinterpret_cast<const uint32_t*>(&h01);
+            packed[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h23);
           }
-        } else {
+          if (p.tma_store) {
+            if (m0 < p.M) {
+              const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
+              if (lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
+              __syncwarp();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) bv[j] = 0.0f;
-        }
-        uint32_t packed[16];
+              for (int u = 0; u < 4; ++u) {
+                const uint32_t addr = sbuf + uint32_t(lane) * 64u + uint32_t((u ^ ((lane >> 1) & 3)) * 16);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[4 * u]),
+                             "r"(packed[4 * u + 1]), "r"(packed[4 * u + 2]), "r"(packed[4 * u + 3])
+                             : "memory");
+              }
+              fence_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(&tmC, sbuf, n0, m0, b);
+                bulk_commit();
+              }
+              buf ^= 1;
+            }
+          } else if (row < p.M) {
+            if (full && p.out_vec) {
+              uint4* o = reinterpret_cast<uint4*>(orow + n0);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float y0 = fmaf(__uint_as_float(r[2 * j]), sab, bv[2 * j]);
-          const float y1 = fmaf(__uint_as_float(r[2 * j + 1]), sab, bv[2 * j + 1]);
-          const __nv_bfloat162 h = __floats2bfloat162_rn(y0, y1);
-          packed[j] = *reinterpret_cast<const uint32_t*>(&h);
-        }
-        if (row < p.M) {
-          if (full && p.out_vec) {
-            uint4* o = reinterpret_cast<uint4*>(orow + n0);
+              for (int j = 0; j < 4; ++j)
+                o[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
+            } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              o[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (n0 + j < p.N) orow[n0 + j] = uint16_t(packed[j >> 1] >> (16 * (j & 1)));
+              for (int j = 0; j < 32; ++j)
+                if (n0 + j < p.N) orow[n0 + j] = uint16_t(packed[j >> 1] >> (16 * (j & 1)));
+            }
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty_bar(acc));
+      if (!released) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(tempty_bar(acc));
+      }
     }
+    if (p.tma_store && lane == 0) bulk_wait_all();
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -424,21 +495,9 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
-EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
+EncodeTiledFn get_encode_fn() { return reinterpret_cast<EncodeTiledFn>(tensor_map_encoder()); }
 
-// 3-D map over uint8 [batch, rows, K] with a box of [1, box_rows, 128].
+// 3-D map over uint8 [batch, rows, K] with a box of [1, box_rows, 128], 128B swizzle.
 bool make_map(CUtensorMap* m, const uint8_t* base, int64_t K, int64_t rows, int64_t batch, int64_t bstride,
               int box_rows) {
   EncodeTiledFn enc = get_encode_fn();
@@ -450,6 +509,21 @@ bool make_map(CUtensorMap* m, const uint8_t* base, int64_t K, int64_t rows, int6
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// 3-D map over the bf16 output [batch, M, N] with a 32x32 box, 64B swizzle
+// (the staging-buffer layout the epilogue writes).
+bool make_out_map(CUtensorMap* m, uint16_t* base, int64_t M, int64_t N, int64_t batch, int64_t c_stride) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {cuuint64_t(N), cuuint64_t(M), cuuint64_t(batch)};
+  const cuuint64_t strides[2] = {cuuint64_t(N * 2), cuuint64_t((batch > 1 ? c_stride : M * N) * 2)};
+  const cuuint32_t box[3] = {32u, 32u, 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -482,11 +556,13 @@ bool ensure_smem_attr() {
 template <int BN>
 int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
               const int64_t* strides, MmParams p, int sms, cudaStream_t st) {
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, tc;
   const int64_t ba = (batch > 1 && strides[0] != 0) ? batch : 1;
   const int64_t bb = (batch > 1 && strides[1] != 0) ? batch : 1;
   if (!make_map(&ta, A, K, M, ba, ba > 1 ? strides[0] : 0, kBM)) return FP8_ERR_CUDA;
   if (!make_map(&tb, B, K, N, bb, bb > 1 ? strides[1] : 0, BN)) return FP8_ERR_CUDA;
+  memset(&tc, 0, sizeof(tc));
+  if (p.tma_store && !make_out_map(&tc, p.out, M, N, batch, p.c_stride)) return FP8_ERR_CUDA;
   p.a_bcast = ba == 1;
   p.b_bcast = bb == 1;
   p.m_tiles = int((M + kBM - 1) / kBM);
@@ -497,7 +573,7 @@ int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t 
   p.idesc |= uint32_t(BN >> 3) << 17;
   if (!ensure_smem_attr<BN>()) return FP8_ERR_CUDA;
   const int grid = std::max(1, std::min(p.tiles_total, sms));
-  mm_fp8_kernel<BN><<<grid, kThreadsMM, Cfg<BN>::kSmemBytes, st>>>(ta, tb, p);
+  mm_fp8_kernel<BN><<<grid, kThreadsMM, Cfg<BN>::kSmemBytes, st>>>(ta, tb, tc, p);
   return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
@@ -545,6 +621,7 @@ extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, 
   p.bias = bias;
   p.out = out_bf16;
   p.out_vec = (reinterpret_cast<uintptr_t>(out_bf16) % 16 == 0) && (N % 8 == 0) && (c_stride % 8 == 0);
+  p.tma_store = p.out_vec;
   p.bias_vec = bias != nullptr && (reinterpret_cast<uintptr_t>(bias) % 16 == 0);
   const uint32_t fa = (layout & FP8_MM_A_E5M2) ? 1u : 0u;
   const uint32_t fb = (layout & FP8_MM_B_E5M2) ? 1u : 0u;

@@ -28,7 +28,10 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include <cuda.h>
+
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 
@@ -173,14 +176,35 @@ __device__ __forceinline__ uint8_t cvt_one(float x, float s) {
 
 // Block-reduce the per-thread amax, publish it with one atomicMax, draw a
 // ticket; the last block folds the ring.  Must be called by every thread.
+// The ring's history and idx are not written until the last block runs, so
+// each block reads them early (prefetch_ring at kernel start, one lane per
+// word) and the fold itself needs no dependent global reads besides the
+// amax word.
+struct RingCache {
+  float hist;  // history[threadIdx.x] for threads 0..15
+  int idx;     // read by thread 16
+};
+
+__device__ __forceinline__ RingCache prefetch_ring(const RingArgs& ring) {
+  RingCache c{0.0f, 0};
+  if (threadIdx.x < kHistoryLen) c.hist = ring.history[threadIdx.x];
+  if (threadIdx.x == kHistoryLen) c.idx = *ring.idx;
+  return c;
+}
+
 template <int FMT>
-__device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& ring, float s_used) {
+__device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& ring, float s_used,
+                                                 const RingCache& rc) {
   __shared__ float warp_max[kThreads / 32];
+  __shared__ float hist_s[kHistoryLen];
+  __shared__ int idx_s;
   __shared__ int last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
   if (lane == 0) warp_max[warp] = amax;
+  if (threadIdx.x < kHistoryLen) hist_s[threadIdx.x] = rc.hist;
+  if (threadIdx.x == kHistoryLen) idx_s = rc.idx;
   __syncthreads();
   if (threadIdx.x == 0) {
     float m = 0.0f;
@@ -190,25 +214,25 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
     __threadfence();  // release: our amax is visible before our ticket
     const unsigned t = atomicAdd(&ring.scratch[1], 1u);
     last = (t == gridDim.x - 1);
-  }
-  __syncthreads();
-  if (last && threadIdx.x == 0) {
-    __threadfence();  // acquire: every block's amax is visible now
-    const float a = __uint_as_float(atomicExch(&ring.scratch[0], 0u));
-    int idx = *ring.idx;
-    idx = ((idx % kHistoryLen) + kHistoryLen) % kHistoryLen;
-    ring.history[idx] = a;
-    float m = 0.0f;
+    if (last) {
+      __threadfence();  // acquire: every block's amax is visible now
+      const float a = __uint_as_float(atomicExch(&ring.scratch[0], 0u));
+      int idx = idx_s;
+      idx = ((idx % kHistoryLen) + kHistoryLen) % kHistoryLen;
+      hist_s[idx] = a;
+      float mx = 0.0f;
 #pragma unroll
-    for (int i = 0; i < kHistoryLen; ++i) m = fmaxf(m, ring.history[i]);
-    *ring.idx = (idx + 1) % kHistoryLen;
-    const float fmax = FMT == FP8_E4M3 ? kE4M3Max : kE5M2Max;
-    if (m > 0.0f && isfinite(m)) {
-      const float c = __fdiv_rn(fmax, m);
-      if (isfinite(c) && c > 0.0f) *ring.scale = c;
+      for (int i = 0; i < kHistoryLen; ++i) mx = fmaxf(mx, hist_s[i]);
+      ring.history[idx] = a;
+      *ring.idx = (idx + 1) % kHistoryLen;
+      const float fmax = FMT == FP8_E4M3 ? kE4M3Max : kE5M2Max;
+      if (mx > 0.0f && isfinite(mx)) {
+        const float c = __fdiv_rn(fmax, mx);
+        if (isfinite(c) && c > 0.0f) *ring.scale = c;
+      }
+      *ring.scale_inv = __frcp_rn(s_used);
+      ring.scratch[1] = 0u;
     }
-    *ring.scale_inv = __frcp_rn(s_used);
-    atomicExch(&ring.scratch[1], 0u);
   }
 }
 
@@ -246,6 +270,7 @@ template <int DT, int FMT, bool kAligned>
 __global__ void __launch_bounds__(kThreads) quantize_row_kernel(const RowArgs a) {
   constexpr int kB = In<DT>::kBytes;
   const float s = *a.ring.scale;
+  const RingCache rc = prefetch_ring(a.ring);
   float amax = 0.0f;
   const int64_t tid = int64_t(blockIdx.x) * kThreads + threadIdx.x;
   const int64_t nthr = int64_t(gridDim.x) * kThreads;
@@ -268,7 +293,7 @@ __global__ void __launch_bounds__(kThreads) quantize_row_kernel(const RowArgs a)
     row_chunk<DT, FMT, kAligned>(a, j, s, amax);
     if (j + nthr < a.nchunks) row_chunk<DT, FMT, kAligned>(a, j + nthr, s, amax);
   }
-  amax_ticket_fold<FMT>(amax, a.ring, s);
+  amax_ticket_fold<FMT>(amax, a.ring, s, rc);
 }
 
 // ---- T / DUAL layouts --------------------------------------------------------
@@ -293,6 +318,7 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs 
   constexpr int kB = In<DT>::kBytes;
   __shared__ uint32_t sT[kTileC * kPitchW];
   const float s = *a.ring.scale;
+  const RingCache rc = prefetch_ring(a.ring);
   float amax = 0.0f;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int lr0 = 32 * (warp & 3) + 4 * (lane & 7);  // first of this lane's 4 rows
@@ -357,7 +383,212 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs 
       }
     }
   }
-  amax_ticket_fold<FMT>(amax, a.ring, s);
+  amax_ticket_fold<FMT>(amax, a.ring, s, rc);
+}
+
+// ---- T / DUAL layouts, TMA-fed pipeline (16-byte aligned rows) ------------------
+//
+// Same tile geometry and lane mapping as quantize_tile_kernel, but the input
+// tiles arrive by TMA (128 rows x 128 bytes per box, 128B-swizzled) into a
+// kTmaStages-deep shared-memory ring, so each block keeps several tiles of
+// HBM reads in flight while it converts and transposes the current one.
+// Blocks are persistent over tiles.  Used when the input base is 16-byte
+// aligned and a row is a multiple of 16 bytes; ragged edges are zero-filled
+// by TMA and the stores are guarded.
+
+constexpr int kTmaStages = 4;
+
+template <int DT>
+struct TmaTile {
+  static constexpr int kBoxes = In<DT>::kBytes == 4 ? 2 : 1;  // 128-byte-wide boxes per 64-column tile
+  static constexpr int kBoxBytes = kTileR * 128;
+  static constexpr int kStageBytes = kBoxes * kBoxBytes;
+  static constexpr int kStages = DT == FP8_IN_FP32 ? 3 : kTmaStages;
+  static constexpr int kSmem = kStages * kStageBytes + kTileC * kPitchW * 4 + 64 + 1024;
+};
+
+struct TmaTileArgs {
+  TileArgs t;
+  uint32_t* err;
+};
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ bool bar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+__device__ __forceinline__ bool bar_wait_bounded(uint32_t bar, uint32_t parity) {
+  if (bar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  while (!bar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitBudgetNs) return false;
+  }
+  return true;
+}
+
+template <int DT>
+__device__ __forceinline__ void issue_tile_load(const CUtensorMap* tm, uint32_t dst, uint32_t bar, int64_t t,
+                                                int64_t tiles_c) {
+  const int r0 = int((t / tiles_c) * kTileR);
+  const int c0 = int((t % tiles_c) * kTileC);
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+               "r"(uint32_t(TmaTile<DT>::kStageBytes))
+               : "memory");
+#pragma unroll
+  for (int bx = 0; bx < TmaTile<DT>::kBoxes; ++bx) {
+    const int cx = c0 + bx * (128 / In<DT>::kBytes);
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst + uint32_t(bx * TmaTile<DT>::kBoxBytes)),
+        "l"(reinterpret_cast<uint64_t>(tm)), "r"(cx), "r"(r0), "r"(bar)
+        : "memory");
+  }
+}
+
+template <int DT, int FMT, bool kDual>
+__global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __grid_constant__ CUtensorMap tmIn,
+                                                                      const TmaTileArgs args) {
+  using TT = TmaTile<DT>;
+  constexpr int kB = In<DT>::kBytes;
+  const TileArgs& a = args.t;
+  extern __shared__ uint8_t qsmem_raw[];
+  uint8_t* smem = qsmem_raw + ((1024u - (smem_addr(qsmem_raw) & 1023u)) & 1023u);
+  const uint32_t sbase = smem_addr(smem);
+  uint32_t* sT = reinterpret_cast<uint32_t*>(smem + TT::kStages * TT::kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sT + kTileC * kPitchW);
+  const uint32_t bar0 = smem_addr(bars);
+
+  const float s = *a.ring.scale;
+  const RingCache rc = prefetch_ring(a.ring);
+  float amax = 0.0f;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lr0 = 32 * (warp & 3) + 4 * (lane & 7);
+  const int lc0 = 32 * (warp >> 2) + 8 * (lane >> 3);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < TT::kStages; ++i)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8u * i) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmIn)) : "memory");
+  }
+  __syncthreads();
+  int64_t issued = 0;  // tiles of this block whose loads thread 0 has issued
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < TT::kStages; ++i) {
+      const int64_t t = blockIdx.x + int64_t(i) * gridDim.x;
+      if (t >= a.ntiles) break;
+      issue_tile_load<DT>(&tmIn, sbase + uint32_t(i * TT::kStageBytes), bar0 + 8u * i, t, a.tiles_c);
+      ++issued;
+    }
+  }
+
+  int64_t k = 0;
+  for (int64_t t = blockIdx.x; t < a.ntiles; t += gridDim.x, ++k) {
+    const int stage = int(k % TT::kStages);
+    const uint32_t parity = uint32_t((k / TT::kStages) & 1);
+    const bool ok = bar_wait_bounded(bar0 + 8u * stage, parity);
+    const uint8_t* st = smem + stage * TT::kStageBytes;
+    const int64_t r0 = (t / a.tiles_c) * kTileR;
+    const int64_t c0 = (t % a.tiles_c) * kTileC;
+    uint32_t q[4][2];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int r = lr0 + i;
+      float v[8];
+      if constexpr (kB == 2) {
+        const int chunk = (lc0 >> 3) ^ (r & 7);
+        const uint4 w = *reinterpret_cast<const uint4*>(st + r * 128 + chunk * 16);
+        unpack2<DT>(w.x, v[0], v[1]);
+        unpack2<DT>(w.y, v[2], v[3]);
+        unpack2<DT>(w.z, v[4], v[5]);
+        unpack2<DT>(w.w, v[6], v[7]);
+      } else {
+        const int box = lc0 >> 5;
+        const int ch = (lc0 & 31) >> 2;
+        const uint8_t* rowp = st + box * TT::kBoxBytes + r * 128;
+        const float4 f0 = *reinterpret_cast<const float4*>(rowp + ((ch ^ (r & 7)) * 16));
+        const float4 f1 = *reinterpret_cast<const float4*>(rowp + (((ch + 1) ^ (r & 7)) * 16));
+        v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+        v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+      q[i][0] = cvt_pair<FMT>(v[0], v[1], s) | (cvt_pair<FMT>(v[2], v[3], s) << 16);
+      q[i][1] = cvt_pair<FMT>(v[4], v[5], s) | (cvt_pair<FMT>(v[6], v[7], s) << 16);
+    }
+    // Every thread is done with this stage and with the previous tile's sT.
+    if (!__syncthreads_and(ok ? 1 : 0)) {
+      if (threadIdx.x == 0) record_device_error(args.err, kWaitQuantizeTma);
+      break;
+    }
+    if (threadIdx.x == 0) {
+      const int64_t tn = t + int64_t(TT::kStages) * gridDim.x;
+      if (tn < a.ntiles) {
+        issue_tile_load<DT>(&tmIn, sbase + uint32_t(stage * TT::kStageBytes), bar0 + 8u * stage, tn, a.tiles_c);
+        ++issued;
+      }
+    }
+    const bool interior = (r0 + kTileR <= a.rows) && (c0 + kTileC <= a.cols);
+    if constexpr (kDual) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int64_t r = r0 + lr0 + i;
+        const int64_t c = c0 + lc0;
+        uint8_t* o = a.out + r * a.cols + c;
+        if (interior && a.out8) {
+          *reinterpret_cast<uint2*>(o) = make_uint2(q[i][0], q[i][1]);
+        } else if (r < a.rows) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (c + j < a.cols) o[j] = uint8_t(q[i][j >> 2] >> (8 * (j & 3)));
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int sh = 8 * (j & 3);
+      const uint32_t w = ((q[0][j >> 2] >> sh) & 0xFFu) | (((q[1][j >> 2] >> sh) & 0xFFu) << 8) |
+                         (((q[2][j >> 2] >> sh) & 0xFFu) << 16) | (((q[3][j >> 2] >> sh) & 0xFFu) << 24);
+      sT[(lc0 + j) * kPitchW + (lr0 >> 2)] = w;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kTileC / 8; ++kk) {
+      const int cl = 8 * warp + kk;
+      const int64_t c = c0 + cl;
+      const int64_t r = r0 + 4 * lane;
+      const uint32_t w = sT[cl * kPitchW + lane];
+      if (c < a.cols) {
+        uint8_t* o = a.out_t + c * a.rows + r;
+        if (a.outt4 && r + 4 <= a.rows) {
+          *reinterpret_cast<uint32_t*>(o) = w;
+        } else {
+#pragma unroll
+          for (int b = 0; b < 4; ++b)
+            if (r + b < a.rows) o[b] = uint8_t(w >> (8 * b));
+        }
+      }
+    }
+  }
+  // After an abort, let every copy this block issued land before its shared
+  // memory is released (bounded).
+  if (threadIdx.x == 0) {
+    for (int64_t j = k; j < issued; ++j)
+      bar_wait_bounded(bar0 + 8u * uint32_t(j % TT::kStages), uint32_t((j / TT::kStages) & 1));
+  }
+  amax_ticket_fold<FMT>(amax, a.ring, s, rc);
 }
 
 // ---- host side ---------------------------------------------------------------
@@ -399,6 +630,60 @@ template <int DT>
 int dispatch_fmt_tile(int fmt, const TileArgs& a, int grid, cudaStream_t st, bool dual) {
   return fmt == FP8_E4M3 ? launch_tile<DT, FP8_E4M3>(a, grid, st, dual)
                          : launch_tile<DT, FP8_E5M2>(a, grid, st, dual);
+}
+
+using EncodeTiledFnQ = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// 2-D map over the input [rows, cols] with a 128-row x 128-byte box, 128B swizzle.
+bool make_input_map(CUtensorMap* m, const void* in, int dtype, int64_t rows, int64_t cols) {
+  auto enc = reinterpret_cast<EncodeTiledFnQ>(tensor_map_encoder());
+  if (!enc) return false;
+  const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
+  const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
+  const cuuint64_t strides[1] = {cuuint64_t(cols * eb)};
+  const cuuint32_t box[2] = {cuuint32_t(128 / eb), cuuint32_t(kTileR)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  const CUtensorMapDataType dt = eb == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
+  return enc(m, dt, 2, const_cast<void*>(in), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Resident blocks per SM of a TMA tile kernel instantiation (cached per device).
+template <int DT, int FMT, bool kDual>
+int tma_blocks_per_sm() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (cached[dev] == 0) {
+    auto kern = quantize_tile_tma_kernel<DT, FMT, kDual>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TmaTile<DT>::kSmem) != cudaSuccess)
+      return -1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, TmaTile<DT>::kSmem) != cudaSuccess || n < 1)
+      return -1;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int DT, int FMT>
+int launch_tile_tma(const TileArgs& t, const CUtensorMap& map, int sms, cudaStream_t st, bool dual) {
+  TmaTileArgs a{t, error_word_ptr()};
+  const int bps = dual ? tma_blocks_per_sm<DT, FMT, true>() : tma_blocks_per_sm<DT, FMT, false>();
+  if (bps <= 0) return FP8_ERR_CUDA;
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(t.ntiles, int64_t(bps) * sms)));
+  if (dual) quantize_tile_tma_kernel<DT, FMT, true><<<grid, kThreads, TmaTile<DT>::kSmem, st>>>(map, a);
+  else quantize_tile_tma_kernel<DT, FMT, false><<<grid, kThreads, TmaTile<DT>::kSmem, st>>>(map, a);
+  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+template <int DT>
+int dispatch_fmt_tile_tma(int fmt, const TileArgs& a, const CUtensorMap& map, int sms, cudaStream_t st, bool dual) {
+  return fmt == FP8_E4M3 ? launch_tile_tma<DT, FP8_E4M3>(a, map, sms, st, dual)
+                         : launch_tile_tma<DT, FP8_E5M2>(a, map, sms, st, dual);
 }
 
 }  // namespace
@@ -457,8 +742,18 @@ extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t col
   a.out8 = (layout == FP8_LAYOUT_DUAL) && (reinterpret_cast<uintptr_t>(out) % 8 == 0) && (cols % 8 == 0);
   a.outt4 = (reinterpret_cast<uintptr_t>(out_t) % 4 == 0) && (rows % 4 == 0);
   a.ring = r;
-  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(a.ntiles, max_grid)));
   const bool dual = layout == FP8_LAYOUT_DUAL;
+  if (n > 0 && reinterpret_cast<uintptr_t>(in) % 16 == 0 && (cols * eb) % 16 == 0) {
+    CUtensorMap map;
+    std::memset(&map, 0, sizeof(map));
+    if (!make_input_map(&map, in, dtype, rows, cols)) return FP8_ERR_CUDA;
+    switch (dtype) {
+      case FP8_IN_BF16: return dispatch_fmt_tile_tma<FP8_IN_BF16>(fmt, a, map, sms, st, dual);
+      case FP8_IN_FP16: return dispatch_fmt_tile_tma<FP8_IN_FP16>(fmt, a, map, sms, st, dual);
+      default: return dispatch_fmt_tile_tma<FP8_IN_FP32>(fmt, a, map, sms, st, dual);
+    }
+  }
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(a.ntiles, max_grid)));
   switch (dtype) {
     case FP8_IN_BF16: return dispatch_fmt_tile<FP8_IN_BF16>(fmt, a, grid, st, dual);
     case FP8_IN_FP16: return dispatch_fmt_tile<FP8_IN_FP16>(fmt, a, grid, st, dual);

@@ -8,7 +8,9 @@ workload (hidden 1536, FFN 4096) at M = 8192 tokens, for both linear shapes
   fwd  Y  = Xq . Wq^T * sx*sw + b      (M x N x 1536)
   dX   = Gq . (W^T)q^T * sg*sw          (M x 1536 x N, A = E5M2)
   dW   = (G^T)q . (X^T)q^T * sg*sx      (N x 1536 x M, A = E5M2)
-12 kernel launches per step (6 quantize, 6 GEMM).
+12 kernel launches per step (6 quantize, 6 GEMM).  The device-timed steps
+replay a CUDA graph of the step; the end-to-end figure calls the C ABI
+directly every step with host copies in and out.
 
 Printed JSON line (rank 0): value = GEMM TFLOP/s of the whole step (GEMM
 flops / step time, quantize time included), plus the GEMM-only TFLOP/s,
@@ -179,23 +181,44 @@ def run_step(lins, ops, i):
         L.gemms(ops)
 
 
-def time_split(lins, ops, torch, reps):
-    """Per-phase device time (quantize vs GEMM) with events on the launching stream."""
+def capture(torch, fn):
+    """CUDA graph of fn() (the library allocates nothing and never syncs, so it captures)."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    return g
+
+
+def time_graph(torch, g, reps):
     st = torch.cuda.current_stream()
-    q_ms, g_ms = 0.0, 0.0
-    for i in range(reps):
-        for L in lins:
-            x, g = L.inputs[i % len(L.inputs)]
-            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-            e0.record(st)
-            L.quantize(ops, x, g)
-            e1.record(st)
-            L.gemms(ops)
-            e2.record(st)
-            e2.synchronize()
-            q_ms += e0.elapsed_time(e1)
-            g_ms += e1.elapsed_time(e2)
-    return q_ms / reps, g_ms / reps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    g.replay()
+    e0.record(st)
+    for _ in range(reps):
+        g.replay()
+    e1.record(st)
+    e1.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def time_split(lins, ops, torch, reps):
+    """Device time per step of the quantize phase and of the GEMM phase (graph replays)."""
+    def quant():
+        for i in range(2):
+            for L in lins:
+                x, g = L.inputs[i % len(L.inputs)]
+                L.quantize(ops, x, g)
+
+    def gemm():
+        for _ in range(2):
+            for L in lins:
+                L.gemms(ops)
+
+    gq, gm = capture(torch, quant), capture(torch, gemm)
+    q_ms = time_graph(torch, gq, reps) / 2
+    g_ms = time_graph(torch, gm, reps) / 2
+    del gq, gm
+    return q_ms, g_ms
 
 
 # ------------------------------------------------------------- CPU oracle ----
@@ -246,19 +269,22 @@ GEMM_SHAPES = [(1, n, n, n) for n in (512, 1024, 1152, 2048, 3072, 4096, 8192)] 
 QUANT_SHAPES = [(128, 1536), (2048, 1536), (8192, 1536), (16384, 4096), (2048, 1537), (8192, 1537)]
 
 
-def _median_ms(fn, torch, iters, flush=None):
-    st = torch.cuda.current_stream()
-    times = []
-    for _ in range(iters):
-        if flush is not None:
-            flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(st)
-        fn()
-        b.record(st)
-        b.synchronize()
-        times.append(a.elapsed_time(b))
-    return statistics.median(times)
+def _kernel_ms(fn, torch, iters, flush=None):
+    """Average device time of fn() from a CUDA graph of `iters` calls.  With
+    `flush`, every call is preceded by a write of a buffer twice the L2 size
+    and the time of a graph of the flushes alone is subtracted."""
+    def body():
+        for _ in range(iters):
+            if flush is not None:
+                flush.zero_()
+            fn()
+    t = time_graph(torch, capture(torch, body), 3)
+    if flush is not None:
+        def flush_only():
+            for _ in range(iters):
+                flush.zero_()
+        t -= time_graph(torch, capture(torch, flush_only), 3)
+    return t / iters
 
 
 def sweep(args):
@@ -285,7 +311,7 @@ def sweep(args):
                 fn = lambda: ops.mm(a, b, one, one, bias if with_bias else None, out=out)  # noqa: E731
                 for _ in range(3):
                     fn()
-                ms = _median_ms(fn, torch, args.iters)
+                ms = _kernel_ms(fn, torch, args.iters)
                 fl = 2.0 * bt * M * N * K
                 print(json.dumps({"kernel": "mm_fp8", "batch": bt, "M": M, "N": N, "K": K, "bias": with_bias,
                                   "us": round(ms * 1e3, 2), "tflops": round(fl / ms / 1e9, 1)}))
@@ -301,7 +327,7 @@ def sweep(args):
                     fn = lambda: ops.quantize(x, ops.E4M3, layout, ring, out, out_t)  # noqa: E731
                     for _ in range(3):
                         fn()
-                    ms = _median_ms(fn, torch, args.iters, flush)
+                    ms = _kernel_ms(fn, torch, args.iters, flush)
                     nbytes = rows * cols * (eb + (2 if layout == ops.DUAL else 1)) + 96
                     print(json.dumps({"kernel": "quantize", "dtype": dt, "layout": name, "rows": rows,
                                       "cols": cols, "us": round(ms * 1e3, 2),
@@ -356,8 +382,13 @@ def main():
     for i in range(max(3, args.warmup)):
         run_step(lins, ops, i)
     torch.cuda.synchronize()
-    q_ms, g_ms = time_split(lins, ops, torch, 5)
+    q_ms, g_ms = time_split(lins, ops, torch, 50)
 
+    # The timed steps replay a CUDA graph of two consecutive steps (one per
+    # input set), so the host launch cost is off the measured device time.
+    steps = args.steps + (args.steps % 2)
+    graph = capture(torch, lambda: (run_step(lins, ops, 0), run_step(lins, ops, 1)))
+    graph.replay()
     st = torch.cuda.current_stream()
     if pg:
         pg.barrier()
@@ -367,12 +398,13 @@ def main():
         time.sleep(0.6)  # let nvidia-smi start sampling before the timed region
         t_clk0 = time.monotonic()
         e0.record(st)
-        for i in range(args.steps):
-            run_step(lins, ops, i)
+        for i in range(steps // 2):
+            graph.replay()
         e1.record(st)
         torch.cuda.synchronize()
         t_clk1 = time.monotonic()
-    ms = e0.elapsed_time(e1) / args.steps
+    ms = e0.elapsed_time(e1) / steps
+    del graph
     if pg:
         t = torch.tensor([ms], device="cuda")
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
@@ -435,7 +467,7 @@ def main():
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
-            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4),
+            "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp8e4m3/e5m2->f32acc->bf16",
             "data": "synthetic",
             "config": {"workload": f"1.2B-model linears fwd+bwd (hidden 1536, FFN 4096), M={M} tokens, "
@@ -451,7 +483,8 @@ def main():
             "quantize_roofline": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                                   "frac": round(quant_gbs / hbm_peak, 4), "peak_source": "of measured hbm_gbs"},
             "clocks": clk.summary(t_clk0, t_clk1),
-            "gpu_launches": 12 * args.steps,
+            "gpu_launches": 12 * steps,
+            "timing": "device events around CUDA-graph replays of the step (12 kernels per step)",
             "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -1,6 +1,8 @@
 // Status strings, the device error word and device info of the fp8ds C ABI.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -37,6 +39,74 @@ void* tensor_map_encoder() {
       fn = p;
   });
   return fn;
+}
+
+namespace {
+using EncodeTiledFnC = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct MapKey {
+  const void* base;
+  uint64_t dims[3];
+  uint64_t strides[2];
+  uint32_t box[3];
+  int dtype, rank, swizzle, promo;
+  bool operator==(const MapKey& o) const { return std::memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+
+struct MapEntry {
+  MapKey key;
+  alignas(64) CUtensorMap map;
+  bool valid;
+};
+
+constexpr int kMapCacheSize = 32;
+thread_local MapEntry t_map_cache[kMapCacheSize];
+thread_local int t_map_next = 0;
+}  // namespace
+
+bool encode_tiled_cached(void* map, int data_type, int rank, const void* base, const uint64_t* dims,
+                         const uint64_t* strides, const uint32_t* box, int swizzle, int l2_promotion) {
+  if (rank < 1 || rank > 3) return false;
+  MapKey k;
+  std::memset(&k, 0, sizeof(k));
+  k.base = base;
+  for (int i = 0; i < rank; ++i) {
+    k.dims[i] = dims[i];
+    k.box[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) k.strides[i] = strides[i];
+  k.dtype = data_type;
+  k.rank = rank;
+  k.swizzle = swizzle;
+  k.promo = l2_promotion;
+  for (int i = 0; i < kMapCacheSize; ++i) {
+    if (t_map_cache[i].valid && t_map_cache[i].key == k) {
+      std::memcpy(map, &t_map_cache[i].map, sizeof(CUtensorMap));
+      return true;
+    }
+  }
+  auto enc = reinterpret_cast<EncodeTiledFnC>(tensor_map_encoder());
+  if (!enc) return false;
+  cuuint64_t d[3], st[2];
+  cuuint32_t bx[3], es[3] = {1u, 1u, 1u};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides[i];
+  MapEntry& e = t_map_cache[t_map_next];
+  e.valid = false;
+  if (enc(&e.map, CUtensorMapDataType(data_type), cuuint32_t(rank), const_cast<void*>(base), d, st, bx, es,
+          CU_TENSOR_MAP_INTERLEAVE_NONE, CUtensorMapSwizzle(swizzle), CUtensorMapL2promotion(l2_promotion),
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return false;
+  e.key = k;
+  e.valid = true;
+  t_map_next = (t_map_next + 1) % kMapCacheSize;
+  std::memcpy(map, &e.map, sizeof(CUtensorMap));
+  return true;
 }
 }  // namespace fp8ds
 

@@ -491,40 +491,24 @@ __global__ void mm_bias_only_kernel(uint16_t* out, const float* bias, int64_t M,
 
 // ---- host side -----------------------------------------------------------------
 
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn get_encode_fn() { return reinterpret_cast<EncodeTiledFn>(tensor_map_encoder()); }
-
 // 3-D map over uint8 [batch, rows, K] with a box of [1, box_rows, 128], 128B swizzle.
 bool make_map(CUtensorMap* m, const uint8_t* base, int64_t K, int64_t rows, int64_t batch, int64_t bstride,
               int box_rows) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {cuuint64_t(K), cuuint64_t(rows), cuuint64_t(batch)};
-  const cuuint64_t strides[2] = {cuuint64_t(K), cuuint64_t(batch > 1 ? bstride : K * rows)};
-  const cuuint32_t box[3] = {cuuint32_t(kBK), cuuint32_t(box_rows), 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(base), dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  const uint64_t dims[3] = {uint64_t(K), uint64_t(rows), uint64_t(batch)};
+  const uint64_t strides[2] = {uint64_t(K), uint64_t(batch > 1 ? bstride : K * rows)};
+  const uint32_t box[3] = {uint32_t(kBK), uint32_t(box_rows), 1u};
+  return encode_tiled_cached(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 // 3-D map over the bf16 output [batch, M, N] with a 32x32 box, 64B swizzle
 // (the staging-buffer layout the epilogue writes).
 bool make_out_map(CUtensorMap* m, uint16_t* base, int64_t M, int64_t N, int64_t batch, int64_t c_stride) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {cuuint64_t(N), cuuint64_t(M), cuuint64_t(batch)};
-  const cuuint64_t strides[2] = {cuuint64_t(N * 2), cuuint64_t((batch > 1 ? c_stride : M * N) * 2)};
-  const cuuint32_t box[3] = {32u, 32u, 1u};
-  const cuuint32_t estr[3] = {1u, 1u, 1u};
-  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
-                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
-                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  const uint64_t dims[3] = {uint64_t(N), uint64_t(M), uint64_t(batch)};
+  const uint64_t strides[2] = {uint64_t(N * 2), uint64_t((batch > 1 ? c_stride : M * N) * 2)};
+  const uint32_t box[3] = {32u, 32u, 1u};
+  return encode_tiled_cached(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE);
 }
 
 int sm_count() {

@@ -632,23 +632,14 @@ int dispatch_fmt_tile(int fmt, const TileArgs& a, int grid, cudaStream_t st, boo
                          : launch_tile<DT, FP8_E5M2>(a, grid, st, dual);
 }
 
-using EncodeTiledFnQ = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
 // 2-D map over the input [rows, cols] with a 128-row x 128-byte box, 128B swizzle.
 bool make_input_map(CUtensorMap* m, const void* in, int dtype, int64_t rows, int64_t cols) {
-  auto enc = reinterpret_cast<EncodeTiledFnQ>(tensor_map_encoder());
-  if (!enc) return false;
   const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
-  const cuuint64_t dims[2] = {cuuint64_t(cols), cuuint64_t(rows)};
-  const cuuint64_t strides[1] = {cuuint64_t(cols * eb)};
-  const cuuint32_t box[2] = {cuuint32_t(128 / eb), cuuint32_t(kTileR)};
-  const cuuint32_t estr[2] = {1u, 1u};
-  const CUtensorMapDataType dt = eb == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16;
-  return enc(m, dt, 2, const_cast<void*>(in), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const uint64_t dims[2] = {uint64_t(cols), uint64_t(rows)};
+  const uint64_t strides[1] = {uint64_t(cols * eb)};
+  const uint32_t box[2] = {uint32_t(128 / eb), uint32_t(kTileR)};
+  return encode_tiled_cached(m, eb == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, in,
+                             dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
 // Resident blocks per SM of a TMA tile kernel instantiation (cached per device).

@@ -83,14 +83,18 @@ def _check(rc, what):
         raise Fp8Error(rc, what)
 
 
-def _stream(stream):
+_raw_stream = torch._C._cuda_getCurrentRawStream
+
+
+def _stream(stream, device_index):
+    """Raw cudaStream_t (as an int) of ``stream`` or of the device's current stream."""
     if stream is None:
-        stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream)
+        return _raw_stream(device_index)
+    return stream.cuda_stream
 
 
 def _ptr(t):
-    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+    return t.data_ptr() if t is not None else None
 
 
 class Ring:
@@ -128,8 +132,11 @@ class Ring:
         return self.buf[19:21]
 
     def c(self):
-        base = self.buf.data_ptr()
-        return CRing(base, base + 16 * 4, base + 17 * 4, base + 18 * 4, base + 19 * 4)
+        c = getattr(self, "_c", None)
+        if c is None:
+            base = self.buf.data_ptr()
+            c = self._c = CRing(base, base + 16 * 4, base + 17 * 4, base + 18 * 4, base + 19 * 4)
+        return c
 
     def state(self):
         """Host copy: (history float32[16], idx, scale, scale_inv, scratch[2])."""
@@ -150,9 +157,10 @@ def quantize(x, fmt, layout, ring, out=None, out_t=None, stream=None):
         out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
     if layout in (TRANSPOSED, DUAL) and out_t is None:
         out_t = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
-    rc = lib().fp8_quantize(_ptr(x), IN_DTYPE[x.dtype], rows, cols, layout, fmt, ring.c(),
-                            _ptr(out if layout in (ROW, DUAL) else None),
-                            _ptr(out_t if layout in (TRANSPOSED, DUAL) else None), _stream(stream))
+    rc = (_LIB or lib()).fp8_quantize(x.data_ptr(), IN_DTYPE[x.dtype], rows, cols, layout, fmt, ring.c(),
+                                      _ptr(out if layout in (ROW, DUAL) else None),
+                                      _ptr(out_t if layout in (TRANSPOSED, DUAL) else None),
+                                      _stream(stream, x.get_device()))
     _check(rc, "fp8_quantize")
     return (out if layout in (ROW, DUAL) else None), (out_t if layout in (TRANSPOSED, DUAL) else None)
 
@@ -166,6 +174,24 @@ def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream
     """
     if a.dtype != torch.uint8 or b.dtype != torch.uint8:
         raise ValueError("a and b hold FP8 codes as uint8")
+    layout = MM_NT | (MM_A_E5M2 if fmt_a == E5M2 else 0) | (MM_B_E5M2 if fmt_b == E5M2 else 0)
+    L = _LIB or lib()
+    if a.dim() == 2 and b.dim() == 2:
+        M, K = a.shape
+        N = b.shape[0]
+        if b.shape[1] != K:
+            raise ValueError("K mismatch")
+        if K > 0 and ((M > 1 and a.stride(0) != K) or a.stride(1) != 1 or (N > 1 and b.stride(0) != K)
+                      or b.stride(1) != 1):
+            raise ValueError("operands must be K-contiguous")
+        if out is None:
+            out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+        elif not out.is_contiguous() or out.shape != (M, N):
+            raise ValueError("out must be a contiguous [M, N] bf16 tensor")
+        rc = L.fp8_mm(a.data_ptr(), b.data_ptr(), M, N, K, 1, None, layout, sinv_a.data_ptr(),
+                      sinv_b.data_ptr(), _ptr(bias), out.data_ptr(), _stream(stream, a.get_device()))
+        _check(rc, "fp8_mm")
+        return out
     a3 = a if a.dim() == 3 else a.unsqueeze(0)
     b3 = b if b.dim() == 3 else b.unsqueeze(0)
     batch = max(a3.shape[0], b3.shape[0])
@@ -173,21 +199,19 @@ def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream
     N = b3.shape[1]
     if b3.shape[2] != K:
         raise ValueError("K mismatch")
-    for t, n in ((a3, M * K), (b3, N * K)):
+    for t in (a3, b3):
         if t.shape[0] not in (1, batch) or (K > 0 and t.shape[1] > 1 and (t.stride(2) != 1 or t.stride(1) != K)):
             raise ValueError("operands must be K-contiguous with matching batch")
     sa = 0 if a3.shape[0] == 1 else a3.stride(0)
     sb = 0 if b3.shape[0] == 1 else b3.stride(0)
-    squeeze = a.dim() == 2 and b.dim() == 2
     if out is None:
         out = torch.empty((batch, M, N), dtype=torch.bfloat16, device=a.device)
     out3 = out if out.dim() == 3 else out.unsqueeze(0)
     strides = (ctypes.c_int64 * 3)(sa, sb, out3.stride(0) if batch > 1 else M * N)
-    layout = MM_NT | (MM_A_E5M2 if fmt_a == E5M2 else 0) | (MM_B_E5M2 if fmt_b == E5M2 else 0)
-    rc = lib().fp8_mm(_ptr(a3), _ptr(b3), M, N, K, batch, strides, layout, _ptr(sinv_a), _ptr(sinv_b),
-                      _ptr(bias), _ptr(out3), _stream(stream))
+    rc = L.fp8_mm(a3.data_ptr(), b3.data_ptr(), M, N, K, batch, strides, layout, sinv_a.data_ptr(),
+                  sinv_b.data_ptr(), _ptr(bias), out3.data_ptr(), _stream(stream, a.get_device()))
     _check(rc, "fp8_mm")
-    return out3[0] if squeeze and out.dim() == 3 else out
+    return out
 
 
 def device_error(clear=True):

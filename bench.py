@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--sweep", choices=["gemm", "quantize"], default=None,
                     help="per-shape kernel rows instead of the step line")
     ap.add_argument("--iters", type=int, default=50)
+    ap.add_argument("--profile", action="store_true",
+                    help="warm up, run exactly one step inside the NVTX range fp8_profile_step, exit (for ncu)")
     ap.add_argument("--shapes", default=None, help="sweep subset, e.g. 8192x8192x8192,64x8192x2048")
     return ap.parse_args()
 
@@ -382,6 +384,13 @@ def main():
     for i in range(max(3, args.warmup)):
         run_step(lins, ops, i)
     torch.cuda.synchronize()
+    if args.profile:
+        torch.cuda.nvtx.range_push("fp8_profile_step")
+        run_step(lins, ops, 0)
+        torch.cuda.nvtx.range_pop()
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_step": "done", "M": M, "launches": 12}))
+        return 0
     q_ms, g_ms = time_split(lins, ops, torch, 50)
 
     # The timed steps replay a CUDA graph of two consecutive steps (one per

@@ -48,17 +48,22 @@ constexpr int kEpiWarps = 8;      // two warps per TMEM lane quadrant, each owni
 constexpr int kThreadsMM = 32 * (2 + kEpiWarps);
 constexpr int kStagingBytes = 2048;  // one 32x32 bf16 box per staging buffer
 
-template <int BN>
+// PAIR = 1: one CTA computes a 128 x BN tile.  PAIR = 2: a cluster of two
+// CTAs on two SMs computes a 256 x BN tile with tcgen05 cta_group::2; each CTA
+// holds 128 rows of A, BN/2 rows of B and its 128 x BN half of the accumulator.
+template <int BN, int PAIR>
 struct Cfg {
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kBRows = BN / PAIR;
   static constexpr int kABytes = kBM * kBK;
-  static constexpr int kBBytes = BN * kBK;
+  static constexpr int kBBytes = kBRows * kBK;
   static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (192 * 1024) / kStageBytes;
   static constexpr int kTmemCols = 2 * BN;  // two accumulators
   static constexpr int kStagingOffset = kStages * kStageBytes;  // 2 buffers per epilogue warp
   static constexpr int kBarOffset = kStagingOffset + kEpiWarps * 2 * kStagingBytes;
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(2 * kStages + 5 <= 28, "barrier area");
 };
 
 struct MmParams {
@@ -154,6 +159,87 @@ __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+// TMA load whose completion is counted on the leader CTA's barrier (bar is a
+// shared::cluster address).  No multicast.
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+      : "memory");
+}
+
+template <int PAIR>
+__device__ __forceinline__ void tmem_alloc_g(uint32_t slot, uint32_t ncols) {
+  if constexpr (PAIR == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  } else {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+}
+
+template <int PAIR>
+__device__ __forceinline__ void tmem_dealloc_g(uint32_t taddr, uint32_t ncols) {
+  if constexpr (PAIR == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+  } else {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+  }
+}
+
+// cta_group::2 MMA issued by the leader CTA: A rows 0..127 and B rows 0..BN/2-1
+// come from the leader's shared memory, the other halves from the peer's at
+// the same offsets; D rows 0..127 land in the leader's TMEM, 128..255 in the peer's.
+__device__ __forceinline__ void umma_f8_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrive once on the barrier at offset `bar` in both CTAs of the pair when all
+// prior MMAs of this thread complete.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(uint16_t(3))
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_pair_local(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
   asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
@@ -220,13 +306,14 @@ __device__ __forceinline__ void decode_tile(const MmParams& p, int t, int& b, in
   nt = rr / gm;
 }
 
-template <int BN>
+template <int BN, int PAIR>
 __global__ void __launch_bounds__(kThreadsMM, 1)
     mm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const MmParams p) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, PAIR>;
+  constexpr int kTileM = kBM * PAIR;
   extern __shared__ uint8_t smem_raw[];
-  // 1024-byte alignment for the swizzled tiles.
+  // 1024-byte alignment for the swizzled tiles (the same offset in both CTAs of a pair).
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* smem = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
   const uint32_t sbase = smem_u32(smem);
@@ -243,6 +330,10 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit0 = int(blockIdx.x) / PAIR;   // this CTA's (pair's) first tile
+  const int units = int(gridDim.x) / PAIR;    // tiles advance by the number of CTAs (pairs)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -251,7 +342,7 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(tfull_bar(a), 1);
-      mbar_init(tempty_bar(a), kEpiWarps);
+      mbar_init(tempty_bar(a), kEpiWarps * PAIR);
     }
     mbar_init(done_bar, 1);
     *abort = 0;
@@ -263,34 +354,46 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
     prefetch_tmap(&tmB);
     if (p.tma_store) prefetch_tmap(&tmC);
   }
-  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), C::kTmemCols);
+  if constexpr (PAIR == 2) cluster_sync();  // the peer's barriers exist before any remote arrive
+  if (warp == 1) tmem_alloc_g<PAIR>(smem_u32(tmem_slot), C::kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs of a pair) ----------------
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;  // bit s: stage s armed; its parity
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < p.tiles_total; t += gridDim.x) {
+      for (int t = unit0; ok && t < p.tiles_total; t += units) {
         int b, mt, nt;
         decode_tile(p, t, b, mt, nt);
         const int ba = p.a_bcast ? 0 : b;
         const int bb = p.b_bcast ? 0 : b;
+        const int arow = mt * kTileM + int(rank) * kBM;
+        const int brow = nt * BN + int(rank) * C::kBRows;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort, p.err, kWaitProducerEmpty)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
           const uint32_t sa = sbase + stage * C::kABytes;
           const uint32_t sb = sbase + C::kStages * C::kABytes + stage * C::kBBytes;
-          tma_load_3d(sa, &tmA, kb * kBK, mt * kBM, ba, full_bar(stage));
-          tma_load_3d(sb, &tmB, kb * kBK, nt * BN, bb, full_bar(stage));
+          if constexpr (PAIR == 1) {
+            mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
+            tma_load_3d(sa, &tmA, kb * kBK, arow, ba, full_bar(stage));
+            tma_load_3d(sb, &tmB, kb * kBK, brow, bb, full_bar(stage));
+          } else {
+            // Both CTAs' loads complete on the leader's barrier; the leader
+            // expects the bytes of both.
+            if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * C::kStageBytes);
+            const uint32_t lbar = mapa_shared(full_bar(stage), 0);
+            tma_load_3d_pair(sa, &tmA, kb * kBK, arow, ba, lbar);
+            tma_load_3d_pair(sb, &tmB, kb * kBK, brow, bb, lbar);
+          }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           if (++stage == C::kStages) {
@@ -299,8 +402,8 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
           }
         }
       }
-      if (!ok) {
-        // Let every copy this thread issued land before shared memory is released.
+      if (!ok && leader) {
+        // Let every copy armed on this barrier land before shared memory is released.
         for (int s = 0; s < C::kStages; ++s)
           if (armed & (1u << s)) {
             const unsigned long long t0 = globaltimer_ns();
@@ -311,15 +414,15 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
+    // ---------------- MMA issuer (leader CTA only) ----------------
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int i = 0;
       bool ok = true;
       const uint32_t sa0 = sbase;
       const uint32_t sb0 = sbase + C::kStages * C::kABytes;
-      for (int t = blockIdx.x; ok && t < p.tiles_total; t += gridDim.x, ++i) {
+      for (int t = unit0; ok && t < p.tiles_total; t += units, ++i) {
         const int acc = i & 1;
         const uint32_t acc_par = (i >> 1) & 1;
         if (!mbar_wait(tempty_bar(acc), acc_par ^ 1u, abort, p.err, kWaitMmaTmemEmpty)) break;
@@ -336,34 +439,39 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k) {
             // +32 bytes along K inside the swizzle atom = +2 in the address field.
-            umma_f8(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), p.idesc, (kb | k) != 0 ? 1u : 0u);
+            if constexpr (PAIR == 1)
+              umma_f8(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), p.idesc, (kb | k) != 0 ? 1u : 0u);
+            else
+              umma_f8_pair(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), p.idesc, (kb | k) != 0 ? 1u : 0u);
           }
-          umma_commit(empty_bar(stage));
+          if constexpr (PAIR == 1) umma_commit(empty_bar(stage));
+          else umma_commit_pair(empty_bar(stage));
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
-        if (p.k_blocks > 0) umma_commit(tfull_bar(acc));
-        else mbar_arrive(tfull_bar(acc));
+        if constexpr (PAIR == 1) umma_commit(tfull_bar(acc));
+        else umma_commit_pair(tfull_bar(acc));
       }
       // All MMAs this thread issued are complete before TMEM is released.
-      umma_commit(done_bar);
+      if constexpr (PAIR == 1) umma_commit(done_bar);
+      else umma_commit_pair_local(done_bar);
       const unsigned long long t0 = globaltimer_ns();
       while (!mbar_try_wait(done_bar, 0) && globaltimer_ns() - t0 < kWaitBudgetNs) {
       }
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..9) ----------------
-    // Warp w reads TMEM lane quadrant w % 4 (rows 32*(w%4) .. +31 of the tile)
-    // and half (w-2)/4 of the columns.  Two 32-column chunks are loaded per
-    // tcgen05.wait::ld; the accumulator is released to the MMA warp as soon
-    // as its last chunk is in registers.  Results leave through 32x32 bf16
-    // TMA stores from two 64B-swizzled staging buffers per warp (rows of
-    // 64 bytes, 16-byte unit j of row r at unit j ^ ((r >> 1) & 3)), or,
-    // when the output rows are not 16-byte aligned, through guarded stores.
+    // ---------------- epilogue (warps 2..9 of each CTA) ----------------
+    // Warp w reads TMEM lane quadrant w % 4 (rows 32*(w%4) .. +31 of this
+    // CTA's 128-row half) and half (w-2)/4 of the columns.  Two 32-column
+    // chunks are loaded per tcgen05.wait::ld; the accumulator is released to
+    // the MMA issuer as soon as its last chunk is in registers.  Results leave
+    // through 32x32 bf16 TMA stores from two 64B-swizzled staging buffers per
+    // warp (rows of 64 bytes, 16-byte unit j of row r at unit j ^ ((r>>1)&3)),
+    // or, when output rows are not 16-byte aligned, through guarded stores.
     const int ew = warp - 2;
     const int quad = warp & 3;
     const int half = ew >> 2;
@@ -372,18 +480,19 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
     const uint32_t stage0 = sbase + C::kStagingOffset + uint32_t(ew) * 2u * kStagingBytes;
     int buf = 0;
     int i = 0;
-    for (int t = blockIdx.x; t < p.tiles_total; t += gridDim.x, ++i) {
+    for (int t = unit0; t < p.tiles_total; t += units, ++i) {
       const int acc = i & 1;
       const uint32_t acc_par = (i >> 1) & 1;
       if (!mbar_wait(tfull_bar(acc), acc_par, abort, p.err, kWaitEpilogueTmemFull)) break;
       tc_fence_after();
       int b, mt, nt;
       decode_tile(p, t, b, mt, nt);
-      const int m0 = mt * kBM + quad * 32;
+      const int m0 = mt * kTileM + int(rank) * kBM + quad * 32;
       const int row = m0 + lane;
       uint16_t* orow = p.out + int64_t(b) * p.c_stride + int64_t(row) * p.N;
       const uint32_t tbase = tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + half * kHalfCols);
       const int nbase = nt * BN + half * kHalfCols;
+      const uint32_t release_bar = PAIR == 1 ? tempty_bar(acc) : mapa_shared(tempty_bar(acc), 0);
       bool released = false;
 #pragma unroll 1
       for (int c = 0; c < kHalfCols / 32; c += 2) {
@@ -396,7 +505,7 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
           // Last TMEM read of this tile for this warp: hand the accumulator back.
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(tempty_bar(acc));
+          if (lane == 0) mbar_arrive_cluster(release_bar);
           released = true;
         }
 #pragma unroll
@@ -465,7 +574,7 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
       if (!released) {
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(tempty_bar(acc));
+        if (lane == 0) mbar_arrive_cluster(release_bar);
       }
     }
     if (p.tma_store && lane == 0) bulk_wait_all();
@@ -474,8 +583,11 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
 
   tc_fence_before();
   __syncthreads();
+  // A pair leaves together: the leader's MMAs read the peer's shared memory
+  // and write the peer's TMEM until done_bar fired.
+  if constexpr (PAIR == 2) cluster_sync();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem_base, C::kTmemCols);
+  if (warp == 1) tmem_dealloc_g<PAIR>(tmem_base, C::kTmemCols);
 }
 
 // K == 0: Y = bf16(bias) or 0.
@@ -523,42 +635,119 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int BN>
+template <int BN, int PAIR>
 bool ensure_smem_attr() {
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(mm_fp8_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg<BN>::kSmemBytes) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(mm_fp8_kernel<BN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg<BN, PAIR>::kSmemBytes) != cudaSuccess)
       return false;
     done[dev] = true;
   }
   return true;
 }
 
+// CTA pairs that can be resident at once (one pair per two SMs at best).
 template <int BN>
+int max_pairs(int sms) {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return sms / 2;
+  if (cached[dev] == 0) {
+    if (!ensure_smem_attr<BN, 2>()) return sms / 2;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (sms / 2));
+    cfg.blockDim = dim3(kThreadsMM);
+    cfg.dynamicSmemBytes = Cfg<BN, 2>::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, mm_fp8_kernel<BN, 2>, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = sms / 2;
+    }
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+template <int BN, int PAIR>
 int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
-              const int64_t* strides, MmParams p, int sms, cudaStream_t st) {
+              const int64_t* strides, MmParams p, int slots, cudaStream_t st) {
   CUtensorMap ta, tb, tc;
   const int64_t ba = (batch > 1 && strides[0] != 0) ? batch : 1;
   const int64_t bb = (batch > 1 && strides[1] != 0) ? batch : 1;
   if (!make_map(&ta, A, K, M, ba, ba > 1 ? strides[0] : 0, kBM)) return FP8_ERR_CUDA;
-  if (!make_map(&tb, B, K, N, bb, bb > 1 ? strides[1] : 0, BN)) return FP8_ERR_CUDA;
+  if (!make_map(&tb, B, K, N, bb, bb > 1 ? strides[1] : 0, BN / PAIR)) return FP8_ERR_CUDA;
   memset(&tc, 0, sizeof(tc));
   if (p.tma_store && !make_out_map(&tc, p.out, M, N, batch, p.c_stride)) return FP8_ERR_CUDA;
   p.a_bcast = ba == 1;
   p.b_bcast = bb == 1;
-  p.m_tiles = int((M + kBM - 1) / kBM);
+  p.m_tiles = int((M + kBM * PAIR - 1) / (kBM * PAIR));
   p.n_tiles = int((N + BN - 1) / BN);
   p.tiles_per_batch = p.m_tiles * p.n_tiles;
   p.tiles_total = int(p.tiles_per_batch * batch);
   p.group_m = 8;
-  p.idesc |= uint32_t(BN >> 3) << 17;
-  if (!ensure_smem_attr<BN>()) return FP8_ERR_CUDA;
-  const int grid = std::max(1, std::min(p.tiles_total, sms));
-  mm_fp8_kernel<BN><<<grid, kThreadsMM, Cfg<BN>::kSmemBytes, st>>>(ta, tb, tc, p);
-  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+  p.idesc |= (uint32_t(BN >> 3) << 17) | (uint32_t((kBM * PAIR) >> 4) << 24);
+  if (!ensure_smem_attr<BN, PAIR>()) return FP8_ERR_CUDA;
+  const int units = std::max(1, std::min(p.tiles_total, slots));
+  if constexpr (PAIR == 1) {
+    mm_fp8_kernel<BN, 1><<<units, kThreadsMM, Cfg<BN, 1>::kSmemBytes, st>>>(ta, tb, tc, p);
+    return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * units);
+    cfg.blockDim = dim3(kThreadsMM);
+    cfg.dynamicSmemBytes = Cfg<BN, 2>::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, mm_fp8_kernel<BN, 2>, ta, tb, tc, p) == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+  }
+}
+
+// Tile-shape choice: time ~ waves x per-SM tile width / relative efficiency,
+// over {one CTA, CTA pair} x {BN 256, 128}.  A pair halves each SM's share of
+// the B operand in shared memory and the L2 traffic per flop.
+struct MmChoice {
+  int bn, pair, slots;
+};
+
+MmChoice choose_mm(int64_t M, int64_t N, int64_t batch, int sms) {
+  struct Opt {
+    int bn, pair;
+    double eff;
+  };
+  // Relative per-SM MMA efficiency measured on B200: a 128-wide MMA issues at
+  // about the rate of a 256-wide one, so BN = 128 does half the work per
+  // instruction whether or not the CTAs are paired.
+  const Opt opts[4] = {{256, 2, 1.0}, {256, 1, 0.85}, {128, 2, 0.5}, {128, 1, 0.45}};
+  MmChoice best{256, 1, sms};
+  double best_cost = 1e300;
+  for (const Opt& o : opts) {
+    if (o.pair == 2 && M <= kBM) continue;  // the second CTA would hold no rows
+    const int slots = o.pair == 2 ? (o.bn == 256 ? max_pairs<256>(sms) : max_pairs<128>(sms)) : sms;
+    const int64_t units = ((M + kBM * o.pair - 1) / (kBM * o.pair)) * ((N + o.bn - 1) / o.bn) * batch;
+    const double waves = double((units + slots - 1) / slots);
+    const double cost = waves * o.bn / o.eff;
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = MmChoice{o.bn, o.pair, slots};
+    }
+  }
+  return best;
 }
 
 }  // namespace
@@ -610,12 +799,16 @@ extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, 
   const uint32_t fa = (layout & FP8_MM_A_E5M2) ? 1u : 0u;
   const uint32_t fb = (layout & FP8_MM_B_E5M2) ? 1u : 0u;
   // Instruction descriptor: fp32 accumulator (bits 4-5 = 1), A format bits 7-9,
-  // B format bits 10-12 (0 = E4M3, 1 = E5M2), both K-major, M/16 at bits 24-28;
-  // N/8 (bits 17-22) is added by the launcher for its tile width.
-  p.idesc = (1u << 4) | (fa << 7) | (fb << 10) | (uint32_t(kBM >> 4) << 24);
+  // B format bits 10-12 (0 = E4M3, 1 = E5M2), both K-major; N/8 (bits 17-22)
+  // and M/16 (bits 24-28) are added by the launcher for its tile shape.
+  p.idesc = (1u << 4) | (fa << 7) | (fb << 10);
   p.err = error_word_ptr();
 
-  const int64_t tiles256 = ((M + kBM - 1) / kBM) * ((N + 255) / 256) * batch;
-  if (N > 128 && tiles256 >= sms) return launch_mm<256>(A, B, M, N, K, batch, strides, p, sms, st);
-  return launch_mm<128>(A, B, M, N, K, batch, strides, p, sms, st);
+  const MmChoice c = choose_mm(M, N, batch, sms);
+  if (c.pair == 2) {
+    if (c.bn == 256) return launch_mm<256, 2>(A, B, M, N, K, batch, strides, p, c.slots, st);
+    return launch_mm<128, 2>(A, B, M, N, K, batch, strides, p, c.slots, st);
+  }
+  if (c.bn == 256) return launch_mm<256, 1>(A, B, M, N, K, batch, strides, p, c.slots, st);
+  return launch_mm<128, 1>(A, B, M, N, K, batch, strides, p, c.slots, st);
 }

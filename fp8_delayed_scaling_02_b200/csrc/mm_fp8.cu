@@ -330,6 +330,7 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_launch_dependents();
   const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
   const int unit0 = int(blockIdx.x) / PAIR;   // this CTA's (pair's) first tile
@@ -360,6 +361,7 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait_prior_grid();  // inputs, scales and the output buffer belong to earlier work until here
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs of a pair) ----------------
@@ -488,8 +490,6 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
       int b, mt, nt;
       decode_tile(p, t, b, mt, nt);
       const int m0 = mt * kTileM + int(rank) * kBM + quad * 32;
-      const int row = m0 + lane;
-      uint16_t* orow = p.out + int64_t(b) * p.c_stride + int64_t(row) * p.N;
       const uint32_t tbase = tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + half * kHalfCols);
       const int nbase = nt * BN + half * kHalfCols;
       const uint32_t release_bar = PAIR == 1 ? tempty_bar(acc) : mapa_shared(tempty_bar(acc), 0);
@@ -557,17 +557,31 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
               }
               buf ^= 1;
             }
-          } else if (row < p.M) {
-            if (full && p.out_vec) {
-              uint4* o = reinterpret_cast<uint4*>(orow + n0);
+          } else if (m0 < p.M) {
+            // Rows not 16-byte aligned: stage the 32x32 chunk in the same
+            // swizzled layout, then write it row by row, lane l taking column
+            // n0 + l, so each store instruction covers 64 contiguous bytes.
+            const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
+            __syncwarp();
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                o[j] = make_uint4(packed[4 * j], packed[4 * j + 1], packed[4 * j + 2], packed[4 * j + 3]);
-            } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (n0 + j < p.N) orow[n0 + j] = uint16_t(packed[j >> 1] >> (16 * (j & 1)));
+            for (int u = 0; u < 4; ++u) {
+              const uint32_t addr = sbuf + uint32_t(lane) * 64u + uint32_t((u ^ ((lane >> 1) & 3)) * 16);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[4 * u]),
+                           "r"(packed[4 * u + 1]), "r"(packed[4 * u + 2]), "r"(packed[4 * u + 3])
+                           : "memory");
             }
+            __syncwarp();
+            const bool col_ok = n0 + lane < p.N;
+            uint16_t* obase = p.out + int64_t(b) * p.c_stride + int64_t(m0) * p.N + n0 + lane;
+#pragma unroll 4
+            for (int rr = 0; rr < 32; ++rr) {
+              const uint32_t addr = sbuf + uint32_t(rr) * 64u + uint32_t((((lane >> 3) ^ ((rr >> 1) & 3)) << 4)) +
+                                    uint32_t((lane & 7) << 1);
+              uint16_t v;
+              asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+              if (col_ok && m0 + rr < p.M) obase[int64_t(rr) * p.N] = v;
+            }
+            buf ^= 1;
           }
         }
       }
@@ -593,6 +607,8 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
 // K == 0: Y = bf16(bias) or 0.
 __global__ void mm_bias_only_kernel(uint16_t* out, const float* bias, int64_t M, int64_t N, int64_t batch,
                                     int64_t c_stride) {
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
   const int64_t total = batch * M * N;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t b = i / (M * N), r = i - b * M * N, n = r % N;
@@ -698,24 +714,9 @@ int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t 
   p.idesc |= (uint32_t(BN >> 3) << 17) | (uint32_t((kBM * PAIR) >> 4) << 24);
   if (!ensure_smem_attr<BN, PAIR>()) return FP8_ERR_CUDA;
   const int units = std::max(1, std::min(p.tiles_total, slots));
-  if constexpr (PAIR == 1) {
-    mm_fp8_kernel<BN, 1><<<units, kThreadsMM, Cfg<BN, 1>::kSmemBytes, st>>>(ta, tb, tc, p);
-    return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(2 * units);
-    cfg.blockDim = dim3(kThreadsMM);
-    cfg.dynamicSmemBytes = Cfg<BN, 2>::kSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, mm_fp8_kernel<BN, 2>, ta, tb, tc, p) == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
-  }
+  const cudaError_t e = launch_pdl(mm_fp8_kernel<BN, PAIR>, dim3(PAIR * units), dim3(kThreadsMM),
+                                   Cfg<BN, PAIR>::kSmemBytes, st, PAIR, ta, tb, tc, p);
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 // Tile-shape choice: time ~ waves x per-SM tile width / relative efficiency,
@@ -774,8 +775,9 @@ extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, 
   if (K == 0) {
     const int64_t total = batch * M * N;
     const int grid = int(std::min<int64_t>((total + 255) / 256, 4096));
-    mm_bias_only_kernel<<<grid, 256, 0, st>>>(out_bf16, bias, M, N, batch, c_stride);
-    return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+    const cudaError_t e = launch_pdl(mm_bias_only_kernel, dim3(grid), dim3(256), 0, st, 1, out_bf16, bias, M, N,
+                                     batch, c_stride);
+    return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
   }
   if (reinterpret_cast<uintptr_t>(A) % 16 != 0 || reinterpret_cast<uintptr_t>(B) % 16 != 0) return FP8_ERR_UNSUPPORTED;
   if (batch > 1 && ((strides[0] % 16) != 0 || (strides[1] % 16) != 0)) return FP8_ERR_UNSUPPORTED;

@@ -269,6 +269,8 @@ __device__ __forceinline__ void row_chunk(const RowArgs& a, int64_t j, float s, 
 template <int DT, int FMT, bool kAligned>
 __global__ void __launch_bounds__(kThreads) quantize_row_kernel(const RowArgs a) {
   constexpr int kB = In<DT>::kBytes;
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
   const float s = *a.ring.scale;
   const RingCache rc = prefetch_ring(a.ring);
   float amax = 0.0f;
@@ -317,6 +319,8 @@ template <int DT, int FMT, bool kDual>
 __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs a) {
   constexpr int kB = In<DT>::kBytes;
   __shared__ uint32_t sT[kTileC * kPitchW];
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
   const float s = *a.ring.scale;
   const RingCache rc = prefetch_ring(a.ring);
   float amax = 0.0f;
@@ -469,9 +473,7 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
   uint64_t* bars = reinterpret_cast<uint64_t*>(sT + kTileC * kPitchW);
   const uint32_t bar0 = smem_addr(bars);
 
-  const float s = *a.ring.scale;
-  const RingCache rc = prefetch_ring(a.ring);
-  float amax = 0.0f;
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int lr0 = 32 * (warp & 3) + 4 * (lane & 7);
   const int lc0 = 32 * (warp >> 2) + 8 * (lane >> 3);
@@ -484,6 +486,10 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmIn)) : "memory");
   }
   __syncthreads();
+  pdl_wait_prior_grid();
+  const float s = *a.ring.scale;
+  const RingCache rc = prefetch_ring(a.ring);
+  float amax = 0.0f;
   int64_t issued = 0;  // tiles of this block whose loads thread 0 has issued
   if (threadIdx.x == 0) {
     for (int i = 0; i < TT::kStages; ++i) {
@@ -608,16 +614,16 @@ int sm_count_current() {
 
 template <int DT, int FMT>
 int launch_row(const RowArgs& a, int grid, cudaStream_t st, bool aligned) {
-  if (aligned) quantize_row_kernel<DT, FMT, true><<<grid, kThreads, 0, st>>>(a);
-  else quantize_row_kernel<DT, FMT, false><<<grid, kThreads, 0, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+  const cudaError_t e = aligned ? launch_pdl(quantize_row_kernel<DT, FMT, true>, grid, kThreads, 0, st, 1, a)
+                                : launch_pdl(quantize_row_kernel<DT, FMT, false>, grid, kThreads, 0, st, 1, a);
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 template <int DT, int FMT>
 int launch_tile(const TileArgs& a, int grid, cudaStream_t st, bool dual) {
-  if (dual) quantize_tile_kernel<DT, FMT, true><<<grid, kThreads, 0, st>>>(a);
-  else quantize_tile_kernel<DT, FMT, false><<<grid, kThreads, 0, st>>>(a);
-  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+  const cudaError_t e = dual ? launch_pdl(quantize_tile_kernel<DT, FMT, true>, grid, kThreads, 0, st, 1, a)
+                             : launch_pdl(quantize_tile_kernel<DT, FMT, false>, grid, kThreads, 0, st, 1, a);
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 template <int DT>
@@ -666,9 +672,10 @@ int launch_tile_tma(const TileArgs& t, const CUtensorMap& map, int sms, cudaStre
   const int bps = dual ? tma_blocks_per_sm<DT, FMT, true>() : tma_blocks_per_sm<DT, FMT, false>();
   if (bps <= 0) return FP8_ERR_CUDA;
   const int grid = int(std::max<int64_t>(1, std::min<int64_t>(t.ntiles, int64_t(bps) * sms)));
-  if (dual) quantize_tile_tma_kernel<DT, FMT, true><<<grid, kThreads, TmaTile<DT>::kSmem, st>>>(map, a);
-  else quantize_tile_tma_kernel<DT, FMT, false><<<grid, kThreads, TmaTile<DT>::kSmem, st>>>(map, a);
-  return cudaGetLastError() == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+  const cudaError_t e =
+      dual ? launch_pdl(quantize_tile_tma_kernel<DT, FMT, true>, grid, kThreads, TmaTile<DT>::kSmem, st, 1, map, a)
+           : launch_pdl(quantize_tile_tma_kernel<DT, FMT, false>, grid, kThreads, TmaTile<DT>::kSmem, st, 1, map, a);
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 template <int DT>

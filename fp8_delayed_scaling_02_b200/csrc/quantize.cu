@@ -157,19 +157,58 @@ __device__ __forceinline__ void load_vec_aligned(const uint8_t* p, float (&v)[N]
 
 // ---- conversion ------------------------------------------------------------
 
-// fp8 codes of (lo*s, hi*s) packed low byte first: one fp32 multiply each (no
-// contraction), then the hardware round-to-nearest-even conversion with
-// saturation to the largest finite value.
+// (a*s, b*s) with one packed fp32x2 multiply, each lane rounded to nearest
+// even exactly as a scalar fp32 multiply (no contraction into anything else).
+__device__ __forceinline__ void scale2(float& a, float& b, float s) {
+  asm("{\n\t.reg .b64 ra, rs, rd;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rs, {%2, %2};\n\t"
+      "mul.rn.f32x2 rd, ra, rs;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(s));
+}
+
+// fp8 codes of two already-scaled values packed low byte first: the hardware
+// round-to-nearest-even conversion with saturation to the largest finite value.
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
+  return uint32_t(
+      __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, FMT == FP8_E4M3 ? __NV_E4M3 : __NV_E5M2));
+}
+
+// Codes of v[0..3] * s in one word (v[0] in the low byte).
+template <int FMT>
+__device__ __forceinline__ uint32_t cvt4(float v0, float v1, float v2, float v3, float s) {
+  scale2(v0, v1, s);
+  scale2(v2, v3, s);
+  return __byte_perm(cvt2<FMT>(v0, v1), cvt2<FMT>(v2, v3), 0x5410);
+}
+
 template <int FMT>
 __device__ __forceinline__ uint32_t cvt_pair(float lo, float hi, float s) {
-  float2 f = make_float2(__fmul_rn(lo, s), __fmul_rn(hi, s));
-  return uint32_t(__nv_cvt_float2_to_fp8x2(f, __NV_SATFINITE, FMT == FP8_E4M3 ? __NV_E4M3 : __NV_E5M2));
+  scale2(lo, hi, s);
+  return cvt2<FMT>(lo, hi);
 }
 
 template <int FMT>
 __device__ __forceinline__ uint8_t cvt_one(float x, float s) {
   return uint8_t(__nv_cvt_float_to_fp8(__fmul_rn(x, s), __NV_SATFINITE,
                                        FMT == FP8_E4M3 ? __NV_E4M3 : __NV_E5M2));
+}
+
+// 4x4 byte transpose: word r holds bytes (r, 0..3); output word c holds bytes
+// (0..3, c), i.e. byte r of c_out is byte c of r_in.  Eight byte permutes.
+__device__ __forceinline__ void transpose4x4(uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3, uint32_t& c0,
+                                             uint32_t& c1, uint32_t& c2, uint32_t& c3) {
+  const uint32_t t0 = __byte_perm(r0, r1, 0x5140);  // r0.b0 r1.b0 r0.b1 r1.b1
+  const uint32_t t1 = __byte_perm(r0, r1, 0x7362);  // r0.b2 r1.b2 r0.b3 r1.b3
+  const uint32_t t2 = __byte_perm(r2, r3, 0x5140);
+  const uint32_t t3 = __byte_perm(r2, r3, 0x7362);
+  c0 = __byte_perm(t0, t2, 0x5410);
+  c1 = __byte_perm(t0, t2, 0x7632);
+  c2 = __byte_perm(t1, t3, 0x5410);
+  c3 = __byte_perm(t1, t3, 0x7632);
 }
 
 // ---- amax + ring fold --------------------------------------------------------
@@ -254,15 +293,11 @@ __device__ __forceinline__ void row_chunk(const RowArgs& a, int64_t j, float s, 
   float v[16];
   if constexpr (kAligned) load_vec_aligned<DT, 16>(a.in + e * kB, v);
   else load_vec<DT, 16>(a.in + e * kB, v);
-  uint32_t w[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t p0 = cvt_pair<FMT>(v[4 * i], v[4 * i + 1], s);
-    uint32_t p1 = cvt_pair<FMT>(v[4 * i + 2], v[4 * i + 3], s);
-    w[i] = p0 | (p1 << 16);
-  }
 #pragma unroll
   for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+  uint32_t w[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) w[i] = cvt4<FMT>(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3], s);
   *reinterpret_cast<uint4*>(a.out + e) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
@@ -347,8 +382,8 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs 
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
-      q[i][0] = cvt_pair<FMT>(v[0], v[1], s) | (cvt_pair<FMT>(v[2], v[3], s) << 16);
-      q[i][1] = cvt_pair<FMT>(v[4], v[5], s) | (cvt_pair<FMT>(v[6], v[7], s) << 16);
+      q[i][0] = cvt4<FMT>(v[0], v[1], v[2], v[3], s);
+      q[i][1] = cvt4<FMT>(v[4], v[5], v[6], v[7], s);
       if constexpr (kDual) {
         uint8_t* o = a.out + r * a.cols + c;
         if (interior && a.out8) {
@@ -362,11 +397,11 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs 
     }
     __syncthreads();  // previous tile's readers are done with sT
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int sh = 8 * (j & 3);
-      const uint32_t w = ((q[0][j >> 2] >> sh) & 0xFFu) | (((q[1][j >> 2] >> sh) & 0xFFu) << 8) |
-                         (((q[2][j >> 2] >> sh) & 0xFFu) << 16) | (((q[3][j >> 2] >> sh) & 0xFFu) << 24);
-      sT[(lc0 + j) * kPitchW + (lr0 >> 2)] = w;
+    for (int h = 0; h < 2; ++h) {
+      uint32_t c[4];
+      transpose4x4(q[0][h], q[1][h], q[2][h], q[3][h], c[0], c[1], c[2], c[3]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sT[(lc0 + 4 * h + k) * kPitchW + (lr0 >> 2)] = c[k];
     }
     __syncthreads();
 #pragma unroll
@@ -531,8 +566,8 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
       }
 #pragma unroll
       for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
-      q[i][0] = cvt_pair<FMT>(v[0], v[1], s) | (cvt_pair<FMT>(v[2], v[3], s) << 16);
-      q[i][1] = cvt_pair<FMT>(v[4], v[5], s) | (cvt_pair<FMT>(v[6], v[7], s) << 16);
+      q[i][0] = cvt4<FMT>(v[0], v[1], v[2], v[3], s);
+      q[i][1] = cvt4<FMT>(v[4], v[5], v[6], v[7], s);
     }
     // Every thread is done with this stage and with the previous tile's sT.
     if (!__syncthreads_and(ok ? 1 : 0)) {
@@ -563,11 +598,11 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
       }
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int sh = 8 * (j & 3);
-      const uint32_t w = ((q[0][j >> 2] >> sh) & 0xFFu) | (((q[1][j >> 2] >> sh) & 0xFFu) << 8) |
-                         (((q[2][j >> 2] >> sh) & 0xFFu) << 16) | (((q[3][j >> 2] >> sh) & 0xFFu) << 24);
-      sT[(lc0 + j) * kPitchW + (lr0 >> 2)] = w;
+    for (int h = 0; h < 2; ++h) {
+      uint32_t c[4];
+      transpose4x4(q[0][h], q[1][h], q[2][h], q[3][h], c[0], c[1], c[2], c[3]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) sT[(lc0 + 4 * h + k) * kPitchW + (lr0 >> 2)] = c[k];
     }
     __syncthreads();
 #pragma unroll

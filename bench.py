@@ -337,6 +337,28 @@ def sweep(args):
     return 0
 
 
+def measured_traffic():
+    """DRAM bytes per step of the 6 GEMM launches from the committed ncu summary,
+    or None if the GEMM source changed since that capture."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", "traffic_linear_1p2b_M8192.txt")
+    src = os.path.join(ROOT, "fp8_delayed_scaling_02_b200", "csrc", "mm_fp8.cu")
+    try:
+        kv = {}
+        for line in open(path):
+            line = line.split("#", 1)[0].strip()
+            if "=" in line:
+                k, v = line.split("=", 1)
+                kv[k.strip()] = v.strip()
+        sha = hashlib.sha1(open(src, "rb").read()).hexdigest()
+        if kv.get("mm_fp8_cu_sha1") != sha:
+            return None
+        return int(kv["mm_fp8_dram_bytes_per_step"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 # -------------------------------------------------------------------- main ----
 
 def main():
@@ -469,6 +491,7 @@ def main():
     else:
         fp8_peak, peak_src = 2.0 * 1400.0, "of fallback (1.4 PF/s bf16 sustained x 2)"
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    traffic = measured_traffic()
     gemm_tf = flops / (g_ms * 1e-3) / 1e12
     qb = quant_bytes(M)
     quant_gbs = qb / (q_ms * 1e-3) / 1e9
@@ -487,7 +510,8 @@ def main():
             "mm_tflops": round(gemm_tf, 2), "quantize_gbs": round(quant_gbs, 1),
             "quantize_ms_per_step": round(q_ms, 4), "mm_ms_per_step": round(g_ms, 4),
             "roofline": {"bound": "tensor", "achieved": round(gemm_tf, 2), "peak": round(fp8_peak, 1),
-                         "unit": "TFLOP/s", "frac": round(gemm_tf / fp8_peak, 4), "traffic": None,
+                         "unit": "TFLOP/s", "frac": round(gemm_tf / fp8_peak, 4),
+                         "traffic": traffic if M == 8192 else None,
                          "kernel": "mm_fp8_kernel (all 6 GEMM launches of the step)", "peak_source": peak_src},
             "quantize_roofline": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                                   "frac": round(quant_gbs / hbm_peak, 4), "peak_source": "of measured hbm_gbs"},

@@ -297,7 +297,7 @@ def sweep(args):
 
     B.build()
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
-    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    flush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
     want = None
     if args.shapes:
         want = [tuple(int(v) for v in s.split("x")) for s in args.shapes.split(",")]

@@ -19,9 +19,10 @@
 //     word, writes it to a padded shared tile (pitch 33 words: conflict-free
 //     writes and reads) and the block streams 128-byte rows of out_t.
 //   * amax: fmaxf over |x| (NaN ignored) -> warp shuffle -> block -> one
-//     atomicMax on the float bits per block (non-negative floats order as
-//     unsigned integers).  The ticket is an atomicAdd after __threadfence;
-//     the block that draws the last ticket folds the ring, publishes the
+//     atomic update of the float bits per block (non-negative floats order as
+//     unsigned integers), then an acq_rel atomic ticket that orders each
+//     block's amax before its increment; the block that draws the last
+//     ticket acquires them all, folds the ring, publishes the
 //     scale and resets the scratch words to zero for the next call (no
 //     memset launch, no host involvement).
 #include <cuda_bf16.h>
@@ -157,6 +158,26 @@ __device__ __forceinline__ void load_vec_aligned(const uint8_t* p, float (&v)[N]
 
 // ---- conversion ------------------------------------------------------------
 
+// Running max of |x| over 16-bit pairs: max.xorsign.abs keeps max(|a|, |b|)
+// per half (the sign bit of the result is meaningless and masked at the
+// end); a NaN operand yields the other operand, as fmaxf does.
+template <int DT>
+__device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t w) {
+  uint32_t r;
+  if constexpr (DT == FP8_IN_BF16)
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w));
+  else
+    asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w));
+  return r;
+}
+
+template <int DT>
+__device__ __forceinline__ float absmax2_to_float(uint32_t acc) {
+  float lo, hi;
+  unpack2<DT>(acc & 0x7FFF7FFFu, lo, hi);
+  return fmaxf(lo, hi);
+}
+
 // (a*s, b*s) with one packed fp32x2 multiply, each lane rounded to nearest
 // even exactly as a scalar fp32 multiply (no contraction into anything else).
 __device__ __forceinline__ void scale2(float& a, float& b, float s) {
@@ -249,13 +270,21 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
     float m = 0.0f;
 #pragma unroll
     for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, warp_max[w]);
-    if (m > 0.0f) atomicMax(&ring.scratch[0], __float_as_uint(m));
-    __threadfence();  // release: our amax is visible before our ticket
-    const unsigned t = atomicAdd(&ring.scratch[1], 1u);
+    if (m > 0.0f)
+      asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(ring.scratch), "r"(__float_as_uint(m))
+                   : "memory");
+    // acq_rel ticket: releases our amax before the increment; the block that
+    // draws the last ticket acquires every other block's amax.  (A single
+    // 64-bit compare-and-swap carrying both was tried: hundreds of blocks
+    // finishing together made its retries quadratic.)
+    unsigned t;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(ring.scratch + 1) : "memory");
     last = (t == gridDim.x - 1);
     if (last) {
-      __threadfence();  // acquire: every block's amax is visible now
-      const float a = __uint_as_float(atomicExch(&ring.scratch[0], 0u));
+      uint32_t bits;
+      asm volatile("atom.relaxed.gpu.global.exch.b32 %0, [%1], 0;" : "=r"(bits) : "l"(ring.scratch) : "memory");
+      const float a = __uint_as_float(bits);
+      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ring.scratch + 1) : "memory");
       int idx = idx_s;
       idx = ((idx % kHistoryLen) + kHistoryLen) % kHistoryLen;
       hist_s[idx] = a;
@@ -270,7 +299,6 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
         if (isfinite(c) && c > 0.0f) *ring.scale = c;
       }
       *ring.scale_inv = __frcp_rn(s_used);
-      ring.scratch[1] = 0u;
     }
   }
 }
@@ -477,10 +505,11 @@ __device__ __forceinline__ bool bar_wait_bounded(uint32_t bar, uint32_t parity) 
 }
 
 template <int DT>
-__device__ __forceinline__ void issue_tile_load(const CUtensorMap* tm, uint32_t dst, uint32_t bar, int64_t t,
-                                                int64_t tiles_c) {
-  const int r0 = int((t / tiles_c) * kTileR);
-  const int c0 = int((t % tiles_c) * kTileC);
+__device__ __forceinline__ void issue_tile_load(const CUtensorMap* tm, uint32_t dst, uint32_t bar, uint32_t t,
+                                                uint32_t tiles_c) {
+  const uint32_t tr = t / tiles_c;
+  const int r0 = int(tr * kTileR);
+  const int c0 = int((t - tr * tiles_c) * kTileC);
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
                "r"(uint32_t(TmaTile<DT>::kStageBytes))
                : "memory");
@@ -525,24 +554,27 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
   const float s = *a.ring.scale;
   const RingCache rc = prefetch_ring(a.ring);
   float amax = 0.0f;
-  int64_t issued = 0;  // tiles of this block whose loads thread 0 has issued
+  int issued = 0;  // tiles of this block whose loads thread 0 has issued
   if (threadIdx.x == 0) {
     for (int i = 0; i < TT::kStages; ++i) {
-      const int64_t t = blockIdx.x + int64_t(i) * gridDim.x;
-      if (t >= a.ntiles) break;
+      const uint32_t t = blockIdx.x + uint32_t(i) * gridDim.x;
+      if (t >= uint32_t(a.ntiles)) break;
       issue_tile_load<DT>(&tmIn, sbase + uint32_t(i * TT::kStageBytes), bar0 + 8u * i, t, a.tiles_c);
       ++issued;
     }
   }
 
-  int64_t k = 0;
-  for (int64_t t = blockIdx.x; t < a.ntiles; t += gridDim.x, ++k) {
-    const int stage = int(k % TT::kStages);
+  uint32_t amax2 = 0u;  // packed |x| maxima of 16-bit inputs
+  const uint32_t tiles_c = uint32_t(a.tiles_c), ntiles = uint32_t(a.ntiles);
+  int k = 0;
+  for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
+    const int stage = k % TT::kStages;
     const uint32_t parity = uint32_t((k / TT::kStages) & 1);
     const bool ok = bar_wait_bounded(bar0 + 8u * stage, parity);
     const uint8_t* st = smem + stage * TT::kStageBytes;
-    const int64_t r0 = (t / a.tiles_c) * kTileR;
-    const int64_t c0 = (t % a.tiles_c) * kTileC;
+    const uint32_t tr = t / tiles_c;
+    const int64_t r0 = int64_t(tr) * kTileR;
+    const int64_t c0 = int64_t(t - tr * tiles_c) * kTileC;
     uint32_t q[4][2];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -551,6 +583,7 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
       if constexpr (kB == 2) {
         const int chunk = (lc0 >> 3) ^ (r & 7);
         const uint4 w = *reinterpret_cast<const uint4*>(st + r * 128 + chunk * 16);
+        amax2 = absmax2<DT>(absmax2<DT>(amax2, w.x), absmax2<DT>(w.y, absmax2<DT>(w.z, w.w)));
         unpack2<DT>(w.x, v[0], v[1]);
         unpack2<DT>(w.y, v[2], v[3]);
         unpack2<DT>(w.z, v[4], v[5]);
@@ -563,9 +596,9 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
         const float4 f1 = *reinterpret_cast<const float4*>(rowp + (((ch + 1) ^ (r & 7)) * 16));
         v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
         v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
-      }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+      }
       q[i][0] = cvt4<FMT>(v[0], v[1], v[2], v[3], s);
       q[i][1] = cvt4<FMT>(v[4], v[5], v[6], v[7], s);
     }
@@ -575,8 +608,8 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
       break;
     }
     if (threadIdx.x == 0) {
-      const int64_t tn = t + int64_t(TT::kStages) * gridDim.x;
-      if (tn < a.ntiles) {
+      const uint32_t tn = t + uint32_t(TT::kStages) * gridDim.x;
+      if (tn < ntiles) {
         issue_tile_load<DT>(&tmIn, sbase + uint32_t(stage * TT::kStageBytes), bar0 + 8u * stage, tn, a.tiles_c);
         ++issued;
       }
@@ -623,10 +656,11 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
       }
     }
   }
+  if constexpr (kB == 2) amax = fmaxf(amax, absmax2_to_float<DT>(amax2));
   // After an abort, let every copy this block issued land before its shared
   // memory is released (bounded).
   if (threadIdx.x == 0) {
-    for (int64_t j = k; j < issued; ++j)
+    for (int j = k; j < issued; ++j)
       bar_wait_bounded(bar0 + 8u * uint32_t(j % TT::kStages), uint32_t((j / TT::kStages) & 1));
   }
   amax_ticket_fold<FMT>(amax, a.ring, s, rc);
@@ -738,6 +772,7 @@ extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t col
   if ((layout == FP8_LAYOUT_T || layout == FP8_LAYOUT_DUAL) && n > 0 && out_t == nullptr) return FP8_ERR_INVALID_ARG;
   const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
   if (reinterpret_cast<uintptr_t>(in) % eb != 0) return FP8_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(ring.scratch) % 8 != 0) return FP8_ERR_UNSUPPORTED;
 
   const int sms = sm_count_current();
   if (sms <= 0) return FP8_ERR_CUDA;
@@ -776,7 +811,8 @@ extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t col
   a.outt4 = (reinterpret_cast<uintptr_t>(out_t) % 4 == 0) && (rows % 4 == 0);
   a.ring = r;
   const bool dual = layout == FP8_LAYOUT_DUAL;
-  if (n > 0 && reinterpret_cast<uintptr_t>(in) % 16 == 0 && (cols * eb) % 16 == 0) {
+  if (n > 0 && reinterpret_cast<uintptr_t>(in) % 16 == 0 && (cols * eb) % 16 == 0 && a.ntiles < (int64_t(1) << 30) &&
+      rows < (int64_t(1) << 30) && cols < (int64_t(1) << 30)) {
     CUtensorMap map;
     std::memset(&map, 0, sizeof(map));
     if (!make_input_map(&map, in, dtype, rows, cols)) return FP8_ERR_CUDA;

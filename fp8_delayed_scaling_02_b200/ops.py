@@ -100,7 +100,8 @@ def _ptr(t):
 class Ring:
     """One tensor's delayed-scaling state in a single device buffer.
 
-    Layout (32-bit words): history[0:16] | idx[16] | scale[17] | scale_inv[18] | scratch[19:21].
+    Layout (32-bit words): history[0:16] | idx[16] | scale[17] | scale_inv[18] | pad[19] |
+    scratch[20:22] (8-byte aligned: the kernels update it as one 64-bit word).
     """
 
     WORDS = 24
@@ -129,20 +130,20 @@ class Ring:
 
     @property
     def scratch(self):
-        return self.buf[19:21]
+        return self.buf[20:22]
 
     def c(self):
         c = getattr(self, "_c", None)
         if c is None:
             base = self.buf.data_ptr()
-            c = self._c = CRing(base, base + 16 * 4, base + 17 * 4, base + 18 * 4, base + 19 * 4)
+            c = self._c = CRing(base, base + 16 * 4, base + 17 * 4, base + 18 * 4, base + 20 * 4)
         return c
 
     def state(self):
         """Host copy: (history float32[16], idx, scale, scale_inv, scratch[2])."""
         h = self.buf.cpu()
         f = h.view(torch.float32)
-        return f[:16].clone(), int(h[16]), float(f[17]), float(f[18]), h[19:21].clone()
+        return f[:16].clone(), int(h[16]), float(f[17]), float(f[18]), h[20:22].clone()
 
 
 def quantize(x, fmt, layout, ring, out=None, out_t=None, stream=None):

@@ -75,7 +75,8 @@ typedef struct {
                       /*      by the last block of each call)                  */
   float* scale_inv;   /* [1]  1/scale that the MOST RECENT call used: the      */
                       /*      dequantisation factor to hand to fp8_mm          */
-  uint32_t* scratch;  /* [2]  amax bits and block ticket; zero between calls   */
+  uint32_t* scratch;  /* [2]  amax bits and block ticket, 8-byte aligned (one  */
+                      /*      64-bit word); zero between calls                 */
 } fp8_ring;
 
 /*
@@ -100,7 +101,8 @@ typedef struct {
  * Errors: FP8_ERR_INVALID_ARG for a bad enum, a negative size, a NULL ring
  *         field, a NULL in with rows*cols > 0, or a NULL out/out_t the
  *         layout needs; FP8_ERR_UNSUPPORTED for an input address not aligned
- *         to its element size; FP8_ERR_CUDA if the launch fails.
+ *         to its element size or ring.scratch not 8-byte aligned;
+ *         FP8_ERR_CUDA if the launch fails.
  */
 int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
                  fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);

@@ -43,7 +43,7 @@ def test_status_strings(L):
 
 
 def _ring(addr=0x1000):
-    return ops.CRing(addr, addr + 64, addr + 68, addr + 72, addr + 76)
+    return ops.CRing(addr, addr + 64, addr + 68, addr + 72, addr + 80)
 
 
 def _q(L, dtype=0, rows=4, cols=4, layout=0, fmt=0, ring=None, out=0x2000, out_t=0x3000, inp=0x4000):
@@ -63,6 +63,7 @@ def test_quantize_rejects_bad_arguments_without_cuda(L):
     assert _q(L, layout=2, out_t=0) == ops.FP8_ERR_INVALID_ARG
     assert _q(L, dtype=2, inp=0x4002) == ops.FP8_ERR_UNSUPPORTED   # fp32 needs 4-byte alignment
     assert _q(L, dtype=0, inp=0x4001) == ops.FP8_ERR_UNSUPPORTED   # bf16 needs 2-byte alignment
+    assert _q(L, ring=ops.CRing(0x1000, 0x1040, 0x1044, 0x1048, 0x104C)) == ops.FP8_ERR_UNSUPPORTED  # scratch % 8
 
 
 def _mm(L, M=128, N=128, K=128, batch=1, strides=None, layout=0, A=0x10000, B=0x20000, out=0x30000,

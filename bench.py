@@ -56,6 +56,8 @@ def parse():
     ap.add_argument("--profile", action="store_true",
                     help="warm up, run exactly one step inside the NVTX range fp8_profile_step, exit (for ncu)")
     ap.add_argument("--shapes", default=None, help="sweep subset, e.g. 8192x8192x8192,64x8192x2048")
+    ap.add_argument("--qdtypes", default="bf16,fp32", help="quantize sweep input dtypes")
+    ap.add_argument("--qlayouts", default="row,T,dual", help="quantize sweep layouts")
     return ap.parse_args()
 
 
@@ -319,10 +321,12 @@ def sweep(args):
                                   "us": round(ms * 1e3, 2), "tflops": round(fl / ms / 1e9, 1)}))
     else:
         for rows, cols in (QUANT_SHAPES if not want else want):
-            for dt in ("bf16", "fp32"):
+            for dt in args.qdtypes.split(","):
                 x = S.quant_sweep_input(rows, cols, dt, 1.0).cuda()
                 eb = x.element_size()
                 for layout, name in ((ops.ROW, "row"), (ops.TRANSPOSED, "T"), (ops.DUAL, "dual")):
+                    if name not in args.qlayouts.split(","):
+                        continue
                     ring = ops.Ring()
                     out = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
                     out_t = torch.empty((cols, rows), dtype=torch.uint8, device="cuda")

@@ -252,10 +252,10 @@ __device__ __forceinline__ RingCache prefetch_ring(const RingArgs& ring) {
   return c;
 }
 
-template <int FMT>
+template <int FMT, int NT = kThreads>
 __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& ring, float s_used,
                                                  const RingCache& rc) {
-  __shared__ float warp_max[kThreads / 32];
+  __shared__ float warp_max[NT / 32];
   __shared__ float hist_s[kHistoryLen];
   __shared__ int idx_s;
   __shared__ int last;
@@ -269,7 +269,7 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
   if (threadIdx.x == 0) {
     float m = 0.0f;
 #pragma unroll
-    for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, warp_max[w]);
+    for (int w = 0; w < NT / 32; ++w) m = fmaxf(m, warp_max[w]);
     if (m > 0.0f)
       asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(ring.scratch), "r"(__float_as_uint(m))
                    : "memory");
@@ -285,6 +285,7 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
       asm volatile("atom.relaxed.gpu.global.exch.b32 %0, [%1], 0;" : "=r"(bits) : "l"(ring.scratch) : "memory");
       const float a = __uint_as_float(bits);
       asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ring.scratch + 1) : "memory");
+      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ring.scratch + 2) : "memory");  // tile counter
       int idx = idx_s;
       idx = ((idx % kHistoryLen) + kHistoryLen) % kHistoryLen;
       hist_s[idx] = a;
@@ -453,25 +454,35 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs 
   amax_ticket_fold<FMT>(amax, a.ring, s, rc);
 }
 
-// ---- T / DUAL layouts, TMA-fed pipeline (16-byte aligned rows) ------------------
+// ---- T / DUAL layouts, warp-specialised TMA pipeline (16-byte aligned rows) -------
 //
-// Same tile geometry and lane mapping as quantize_tile_kernel, but the input
-// tiles arrive by TMA (128 rows x 128 bytes per box, 128B-swizzled) into a
-// kTmaStages-deep shared-memory ring, so each block keeps several tiles of
-// HBM reads in flight while it converts and transposes the current one.
-// Blocks are persistent over tiles.  Used when the input base is 16-byte
-// aligned and a row is a multiple of 16 bytes; ragged edges are zero-filled
-// by TMA and the stores are guarded.
+// Same 128x64 tiles and lane mapping as quantize_tile_kernel.  Warp 8 is the
+// producer: it claims tiles from a counter in the ring's scratch (so blocks
+// that finish early take more tiles and all blocks end within one tile of
+// each other), writes the tile id into shared memory and loads the tile with
+// TMA (128 rows x 128 bytes per box, 128B-swizzled) into a kStages-deep ring.
+// Warps 0..7 consume: each warp releases a stage with one mbarrier arrive as
+// soon as its lanes have read it, converts, writes the DUAL row pieces, and
+// transposes into one of two 8 KB buffers (16-byte units XOR-swizzled by the
+// column group); one named-barrier reduction per tile publishes the buffer
+// and makes the stop decision uniform, and the buffer leaves as 16-byte
+// stores of 128-byte out_t rows.  Ragged edges are zero-filled by TMA and the
+// stores are guarded.  Used when the input base is 16-byte aligned and a row
+// is a multiple of 16 bytes.
 
-constexpr int kTmaStages = 4;
+constexpr int kConsumerWarps = 8;
+constexpr int kWsThreads = 32 * (kConsumerWarps + 1);
+constexpr uint32_t kNoTile = 0xFFFFFFFFu;
 
 template <int DT>
 struct TmaTile {
   static constexpr int kBoxes = In<DT>::kBytes == 4 ? 2 : 1;  // 128-byte-wide boxes per 64-column tile
   static constexpr int kBoxBytes = kTileR * 128;
   static constexpr int kStageBytes = kBoxes * kBoxBytes;
-  static constexpr int kStages = DT == FP8_IN_FP32 ? 3 : kTmaStages;
-  static constexpr int kSmem = kStages * kStageBytes + kTileC * kPitchW * 4 + 64 + 1024;
+  static constexpr int kStages = DT == FP8_IN_FP32 ? 2 : 3;
+  static constexpr int kTBytes = kTileC * kTileR;  // one transpose buffer: 64 rows of 128 bytes
+  static constexpr int kBarOff = kStages * kStageBytes + 2 * kTBytes;
+  static constexpr int kSmem = kBarOff + 16 * kStages + 8 * kStages + 64 + 1024;
 };
 
 struct TmaTileArgs {
@@ -504,6 +515,24 @@ __device__ __forceinline__ bool bar_wait_bounded(uint32_t bar, uint32_t parity) 
   return true;
 }
 
+__device__ __forceinline__ void bar_arrive_local(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// OR-reduction barrier over the consumer warps only (named barrier 1).
+__device__ __forceinline__ bool consumers_sync_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(v ? 1u : 0u), "r"(32 * kConsumerWarps)
+      : "memory");
+  return r != 0;
+}
+
 template <int DT>
 __device__ __forceinline__ void issue_tile_load(const CUtensorMap* tm, uint32_t dst, uint32_t bar, uint32_t t,
                                                 uint32_t tiles_c) {
@@ -524,27 +553,33 @@ __device__ __forceinline__ void issue_tile_load(const CUtensorMap* tm, uint32_t 
   }
 }
 
+// Byte offset of 16-byte unit v of transpose-buffer row c (rows of 128 bytes;
+// the unit index is XOR-swizzled by the column group so that the column-word
+// writes and the row reads are both free of bank conflicts).
+__device__ __forceinline__ int tbuf_unit(int c, int v) { return c * 128 + ((v ^ ((c >> 2) & 6)) << 4); }
+
 template <int DT, int FMT, bool kDual>
-__global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __grid_constant__ CUtensorMap tmIn,
-                                                                      const TmaTileArgs args) {
+__global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __grid_constant__ CUtensorMap tmIn,
+                                                                        const TmaTileArgs args) {
   using TT = TmaTile<DT>;
   constexpr int kB = In<DT>::kBytes;
+  constexpr int S = TT::kStages;
   const TileArgs& a = args.t;
   extern __shared__ uint8_t qsmem_raw[];
   uint8_t* smem = qsmem_raw + ((1024u - (smem_addr(qsmem_raw) & 1023u)) & 1023u);
   const uint32_t sbase = smem_addr(smem);
-  uint32_t* sT = reinterpret_cast<uint32_t*>(smem + TT::kStages * TT::kStageBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sT + kTileC * kPitchW);
-  const uint32_t bar0 = smem_addr(bars);
+  uint8_t* tbuf = smem + S * TT::kStageBytes;
+  const uint32_t full0 = sbase + TT::kBarOff;        // full[S]
+  const uint32_t empty0 = full0 + 8u * S;            // empty[S]
+  volatile uint32_t* tile_id = reinterpret_cast<volatile uint32_t*>(smem + TT::kBarOff + 16 * S);
 
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int lr0 = 32 * (warp & 3) + 4 * (lane & 7);
-  const int lc0 = 32 * (warp >> 2) + 8 * (lane >> 3);
-
   if (threadIdx.x == 0) {
-    for (int i = 0; i < TT::kStages; ++i)
-      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(bar0 + 8u * i) : "memory");
+    for (int i = 0; i < S; ++i) {
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full0 + 8u * i) : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(empty0 + 8u * i), "r"(kConsumerWarps) : "memory");
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmIn)) : "memory");
@@ -554,116 +589,160 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_tma_kernel(const __gri
   const float s = *a.ring.scale;
   const RingCache rc = prefetch_ring(a.ring);
   float amax = 0.0f;
-  int issued = 0;  // tiles of this block whose loads thread 0 has issued
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < TT::kStages; ++i) {
-      const uint32_t t = blockIdx.x + uint32_t(i) * gridDim.x;
-      if (t >= uint32_t(a.ntiles)) break;
-      issue_tile_load<DT>(&tmIn, sbase + uint32_t(i * TT::kStageBytes), bar0 + 8u * i, t, a.tiles_c);
-      ++issued;
-    }
-  }
-
-  uint32_t amax2 = 0u;  // packed |x| maxima of 16-bit inputs
   const uint32_t tiles_c = uint32_t(a.tiles_c), ntiles = uint32_t(a.ntiles);
-  int k = 0;
-  for (uint32_t t = blockIdx.x; t < ntiles; t += gridDim.x, ++k) {
-    const int stage = k % TT::kStages;
-    const uint32_t parity = uint32_t((k / TT::kStages) & 1);
-    const bool ok = bar_wait_bounded(bar0 + 8u * stage, parity);
-    const uint8_t* st = smem + stage * TT::kStageBytes;
-    const uint32_t tr = t / tiles_c;
-    const int64_t r0 = int64_t(tr) * kTileR;
-    const int64_t c0 = int64_t(t - tr * tiles_c) * kTileC;
-    uint32_t q[4][2];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = lr0 + i;
-      float v[8];
-      if constexpr (kB == 2) {
-        const int chunk = (lc0 >> 3) ^ (r & 7);
-        const uint4 w = *reinterpret_cast<const uint4*>(st + r * 128 + chunk * 16);
-        amax2 = absmax2<DT>(absmax2<DT>(amax2, w.x), absmax2<DT>(w.y, absmax2<DT>(w.z, w.w)));
-        unpack2<DT>(w.x, v[0], v[1]);
-        unpack2<DT>(w.y, v[2], v[3]);
-        unpack2<DT>(w.z, v[4], v[5]);
-        unpack2<DT>(w.w, v[6], v[7]);
-      } else {
-        const int box = lc0 >> 5;
-        const int ch = (lc0 & 31) >> 2;
-        const uint8_t* rowp = st + box * TT::kBoxBytes + r * 128;
-        const float4 f0 = *reinterpret_cast<const float4*>(rowp + ((ch ^ (r & 7)) * 16));
-        const float4 f1 = *reinterpret_cast<const float4*>(rowp + (((ch + 1) ^ (r & 7)) * 16));
-        v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
-        v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
-      }
-      q[i][0] = cvt4<FMT>(v[0], v[1], v[2], v[3], s);
-      q[i][1] = cvt4<FMT>(v[4], v[5], v[6], v[7], s);
-    }
-    // Every thread is done with this stage and with the previous tile's sT.
-    if (!__syncthreads_and(ok ? 1 : 0)) {
-      if (threadIdx.x == 0) record_device_error(args.err, kWaitQuantizeTma);
-      break;
-    }
-    if (threadIdx.x == 0) {
-      const uint32_t tn = t + uint32_t(TT::kStages) * gridDim.x;
-      if (tn < ntiles) {
-        issue_tile_load<DT>(&tmIn, sbase + uint32_t(stage * TT::kStageBytes), bar0 + 8u * stage, tn, a.tiles_c);
-        ++issued;
-      }
-    }
-    const bool interior = (r0 + kTileR <= a.rows) && (c0 + kTileC <= a.cols);
-    if constexpr (kDual) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int64_t r = r0 + lr0 + i;
-        const int64_t c = c0 + lc0;
-        uint8_t* o = a.out + r * a.cols + c;
-        if (interior && a.out8) {
-          *reinterpret_cast<uint2*>(o) = make_uint2(q[i][0], q[i][1]);
-        } else if (r < a.rows) {
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (c + j < a.cols) o[j] = uint8_t(q[i][j >> 2] >> (8 * (j & 3)));
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: claim, then load ----------------
+    if (lane == 0) {
+      uint32_t armed = 0, armed_par = 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t claim = atomicAdd(a.ring.scratch + 2, 1u);
+      while (true) {
+        if (!bar_wait_bounded(empty0 + 8u * stage, phase ^ 1u)) {
+          record_device_error(args.err, kWaitQuantizeTma);
+          break;
         }
-      }
-    }
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t c[4];
-      transpose4x4(q[0][h], q[1][h], q[2][h], q[3][h], c[0], c[1], c[2], c[3]);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) sT[(lc0 + 4 * h + k) * kPitchW + (lr0 >> 2)] = c[k];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < kTileC / 8; ++kk) {
-      const int cl = 8 * warp + kk;
-      const int64_t c = c0 + cl;
-      const int64_t r = r0 + 4 * lane;
-      const uint32_t w = sT[cl * kPitchW + lane];
-      if (c < a.cols) {
-        uint8_t* o = a.out_t + c * a.rows + r;
-        if (a.outt4 && r + 4 <= a.rows) {
-          *reinterpret_cast<uint32_t*>(o) = w;
+        const uint32_t t = claim;
+        if (t < ntiles) {
+          claim = atomicAdd(a.ring.scratch + 2, 1u);  // next claim in flight while this tile loads
+          tile_id[stage] = t;
+          issue_tile_load<DT>(&tmIn, sbase + uint32_t(stage * TT::kStageBytes), full0 + 8u * stage, t, tiles_c);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
         } else {
-#pragma unroll
-          for (int b = 0; b < 4; ++b)
-            if (r + b < a.rows) o[b] = uint8_t(w >> (8 * b));
+          // The copy last armed on this stage was consumed (its empty phase
+          // completed above); the stop marker completes a further phase with
+          // no copy, so this stage has nothing left to drain.
+          armed &= ~(1u << stage);
+          tile_id[stage] = kNoTile;
+          bar_arrive_local(full0 + 8u * stage);  // wakes the consumers with the stop marker
+          break;
+        }
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
+      // Every armed copy has landed before shared memory can be released.
+      for (int i = 0; i < S; ++i)
+        if (armed & (1u << i)) bar_wait_bounded(full0 + 8u * i, (armed_par >> i) & 1u);
     }
+    __syncwarp();
+  } else {
+    // ---------------- consumers ----------------
+    const int lr0 = 32 * (warp & 3) + 4 * (lane & 7);  // first of this lane's 4 rows
+    const int lc0 = 32 * (warp >> 2) + 8 * (lane >> 3);  // first of its 8 columns
+    const bool out16 = a.outt4 && (a.rows % 16 == 0) && (reinterpret_cast<uintptr_t>(a.out_t) % 16 == 0);
+    uint32_t amax2 = 0u;  // packed |x| maxima of 16-bit inputs
+    int stage = 0, buf = 0;
+    uint32_t phase = 0;
+    while (true) {
+      const bool ok = bar_wait_bounded(full0 + 8u * stage, phase);
+      const uint32_t t = ok ? uint32_t(tile_id[stage]) : uint32_t(kNoTile);
+      const bool stop = t == kNoTile;
+      uint32_t q[4][2];
+      if (!stop) {
+        const uint8_t* st = smem + stage * TT::kStageBytes;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = lr0 + i;
+          float v[8];
+          if constexpr (kB == 2) {
+            const int chunk = (lc0 >> 3) ^ (r & 7);
+            const uint4 w = *reinterpret_cast<const uint4*>(st + r * 128 + chunk * 16);
+            amax2 = absmax2<DT>(absmax2<DT>(amax2, w.x), absmax2<DT>(w.y, absmax2<DT>(w.z, w.w)));
+            unpack2<DT>(w.x, v[0], v[1]);
+            unpack2<DT>(w.y, v[2], v[3]);
+            unpack2<DT>(w.z, v[4], v[5]);
+            unpack2<DT>(w.w, v[6], v[7]);
+          } else {
+            const int box = lc0 >> 5;
+            const int ch = (lc0 & 31) >> 2;
+            const uint8_t* rowp = st + box * TT::kBoxBytes + r * 128;
+            const float4 f0 = *reinterpret_cast<const float4*>(rowp + ((ch ^ (r & 7)) * 16));
+            const float4 f1 = *reinterpret_cast<const float4*>(rowp + (((ch + 1) ^ (r & 7)) * 16));
+            v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+            v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+          }
+          q[i][0] = cvt4<FMT>(v[0], v[1], v[2], v[3], s);
+          q[i][1] = cvt4<FMT>(v[4], v[5], v[6], v[7], s);
+        }
+      }
+      // This warp is done reading the stage: let the producer refill it.
+      __syncwarp();
+      if (lane == 0) bar_arrive_local(empty0 + 8u * stage);
+      int64_t r0 = 0, c0 = 0;
+      if (!stop) {
+        const uint32_t tr = t / tiles_c;
+        r0 = int64_t(tr) * kTileR;
+        c0 = int64_t(t - tr * tiles_c) * kTileC;
+        const bool interior = (r0 + kTileR <= a.rows) && (c0 + kTileC <= a.cols);
+        if constexpr (kDual) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int64_t r = r0 + lr0 + i;
+            const int64_t c = c0 + lc0;
+            uint8_t* o = a.out + r * a.cols + c;
+            if (interior && a.out8) {
+              *reinterpret_cast<uint2*>(o) = make_uint2(q[i][0], q[i][1]);
+            } else if (r < a.rows) {
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (c + j < a.cols) o[j] = uint8_t(q[i][j >> 2] >> (8 * (j & 3)));
+            }
+          }
+        }
+        uint8_t* tb = tbuf + buf * TT::kTBytes;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t c[4];
+          transpose4x4(q[0][h], q[1][h], q[2][h], q[3][h], c[0], c[1], c[2], c[3]);
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int col = lc0 + 4 * h + k;
+            const int word = lr0 >> 2;  // 4 rows per word
+            *reinterpret_cast<uint32_t*>(tb + tbuf_unit(col, word >> 2) + ((word & 3) << 2)) = c[k];
+          }
+        }
+      }
+      if (consumers_sync_or(stop)) break;
+      // out_t rows: thread -> (column c, 16-byte unit v), two columns per thread.
+      {
+        const uint8_t* tb = tbuf + buf * TT::kTBytes;
+        const int tid = threadIdx.x;  // 0..255
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int col = (tid >> 3) + 32 * i;
+          const int v = tid & 7;
+          const uint4 w = *reinterpret_cast<const uint4*>(tb + tbuf_unit(col, v));
+          const int64_t c = c0 + col;
+          const int64_t r = r0 + 16 * v;
+          if (c < a.cols) {
+            uint8_t* o = a.out_t + c * a.rows + r;
+            if (out16 && r + 16 <= a.rows) {
+              *reinterpret_cast<uint4*>(o) = w;
+            } else {
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int b = 0; b < 16; ++b)
+                if (r + b < a.rows) o[b] = uint8_t(ww[b >> 2] >> (8 * (b & 3)));
+            }
+          }
+        }
+      }
+      buf ^= 1;
+      if (++stage == S) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+    if constexpr (kB == 2) amax = fmaxf(amax, absmax2_to_float<DT>(amax2));
   }
-  if constexpr (kB == 2) amax = fmaxf(amax, absmax2_to_float<DT>(amax2));
-  // After an abort, let every copy this block issued land before its shared
-  // memory is released (bounded).
-  if (threadIdx.x == 0) {
-    for (int j = k; j < issued; ++j)
-      bar_wait_bounded(bar0 + 8u * uint32_t(j % TT::kStages), uint32_t((j / TT::kStages) & 1));
-  }
-  amax_ticket_fold<FMT>(amax, a.ring, s, rc);
+  __syncthreads();
+  amax_ticket_fold<FMT, kWsThreads>(amax, a.ring, s, rc);
 }
 
 // ---- host side ---------------------------------------------------------------
@@ -728,7 +807,7 @@ int tma_blocks_per_sm() {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TmaTile<DT>::kSmem) != cudaSuccess)
       return -1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kThreads, TmaTile<DT>::kSmem) != cudaSuccess || n < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kWsThreads, TmaTile<DT>::kSmem) != cudaSuccess || n < 1)
       return -1;
     cached[dev] = n;
   }
@@ -742,8 +821,8 @@ int launch_tile_tma(const TileArgs& t, const CUtensorMap& map, int sms, cudaStre
   if (bps <= 0) return FP8_ERR_CUDA;
   const int grid = int(std::max<int64_t>(1, std::min<int64_t>(t.ntiles, int64_t(bps) * sms)));
   const cudaError_t e =
-      dual ? launch_pdl(quantize_tile_tma_kernel<DT, FMT, true>, grid, kThreads, TmaTile<DT>::kSmem, st, 1, map, a)
-           : launch_pdl(quantize_tile_tma_kernel<DT, FMT, false>, grid, kThreads, TmaTile<DT>::kSmem, st, 1, map, a);
+      dual ? launch_pdl(quantize_tile_tma_kernel<DT, FMT, true>, grid, kWsThreads, TmaTile<DT>::kSmem, st, 1, map, a)
+           : launch_pdl(quantize_tile_tma_kernel<DT, FMT, false>, grid, kWsThreads, TmaTile<DT>::kSmem, st, 1, map, a);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
@@ -848,7 +927,7 @@ static __device__ __align__(256) uint32_t g_quantize_static_scratch[64];
 
 namespace {
 constexpr int kStaticScratchWords = 64;    // capacity of g_quantize_static_scratch
-constexpr int kQuantizeScratchWords = 2;   // what one quantize call needs, whatever its size
+constexpr int kQuantizeScratchWords = 4;   // what one quantize call needs, whatever its size
 
 std::mutex g_static_scratch_mu;
 uint32_t* g_static_scratch_ptr[64] = {nullptr};

@@ -101,7 +101,7 @@ class Ring:
     """One tensor's delayed-scaling state in a single device buffer.
 
     Layout (32-bit words): history[0:16] | idx[16] | scale[17] | scale_inv[18] | pad[19] |
-    scratch[20:22] (8-byte aligned: the kernels update it as one 64-bit word).
+    scratch[20:24] (amax bits, block ticket, tile counter, spare; 8-byte aligned).
     """
 
     WORDS = 24
@@ -130,7 +130,7 @@ class Ring:
 
     @property
     def scratch(self):
-        return self.buf[20:22]
+        return self.buf[20:24]
 
     def c(self):
         c = getattr(self, "_c", None)
@@ -140,10 +140,10 @@ class Ring:
         return c
 
     def state(self):
-        """Host copy: (history float32[16], idx, scale, scale_inv, scratch[2])."""
+        """Host copy: (history float32[16], idx, scale, scale_inv, scratch[4])."""
         h = self.buf.cpu()
         f = h.view(torch.float32)
-        return f[:16].clone(), int(h[16]), float(f[17]), float(f[18]), h[20:22].clone()
+        return f[:16].clone(), int(h[16]), float(f[17]), float(f[18]), h[20:24].clone()
 
 
 def quantize(x, fmt, layout, ring, out=None, out_t=None, stream=None):

@@ -75,8 +75,9 @@ typedef struct {
                       /*      by the last block of each call)                  */
   float* scale_inv;   /* [1]  1/scale that the MOST RECENT call used: the      */
                       /*      dequantisation factor to hand to fp8_mm          */
-  uint32_t* scratch;  /* [2]  amax bits and block ticket, 8-byte aligned (one  */
-                      /*      64-bit word); zero between calls                 */
+  uint32_t* scratch;  /* [4]  amax bits, block ticket, tile counter, spare;    */
+                      /*      8-byte aligned; zero between calls (the kernel   */
+                      /*      leaves them at zero)                             */
 } fp8_ring;
 
 /*
@@ -115,18 +116,18 @@ int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layo
  * interfaces that receive only input and output pointers, or deployments that
  * reserve all device memory at start-up.  It computes exactly what
  * fp8_quantize computes, with the same arguments, except that ring.scratch is
- * ignored (it may be NULL): the two scratch words (amax bits and block
- * ticket) live in a 256-byte array owned by the library, which every GPU that
+ * ignored (it may be NULL): the four scratch words (amax bits, block ticket,
+ * tile counter, spare) live in a 256-byte array owned by the library, which every GPU that
  * loads the library holds until the process exits.  The call itself allocates
  * nothing.
  *
- *   - The array holds 64 words; a call needs 2, whatever rows*cols is, so no
+ *   - The array holds 64 words; a call needs 4, whatever rows*cols is, so no
  *     tensor is refused for lack of scratch.  A request needing more than the
  *     array holds would return FP8_ERR_UNSUPPORTED.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture.
- *   - All calls on a device share the array.  Each call clears the two words
+ *   - All calls on a device share the array.  Each call clears the four words
  *     on `stream` before its kernel, and the kernel leaves them at zero, but
  *     two calls that overlap on the GPU (different streams, no ordering
  *     between them) race on the array and give wrong amax and scales.

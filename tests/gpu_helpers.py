@@ -34,7 +34,7 @@ def assert_ring_equal(ring_gpu, ring_ref):
     assert idx == ring_ref.idx
     assert np.float32(scale).view(np.uint32) == np.float32(ring_ref.scale).view(np.uint32), (scale, ring_ref.scale)
     assert np.float32(scale_inv).view(np.uint32) == np.float32(ring_ref.scale_inv).view(np.uint32)
-    assert int(scratch[0]) == 0 and int(scratch[1]) == 0, "scratch must self-reset"
+    assert all(int(v) == 0 for v in scratch), "scratch must self-reset"
 
 
 def quantize_both(x_cpu, fmt, layout, ring_gpu, misalign=False):

@@ -94,7 +94,7 @@ def test_full_size_sampled(shape, layout):
     rng = np.random.default_rng(rows + cols + layout)
     sample = np.unique(np.concatenate([rng.integers(0, rows, 24), [0, rows - 1]]))
     for dtype, fmt, misalign, vs in (("bf16", ops.E4M3, False, 1.0), ("fp32", ops.E5M2, True, 1e3),
-                                     ("fp16", ops.E4M3, True, 1e-3)):
+                                     ("fp16", ops.E4M3, True, 1e-3), ("fp32", ops.E4M3, False, 1.0)):
         x = S.quant_sweep_input(rows, cols, dtype, vs, seed=rows ^ cols)
         ring = ops.Ring()
         for step in range(2):

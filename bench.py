@@ -168,6 +168,20 @@ class Linear:
         ops.mm(self.gq, self.wq_t, self.rg.scale_inv, self.rw.scale_inv, None, fmt_a=ops.E5M2, out=self.dx)
         ops.mm(self.gq_t, self.xq_t, self.rg.scale_inv, self.rx.scale_inv, None, fmt_a=ops.E5M2, out=self.dw)
 
+    # The same step with the layout tag: row-layout quantizes only, and the
+    # backward GEMMs read W, G and X as quantized through MN-major operands.
+    def quantize_row(self, ops, x, g):
+        ops.quantize(x, ops.E4M3, ops.ROW, self.rx, self.xq)
+        ops.quantize(self.w, ops.E4M3, ops.ROW, self.rw, self.wq)
+        ops.quantize(g, ops.E5M2, ops.ROW, self.rg, self.gq)
+
+    def gemms_mn(self, ops):
+        ops.mm(self.xq, self.wq, self.rx.scale_inv, self.rw.scale_inv, self.bias, out=self.y)
+        ops.mm(self.gq, self.wq, self.rg.scale_inv, self.rw.scale_inv, None, fmt_a=ops.E5M2, out=self.dx,
+               b_mn_major=True)
+        ops.mm(self.gq, self.xq, self.rg.scale_inv, self.rx.scale_inv, None, fmt_a=ops.E5M2, out=self.dw,
+               a_mn_major=True, b_mn_major=True)
+
 
 def build_workload(M, torch, ops, S, n_sets=2):
     (w1, b1), (w2, b2) = S.linear_1p2b_weights()
@@ -183,6 +197,13 @@ def run_step(lins, ops, i):
         x, g = L.inputs[i % len(L.inputs)]
         L.quantize(ops, x, g)
         L.gemms(ops)
+
+
+def run_step_layout_tag(lins, ops, i):
+    for L in lins:
+        x, g = L.inputs[i % len(L.inputs)]
+        L.quantize_row(ops, x, g)
+        L.gemms_mn(ops)
 
 
 def capture(torch, fn):
@@ -440,6 +461,17 @@ def main():
         t_clk1 = time.monotonic()
     ms = e0.elapsed_time(e1) / steps
     del graph
+
+    # Layout-tag variant of the same step (reported beside the main line).
+    for i in range(3):
+        run_step_layout_tag(lins, ops, i)
+    graph_lt = capture(torch, lambda: (run_step_layout_tag(lins, ops, 0), run_step_layout_tag(lins, ops, 1)))
+    ms_lt = time_graph(torch, graph_lt, max(50, steps // 10)) / 2
+    del graph_lt
+    if pg:
+        t = torch.tensor([ms_lt], device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_lt = float(t.item())
     if pg:
         t = torch.tensor([ms], device="cuda")
         pg.all_reduce(t, op=pg.ReduceOp.MAX)
@@ -513,6 +545,9 @@ def main():
                        "parallelism": f"replicas x{world}"},
             "mm_tflops": round(gemm_tf, 2), "quantize_gbs": round(quant_gbs, 1),
             "quantize_ms_per_step": round(q_ms, 4), "mm_ms_per_step": round(g_ms, 4),
+            "layout_tag_step": {"ms_per_step": round(ms_lt, 4),
+                                "value": round(world * flops / (ms_lt * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                                "what": "same step with row-only quantizes and MN-major operands for dX/dW"},
             "roofline": {"bound": "tensor", "achieved": round(gemm_tf, 2), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(gemm_tf / fp8_peak, 4),
                          "traffic": traffic if M == 8192 else None,

@@ -70,6 +70,7 @@ struct MmParams {
   int M, N, K;
   int m_tiles, n_tiles, k_blocks, tiles_per_batch, tiles_total, group_m;
   int a_bcast, b_bcast;
+  int a_mn, b_mn;    // operand stored MN-major ([K][M] / [K][N], M or N contiguous)
   int64_t c_stride;  // elements between output batches
   const float* sinv_a;
   const float* sinv_b;
@@ -294,6 +295,21 @@ __device__ __forceinline__ uint64_t sdesc_k128(uint32_t saddr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major tile written by TMA with the
+// 128-byte swizzle: atoms of 8 K-rows x 128 bytes of M (or N), K-row groups
+// every 1024 bytes (stride byte offset), 128-element M/N groups `lbo` bytes
+// apart (leading byte offset), version 1, layout type 2.  One 32-deep K step
+// of the MMA covers 32 K-rows = 4096 bytes.
+__device__ __forceinline__ uint64_t sdesc_mn128(uint32_t saddr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= uint64_t((saddr & 0x3FFFFu) >> 4);
+  d |= uint64_t((lbo >> 4) & 0x3FFFu) << 16;
+  d |= uint64_t(1024 >> 4) << 32;
+  d |= uint64_t(1) << 46;
+  d |= uint64_t(2) << 61;
+  return d;
+}
+
 __device__ __forceinline__ void decode_tile(const MmParams& p, int t, int& b, int& mt, int& nt) {
   b = t / p.tiles_per_batch;
   const int r = t - b * p.tiles_per_batch;
@@ -384,17 +400,28 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
           }
           const uint32_t sa = sbase + stage * C::kABytes;
           const uint32_t sb = sbase + C::kStages * C::kABytes + stage * C::kBBytes;
+          // K-major boxes are [rows][128 K bytes] at (k, row); MN-major boxes
+          // are [128 K rows][128 M/N bytes] at (row, k), one per 128 rows.
+          uint32_t bar = full_bar(stage);
           if constexpr (PAIR == 1) {
-            mbar_arrive_expect_tx(full_bar(stage), C::kStageBytes);
-            tma_load_3d(sa, &tmA, kb * kBK, arow, ba, full_bar(stage));
-            tma_load_3d(sb, &tmB, kb * kBK, brow, bb, full_bar(stage));
+            mbar_arrive_expect_tx(bar, C::kStageBytes);
           } else {
             // Both CTAs' loads complete on the leader's barrier; the leader
             // expects the bytes of both.
-            if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * C::kStageBytes);
-            const uint32_t lbar = mapa_shared(full_bar(stage), 0);
-            tma_load_3d_pair(sa, &tmA, kb * kBK, arow, ba, lbar);
-            tma_load_3d_pair(sb, &tmB, kb * kBK, brow, bb, lbar);
+            if (leader) mbar_arrive_expect_tx(bar, 2 * C::kStageBytes);
+            bar = mapa_shared(bar, 0);
+          }
+          auto load = [&](uint32_t dst, const CUtensorMap* tm, int c0, int c1, int c2) {
+            if constexpr (PAIR == 1) tma_load_3d(dst, tm, c0, c1, c2, bar);
+            else tma_load_3d_pair(dst, tm, c0, c1, c2, bar);
+          };
+          if (p.a_mn) load(sa, &tmA, arow, kb * kBK, ba);
+          else load(sa, &tmA, kb * kBK, arow, ba);
+          if (p.b_mn) {
+#pragma unroll
+            for (int g = 0; g < C::kBRows / 128; ++g) load(sb + g * 16384u, &tmB, brow + 128 * g, kb * kBK, bb);
+          } else {
+            load(sb, &tmB, kb * kBK, brow, bb);
           }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -436,15 +463,20 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
             break;
           }
           tc_fence_after();
-          const uint64_t ad = sdesc_k128(sa0 + stage * C::kABytes);
-          const uint64_t bd = sdesc_k128(sb0 + stage * C::kBBytes);
+          // K-major: +32 bytes along K inside the swizzle atom (+2 in the
+          // address field) per MMA.  MN-major: +32 K-rows = 4096 bytes (+256).
+          const uint64_t ad = p.a_mn ? sdesc_mn128(sa0 + stage * C::kABytes, 16384u)
+                                     : sdesc_k128(sa0 + stage * C::kABytes);
+          const uint64_t bd = p.b_mn ? sdesc_mn128(sb0 + stage * C::kBBytes, 16384u)
+                                     : sdesc_k128(sb0 + stage * C::kBBytes);
+          const uint64_t astep = p.a_mn ? 256u : 2u;
+          const uint64_t bstep = p.b_mn ? 256u : 2u;
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k) {
-            // +32 bytes along K inside the swizzle atom = +2 in the address field.
             if constexpr (PAIR == 1)
-              umma_f8(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), p.idesc, (kb | k) != 0 ? 1u : 0u);
+              umma_f8(d, ad + astep * k, bd + bstep * k, p.idesc, (kb | k) != 0 ? 1u : 0u);
             else
-              umma_f8_pair(d, ad + uint64_t(2 * k), bd + uint64_t(2 * k), p.idesc, (kb | k) != 0 ? 1u : 0u);
+              umma_f8_pair(d, ad + astep * k, bd + bstep * k, p.idesc, (kb | k) != 0 ? 1u : 0u);
           }
           if constexpr (PAIR == 1) umma_commit(empty_bar(stage));
           else umma_commit_pair(empty_bar(stage));
@@ -629,6 +661,16 @@ bool make_map(CUtensorMap* m, const uint8_t* base, int64_t K, int64_t rows, int6
                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
+// 3-D map over an MN-major uint8 operand [batch, K, mn] (mn contiguous) with a
+// box of [1, 128 K rows, 128 mn bytes], 128B swizzle.
+bool make_map_mn(CUtensorMap* m, const uint8_t* base, int64_t K, int64_t mn, int64_t batch, int64_t bstride) {
+  const uint64_t dims[3] = {uint64_t(mn), uint64_t(K), uint64_t(batch)};
+  const uint64_t strides[2] = {uint64_t(mn), uint64_t(batch > 1 ? bstride : K * mn)};
+  const uint32_t box[3] = {128u, uint32_t(kBK), 1u};
+  return encode_tiled_cached(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+}
+
 // 3-D map over the bf16 output [batch, M, N] with a 32x32 box, 64B swizzle
 // (the staging-buffer layout the epilogue writes).
 bool make_out_map(CUtensorMap* m, uint16_t* base, int64_t M, int64_t N, int64_t batch, int64_t c_stride) {
@@ -700,8 +742,11 @@ int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t 
   CUtensorMap ta, tb, tc;
   const int64_t ba = (batch > 1 && strides[0] != 0) ? batch : 1;
   const int64_t bb = (batch > 1 && strides[1] != 0) ? batch : 1;
-  if (!make_map(&ta, A, K, M, ba, ba > 1 ? strides[0] : 0, kBM)) return FP8_ERR_CUDA;
-  if (!make_map(&tb, B, K, N, bb, bb > 1 ? strides[1] : 0, BN / PAIR)) return FP8_ERR_CUDA;
+  const bool okA = p.a_mn ? make_map_mn(&ta, A, K, M, ba, ba > 1 ? strides[0] : 0)
+                          : make_map(&ta, A, K, M, ba, ba > 1 ? strides[0] : 0, kBM);
+  const bool okB = p.b_mn ? make_map_mn(&tb, B, K, N, bb, bb > 1 ? strides[1] : 0)
+                          : make_map(&tb, B, K, N, bb, bb > 1 ? strides[1] : 0, BN / PAIR);
+  if (!okA || !okB) return FP8_ERR_CUDA;
   memset(&tc, 0, sizeof(tc));
   if (p.tma_store && !make_out_map(&tc, p.out, M, N, batch, p.c_stride)) return FP8_ERR_CUDA;
   p.a_bcast = ba == 1;
@@ -726,7 +771,7 @@ struct MmChoice {
   int bn, pair, slots;
 };
 
-MmChoice choose_mm(int64_t M, int64_t N, int64_t batch, int sms) {
+MmChoice choose_mm(int64_t M, int64_t N, int64_t batch, int sms, bool b_mn) {
   struct Opt {
     int bn, pair;
     double eff;
@@ -739,6 +784,7 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t batch, int sms) {
   double best_cost = 1e300;
   for (const Opt& o : opts) {
     if (o.pair == 2 && M <= kBM) continue;  // the second CTA would hold no rows
+    if (b_mn && o.bn / o.pair < 128) continue;
     const int slots = o.pair == 2 ? (o.bn == 256 ? max_pairs<256>(sms) : max_pairs<128>(sms)) : sms;
     const int64_t units = ((M + kBM * o.pair - 1) / (kBM * o.pair)) * ((N + o.bn - 1) / o.bn) * batch;
     const double waves = double((units + slots - 1) / slots);
@@ -760,7 +806,10 @@ extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, 
                       const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b,
                       const float* bias, uint16_t* out_bf16, fp8_stream_t stream) {
   if (M < 0 || N < 0 || K < 0 || batch < 1) return FP8_ERR_INVALID_ARG;
-  if ((layout & ~(FP8_MM_A_E5M2 | FP8_MM_B_E5M2)) != FP8_MM_NT) return FP8_ERR_INVALID_ARG;
+  if ((layout & ~(FP8_MM_A_E5M2 | FP8_MM_B_E5M2 | FP8_MM_A_MN_MAJOR | FP8_MM_B_MN_MAJOR)) != FP8_MM_NT)
+    return FP8_ERR_INVALID_ARG;
+  const bool a_mn = (layout & FP8_MM_A_MN_MAJOR) != 0;
+  const bool b_mn = (layout & FP8_MM_B_MN_MAJOR) != 0;
   if (batch > 1 && strides == nullptr) return FP8_ERR_INVALID_ARG;
   if (batch > 1 && (strides[0] < 0 || strides[1] < 0 || strides[2] < 0)) return FP8_ERR_INVALID_ARG;
   if (M == 0 || N == 0) return FP8_OK;
@@ -768,6 +817,7 @@ extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, 
   if (K > 0 && (A == nullptr || B == nullptr)) return FP8_ERR_INVALID_ARG;
   if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2 || batch > 65535) return FP8_ERR_UNSUPPORTED;
   if (K % 16 != 0) return FP8_ERR_UNSUPPORTED;
+  if ((a_mn && M % 16 != 0) || (b_mn && N % 16 != 0)) return FP8_ERR_UNSUPPORTED;  // MN-major row pitch
   if (reinterpret_cast<uintptr_t>(out_bf16) % 2 != 0) return FP8_ERR_UNSUPPORTED;
   const int64_t c_stride = batch > 1 ? strides[2] : M * N;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -801,12 +851,16 @@ extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, 
   const uint32_t fa = (layout & FP8_MM_A_E5M2) ? 1u : 0u;
   const uint32_t fb = (layout & FP8_MM_B_E5M2) ? 1u : 0u;
   // Instruction descriptor: fp32 accumulator (bits 4-5 = 1), A format bits 7-9,
-  // B format bits 10-12 (0 = E4M3, 1 = E5M2), both K-major; N/8 (bits 17-22)
-  // and M/16 (bits 24-28) are added by the launcher for its tile shape.
-  p.idesc = (1u << 4) | (fa << 7) | (fb << 10);
+  // B format bits 10-12 (0 = E4M3, 1 = E5M2), A/B major bits 15/16 (1 = MN-major);
+  // N/8 (bits 17-22) and M/16 (bits 24-28) are added by the launcher.
+  p.a_mn = a_mn;
+  p.b_mn = b_mn;
+  p.idesc = (1u << 4) | (fa << 7) | (fb << 10) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
   p.err = error_word_ptr();
 
-  const MmChoice c = choose_mm(M, N, batch, sms);
+  // An MN-major B is loaded as boxes of 128 N-rows, so its per-CTA tile must
+  // hold whole boxes (no 128-wide CTA pair).
+  const MmChoice c = choose_mm(M, N, batch, sms, b_mn);
   if (c.pair == 2) {
     if (c.bn == 256) return launch_mm<256, 2>(A, B, M, N, K, batch, strides, p, c.slots, st);
     return launch_mm<128, 2>(A, B, M, N, K, batch, strides, p, c.slots, st);

@@ -17,6 +17,8 @@ E4M3, E5M2 = 0, 1
 ROW, TRANSPOSED, DUAL = 0, 1, 2
 IN_DTYPE = {torch.bfloat16: 0, torch.float16: 1, torch.float32: 2}
 MM_NT = 0
+MM_A_MN_MAJOR = 1 << 0
+MM_B_MN_MAJOR = 1 << 1
 MM_A_E5M2 = 1 << 8
 MM_B_E5M2 = 1 << 9
 HISTORY_LEN = 16
@@ -166,24 +168,30 @@ def quantize(x, fmt, layout, ring, out=None, out_t=None, stream=None):
     return (out if layout in (ROW, DUAL) else None), (out_t if layout in (TRANSPOSED, DUAL) else None)
 
 
-def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream=None):
-    """fp8_mm: Y = bf16(a . b^T * sinv_a * sinv_b + bias).
+def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream=None,
+       a_mn_major=False, b_mn_major=False):
+    """fp8_mm: Y = bf16(A . B^T * sinv_a * sinv_b + bias).
 
-    a: uint8 [M, K] or [Ba, M, K]; b: uint8 [N, K] or [Bb, N, K] (K contiguous);
-    a size-1 (or 2-D) operand broadcasts over the batch at stride 0.
-    sinv_a / sinv_b: one-element float32 CUDA tensors.  bias: float32 [N] or None.
+    a: uint8 [M, K] or [Ba, M, K] (K contiguous), or with a_mn_major=True the
+    stored [K, M] / [Ba, K, M] (M contiguous); b likewise [N, K] or, with
+    b_mn_major=True, [K, N].  A size-1 (or 2-D) operand broadcasts over the
+    batch at stride 0.  sinv_a / sinv_b: one-element float32 CUDA tensors.
+    bias: float32 [N] or None.
     """
     if a.dtype != torch.uint8 or b.dtype != torch.uint8:
         raise ValueError("a and b hold FP8 codes as uint8")
-    layout = MM_NT | (MM_A_E5M2 if fmt_a == E5M2 else 0) | (MM_B_E5M2 if fmt_b == E5M2 else 0)
+    layout = (MM_NT | (MM_A_E5M2 if fmt_a == E5M2 else 0) | (MM_B_E5M2 if fmt_b == E5M2 else 0)
+              | (MM_A_MN_MAJOR if a_mn_major else 0) | (MM_B_MN_MAJOR if b_mn_major else 0))
     L = _LIB or lib()
     if a.dim() == 2 and b.dim() == 2:
-        M, K = a.shape
-        N = b.shape[0]
-        if b.shape[1] != K:
+        if (a_mn_major or b_mn_major) and not (a.is_contiguous() and b.is_contiguous()):
+            raise ValueError("operands must be contiguous")
+        K, M = a.shape if a_mn_major else (a.shape[1], a.shape[0])
+        Kb, N = b.shape if b_mn_major else (b.shape[1], b.shape[0])
+        if Kb != K:
             raise ValueError("K mismatch")
-        if K > 0 and ((M > 1 and a.stride(0) != K) or a.stride(1) != 1 or (N > 1 and b.stride(0) != K)
-                      or b.stride(1) != 1):
+        if not (a_mn_major or b_mn_major) and K > 0 and (
+                (M > 1 and a.stride(0) != K) or a.stride(1) != 1 or (N > 1 and b.stride(0) != K) or b.stride(1) != 1):
             raise ValueError("operands must be K-contiguous")
         if out is None:
             out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
@@ -196,13 +204,13 @@ def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream
     a3 = a if a.dim() == 3 else a.unsqueeze(0)
     b3 = b if b.dim() == 3 else b.unsqueeze(0)
     batch = max(a3.shape[0], b3.shape[0])
-    M, K = a3.shape[1], a3.shape[2]
-    N = b3.shape[1]
-    if b3.shape[2] != K:
+    K, M = (a3.shape[1], a3.shape[2]) if a_mn_major else (a3.shape[2], a3.shape[1])
+    Kb, N = (b3.shape[1], b3.shape[2]) if b_mn_major else (b3.shape[2], b3.shape[1])
+    if Kb != K:
         raise ValueError("K mismatch")
     for t in (a3, b3):
-        if t.shape[0] not in (1, batch) or (K > 0 and t.shape[1] > 1 and (t.stride(2) != 1 or t.stride(1) != K)):
-            raise ValueError("operands must be K-contiguous with matching batch")
+        if t.shape[0] not in (1, batch) or (t.numel() > 0 and (t.stride(2) != 1 or t.stride(1) != t.shape[2])):
+            raise ValueError("operands must be contiguous in their last two dims with matching batch")
     sa = 0 if a3.shape[0] == 1 else a3.stride(0)
     sb = 0 if b3.shape[0] == 1 else b3.stride(0)
     if out is None:

@@ -137,11 +137,19 @@ int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layo
 int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
                                 fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);
 
-/* fp8_mm layout word: FP8_MM_NT plus the operand format bits.  NT means A is
- * [M, K] and B is [N, K], both with K contiguous. */
+/* fp8_mm layout word: FP8_MM_NT plus optional operand-layout and format bits.
+ * NT means A is [M, K] and B is [N, K], both with K contiguous (K-major).
+ * The MN-major bits fold a transposed view into the layout tag at zero copy
+ * (3D batched commit, "tests/extension" page: inner .t() views fold into the
+ * layout tag): with FP8_MM_A_MN_MAJOR, A is stored [K, M] (M contiguous);
+ * with FP8_MM_B_MN_MAJOR, B is stored [K, N] (N contiguous).  So dX = G.W
+ * takes W as quantized ([N_out, N_in] = [K, N]) and dW = G^T.X takes G and X
+ * as quantized, with no transposed copies. */
 #define FP8_MM_NT 0
-#define FP8_MM_A_E5M2 (1 << 8) /* A holds E5M2 codes (default E4M3) */
-#define FP8_MM_B_E5M2 (1 << 9) /* B holds E5M2 codes (default E4M3) */
+#define FP8_MM_A_MN_MAJOR (1 << 0) /* A stored [K, M]; needs M % 16 == 0 */
+#define FP8_MM_B_MN_MAJOR (1 << 1) /* B stored [K, N]; needs N % 16 == 0 */
+#define FP8_MM_A_E5M2 (1 << 8)     /* A holds E5M2 codes (default E4M3) */
+#define FP8_MM_B_E5M2 (1 << 9)     /* B holds E5M2 codes (default E4M3) */
 
 /*
  * fp8_mm -- scaled FP8 GEMM with fused scale, bias and bf16 rounding.
@@ -152,8 +160,10 @@ int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t
  * (bias-fusion commit: the fp32 bias is added before the single bf16
  * rounding; 3D batched commit: size-1 batches broadcast with stride 0).
  *
- * A       uint8 FP8 codes, element (b,m,k) at A[b*strides[0] + m*K + k].
- * B       uint8 FP8 codes, element (b,n,k) at B[b*strides[1] + n*K + k].
+ * A       uint8 FP8 codes, element (b,m,k) at A[b*strides[0] + m*K + k]
+ *         (FP8_MM_A_MN_MAJOR: at A[b*strides[0] + k*M + m]).
+ * B       uint8 FP8 codes, element (b,n,k) at B[b*strides[1] + n*K + k]
+ *         (FP8_MM_B_MN_MAJOR: at B[b*strides[1] + k*N + n]).
  * out_bf16 bfloat16 (uint16 storage), element (b,m,n) at
  *         out_bf16[b*strides[2] + m*N + n].
  * strides host array of 3 int64 batch strides in elements; may be NULL when
@@ -167,7 +177,8 @@ int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t
  *         Y = bf16(bias) (or 0).
  * Errors: FP8_ERR_INVALID_ARG (negative size, batch < 1, NULL A/B/out/sinv,
  *         unknown layout bits, NULL strides with batch > 1);
- *         FP8_ERR_UNSUPPORTED (K % 16 != 0, A/B/stride not 16-byte aligned,
+ *         FP8_ERR_UNSUPPORTED (K % 16 != 0, an MN-major operand whose M or N
+ *         is not a multiple of 16, A/B/stride not 16-byte aligned,
  *         out_bf16 not 2-byte aligned, a dimension beyond 2^31);
  *         FP8_ERR_CUDA (descriptor encoding or launch failed).
  */

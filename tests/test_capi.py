@@ -76,8 +76,10 @@ def _mm(L, M=128, N=128, K=128, batch=1, strides=None, layout=0, A=0x10000, B=0x
 def test_mm_rejects_bad_arguments_without_cuda(L):
     assert _mm(L, M=-1) == ops.FP8_ERR_INVALID_ARG
     assert _mm(L, batch=0) == ops.FP8_ERR_INVALID_ARG
-    assert _mm(L, layout=1) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, layout=1 << 2) == ops.FP8_ERR_INVALID_ARG
     assert _mm(L, layout=1 << 10) == ops.FP8_ERR_INVALID_ARG
+    assert _mm(L, layout=ops.MM_A_MN_MAJOR, M=24) == ops.FP8_ERR_UNSUPPORTED  # [K, M] rows need M % 16 == 0
+    assert _mm(L, layout=ops.MM_B_MN_MAJOR, N=40) == ops.FP8_ERR_UNSUPPORTED
     assert _mm(L, batch=2, strides=None) == ops.FP8_ERR_INVALID_ARG
     assert _mm(L, batch=2, strides=(-16, 0, 0)) == ops.FP8_ERR_INVALID_ARG
     assert _mm(L, out=0) == ops.FP8_ERR_INVALID_ARG

@@ -132,3 +132,50 @@ def test_pr1_linear_end_to_end():
 def test_device_error_word_clear():
     rc, where = ops.device_error(clear=True)
     assert rc == ops.FP8_OK and where == 0
+
+
+# MN-major operands (the layout tag): A stored [K, M] and/or B stored [K, N];
+# the oracle multiplies the untransposed codes.  M/N multiples of 16 (row
+# pitch of the stored operand); K tails inside a 128-deep stage; M <= 128 runs
+# the single-CTA kernel, larger M the CTA pair.
+@pytest.mark.parametrize("a_mn,b_mn", [(True, False), (False, True), (True, True)])
+@pytest.mark.parametrize("M,N,K", [(64, 256, 256), (128, 128, 160), (208, 304, 400), (512, 1536, 640),
+                                   (1536, 1536, 2048)])
+def test_mn_major_layouts(M, N, K, a_mn, b_mn):
+    a = S.fp8_codes((M, K), seed=M + K)
+    b = S.fp8_codes((N, K), seed=N + K + 1)
+    bias = S.uniform((N,), seed=7)
+    ad = a.t().contiguous().cuda() if a_mn else a.cuda()
+    bd = b.t().contiguous().cuda() if b_mn else b.cuda()
+    y = ops.mm(ad, bd, _scalar(0.5), _scalar(0.25), bias.cuda(), a_mn_major=a_mn, b_mn_major=b_mn)
+    torch.cuda.synchronize()
+    assert y.shape == (M, N)
+    mm_check(y, a.numpy(), b.numpy(), ops.E4M3, ops.E4M3, np.float32(0.5), np.float32(0.25), bias.numpy())
+
+
+def test_mn_major_backward_shapes_mixed_formats():
+    """The step's dX (B = W as quantized) and dW (A = G, B = X as quantized) with an E5M2 gradient."""
+    Mtok, n_out, hid = 512, 4096, 1536
+    g = S.fp8_codes((Mtok, n_out), seed=31, fmt=ops.E5M2)
+    w = S.fp8_codes((n_out, hid), seed=32)
+    x = S.fp8_codes((Mtok, hid), seed=33)
+    dx = ops.mm(g.cuda(), w.cuda(), _scalar(0.01), _scalar(2.0), fmt_a=ops.E5M2, b_mn_major=True)
+    dw = ops.mm(g.cuda(), x.cuda(), _scalar(0.01), _scalar(0.5), fmt_a=ops.E5M2, a_mn_major=True, b_mn_major=True)
+    torch.cuda.synchronize()
+    rows = np.array([0, 1, 255, 511])
+    mm_check(dx, g.numpy(), w.numpy().T.copy(), ops.E5M2, ops.E4M3, np.float32(0.01), np.float32(2.0), None, rows)
+    rows = np.array([0, 100, 4095])
+    mm_check(dw, g.numpy().T.copy(), x.numpy().T.copy(), ops.E5M2, ops.E4M3, np.float32(0.01), np.float32(0.5),
+             None, rows)
+
+
+def test_mn_major_batched_broadcast():
+    a = S.fp8_codes((4, 256, 192), seed=41)            # [batch, K, M]
+    b = S.fp8_codes((1, 256, 160), seed=42)            # [1, K, N] broadcast
+    y = ops.mm(a.cuda(), b.cuda(), _scalar(1.0), _scalar(1.0), a_mn_major=True, b_mn_major=True)
+    torch.cuda.synchronize()
+    assert y.shape == (4, 192, 160)
+    for z in range(4):
+        ref, Ssum = OG.mm_fp8(a[z].numpy().T.copy(), b[0].numpy().T.copy(), 0, 0, 1.0, 1.0)
+        ok, ratio = OG.check(y[z].float().cpu().numpy(), ref, Ssum)
+        assert ok, (z, ratio)

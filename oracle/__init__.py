@@ -31,10 +31,11 @@ Modules:
   fp8_formats -- decode table and encoder (RNE + saturation) per format.
   recipe      -- amax, quantize in row/transposed/dual layout, ring fold.
   gemm        -- fp64 scaled GEMM, |a.b| sums and the acceptance bound.
+  bias_grad   -- column sums of the output gradient (the bias gradient).
 
 Parity status: every function is pinned by ``tests/test_oracle_*.py``
 except the treatment of NaN inputs and of a non-finite history maximum,
 which no workload exercises ("parity unpinned" for those two cases).
 """
 
-from . import fp8_formats, recipe, gemm  # noqa: F401
+from . import fp8_formats, recipe, gemm, bias_grad  # noqa: F401

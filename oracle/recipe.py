@@ -113,3 +113,37 @@ def quantize(x, fmt, layout, ring):
     out_t = np.ascontiguousarray(q.T) if layout in (TRANSPOSED, DUAL) else None
     fold(ring, a, fmt)
     return out, out_t, a
+
+
+def current_scale(a, fmt):
+    """Current (dynamic) scaling: fp32(FP8_MAX / amax) of this tensor's own amax.
+
+    The pages' DynamicScaling path ("AstrAI commits, branch main,
+    tests/extension", FP8Recipe commit: a dynamic flag, no rings, scales
+    measured inline).  Reading: an amax of 0 (or a non-finite amax or
+    quotient) gives scale 1.
+    """
+    a = np.float32(a)
+    fmax = np.float32(F.fp8_max(fmt))
+    if a > 0 and np.isfinite(a):
+        with np.errstate(over="ignore"):
+            c = np.float32(fmax / a)
+        if np.isfinite(c) and c > 0:
+            return c
+    return np.float32(1.0)
+
+
+def quantize_current(x, fmt, layout):
+    """Current scaling: returns (out, out_t, amax, scale, scale_inv).
+
+    amax over the raw values, scale from this amax, codes of fp32(x*scale),
+    scale_inv = fp32(1/scale).  No history.
+    """
+    xf = to_float32(x)
+    assert xf.ndim == 2
+    a = amax(xf)
+    s = current_scale(a, fmt)
+    q = scaled_codes(xf, s, fmt)
+    out = q if layout in (ROW, DUAL) else None
+    out_t = np.ascontiguousarray(q.T) if layout in (TRANSPOSED, DUAL) else None
+    return out, out_t, a, s, np.float32(np.float32(1.0) / s)

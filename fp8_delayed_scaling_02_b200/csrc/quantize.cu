@@ -247,6 +247,7 @@ struct RingCache {
 
 __device__ __forceinline__ RingCache prefetch_ring(const RingArgs& ring) {
   RingCache c{0.0f, 0};
+  if (ring.history == nullptr) return c;  // fixed scale (current scaling's cast pass)
   if (threadIdx.x < kHistoryLen) c.hist = ring.history[threadIdx.x];
   if (threadIdx.x == kHistoryLen) c.idx = *ring.idx;
   return c;
@@ -266,6 +267,19 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
   if (threadIdx.x < kHistoryLen) hist_s[threadIdx.x] = rc.hist;
   if (threadIdx.x == kHistoryLen) idx_s = rc.idx;
   __syncthreads();
+  if (ring.history == nullptr) {
+    // Fixed scale: no amax to publish; the last block clears the scratch
+    // words (the tile counter is shared by every kernel that claims tiles).
+    if (threadIdx.x == 0) {
+      unsigned t;
+      asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(ring.scratch + 1) : "memory");
+      if (t == gridDim.x - 1) {
+        asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ring.scratch + 1) : "memory");
+        asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ring.scratch + 2) : "memory");
+      }
+    }
+    return;
+  }
   if (threadIdx.x == 0) {
     float m = 0.0f;
 #pragma unroll
@@ -745,6 +759,79 @@ __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __g
   amax_ticket_fold<FMT, kWsThreads>(amax, a.ring, s, rc);
 }
 
+// ---- current scaling: amax pass ---------------------------------------------------
+//
+// Current (dynamic) scaling measures the scale from the tensor itself: this
+// pass reduces amax exactly as the quantize kernels do (16-byte loads, warp
+// shuffle, one relaxed atomic max per block, acq_rel ticket), and the block
+// that takes the last ticket publishes scale = FP8_MAX / amax (1 when amax is
+// zero or the quotient is not finite), scale_inv = 1 / scale and amax, then
+// clears the scratch words.  The cast pass that follows reads that scale.
+
+struct AmaxArgs {
+  const uint8_t* in;
+  int64_t n, head, nchunks;  // head: scalar elements before the first 16-byte aligned input chunk
+  uint32_t* scratch;
+  float* scale;
+  float* scale_inv;
+  float* amax_out;
+};
+
+template <int DT, int FMT>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const AmaxArgs a) {
+  constexpr int kB = In<DT>::kBytes;
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
+  float amax = 0.0f;
+  const int64_t tid = int64_t(blockIdx.x) * kThreads + threadIdx.x;
+  const int64_t nthr = int64_t(gridDim.x) * kThreads;
+  const int64_t tail0 = a.head + 16 * a.nchunks;
+  if (tid < a.head) amax = fmaxf(amax, fabsf(load_one<DT>(a.in + tid * kB)));
+  if (tid < a.n - tail0) amax = fmaxf(amax, fabsf(load_one<DT>(a.in + (tail0 + tid) * kB)));
+  for (int64_t j = tid; j < a.nchunks; j += 2 * nthr) {
+    float v[16], w[16];
+    const bool two = j + nthr < a.nchunks;
+    load_vec_aligned<DT, 16>(a.in + (a.head + 16 * j) * kB, v);
+    if (two) load_vec_aligned<DT, 16>(a.in + (a.head + 16 * (j + nthr)) * kB, w);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(v[i]));
+    if (two) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(w[i]));
+    }
+  }
+  __shared__ float warp_max[kThreads / 32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if (lane == 0) warp_max[warp] = amax;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float m = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) m = fmaxf(m, warp_max[w]);
+    if (m > 0.0f)
+      asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(a.scratch), "r"(__float_as_uint(m)) : "memory");
+    unsigned t;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(a.scratch + 1) : "memory");
+    if (t == gridDim.x - 1) {
+      uint32_t bits;
+      asm volatile("atom.relaxed.gpu.global.exch.b32 %0, [%1], 0;" : "=r"(bits) : "l"(a.scratch) : "memory");
+      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(a.scratch + 1) : "memory");
+      const float am = __uint_as_float(bits);
+      const float fmax = FMT == FP8_E4M3 ? kE4M3Max : kE5M2Max;
+      float sc = 1.0f;
+      if (am > 0.0f && isfinite(am)) {
+        const float c = __fdiv_rn(fmax, am);
+        if (isfinite(c) && c > 0.0f) sc = c;
+      }
+      *a.scale = sc;
+      *a.scale_inv = __frcp_rn(sc);
+      if (a.amax_out) *a.amax_out = am;
+    }
+  }
+}
+
 // ---- host side ---------------------------------------------------------------
 
 int sm_count_current() {
@@ -837,26 +924,16 @@ int dispatch_fmt_tile_tma(int fmt, const TileArgs& a, const CUtensorMap& map, in
 
 using namespace fp8ds;
 
-extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
-                            fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream) {
-  if (dtype < FP8_IN_BF16 || dtype > FP8_IN_FP32) return FP8_ERR_INVALID_ARG;
-  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
-  if (layout < FP8_LAYOUT_ROW || layout > FP8_LAYOUT_DUAL) return FP8_ERR_INVALID_ARG;
-  if (rows < 0 || cols < 0) return FP8_ERR_INVALID_ARG;
-  if (cols > 0 && rows > INT64_MAX / cols) return FP8_ERR_INVALID_ARG;
-  if (!ring.history || !ring.idx || !ring.scale || !ring.scale_inv || !ring.scratch) return FP8_ERR_INVALID_ARG;
+namespace fp8ds {
+namespace {
+// Launches the cast kernel for the layout (and the ring fold unless r.history
+// is null).  Arguments are already validated.
+int quantize_dispatch(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt, const RingArgs& r,
+                      uint8_t* out, uint8_t* out_t, cudaStream_t st) {
   const int64_t n = rows * cols;
-  if (n > 0 && in == nullptr) return FP8_ERR_INVALID_ARG;
-  if ((layout == FP8_LAYOUT_ROW || layout == FP8_LAYOUT_DUAL) && n > 0 && out == nullptr) return FP8_ERR_INVALID_ARG;
-  if ((layout == FP8_LAYOUT_T || layout == FP8_LAYOUT_DUAL) && n > 0 && out_t == nullptr) return FP8_ERR_INVALID_ARG;
   const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
-  if (reinterpret_cast<uintptr_t>(in) % eb != 0) return FP8_ERR_UNSUPPORTED;
-  if (reinterpret_cast<uintptr_t>(ring.scratch) % 8 != 0) return FP8_ERR_UNSUPPORTED;
-
   const int sms = sm_count_current();
   if (sms <= 0) return FP8_ERR_CUDA;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const RingArgs r{ring.history, ring.idx, ring.scale, ring.scale_inv, ring.scratch};
   const int max_grid = sms * (2048 / kThreads);
 
   if (layout == FP8_LAYOUT_ROW) {
@@ -907,6 +984,75 @@ extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t col
     case FP8_IN_FP16: return dispatch_fmt_tile<FP8_IN_FP16>(fmt, a, grid, st, dual);
     default: return dispatch_fmt_tile<FP8_IN_FP32>(fmt, a, grid, st, dual);
   }
+}
+
+}  // namespace
+}  // namespace fp8ds
+
+// Argument checks shared by the quantize entry points; FP8_OK if the call may
+// proceed.
+static int check_quantize_args(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
+                               uint8_t* out, uint8_t* out_t, const uint32_t* scratch) {
+  if (dtype < FP8_IN_BF16 || dtype > FP8_IN_FP32) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  if (layout < FP8_LAYOUT_ROW || layout > FP8_LAYOUT_DUAL) return FP8_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0) return FP8_ERR_INVALID_ARG;
+  if (cols > 0 && rows > INT64_MAX / cols) return FP8_ERR_INVALID_ARG;
+  if (scratch == nullptr) return FP8_ERR_INVALID_ARG;
+  const int64_t n = rows * cols;
+  if (n > 0 && in == nullptr) return FP8_ERR_INVALID_ARG;
+  if ((layout == FP8_LAYOUT_ROW || layout == FP8_LAYOUT_DUAL) && n > 0 && out == nullptr) return FP8_ERR_INVALID_ARG;
+  if ((layout == FP8_LAYOUT_T || layout == FP8_LAYOUT_DUAL) && n > 0 && out_t == nullptr) return FP8_ERR_INVALID_ARG;
+  const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
+  if (reinterpret_cast<uintptr_t>(in) % eb != 0) return FP8_ERR_UNSUPPORTED;
+  if (reinterpret_cast<uintptr_t>(scratch) % 8 != 0) return FP8_ERR_UNSUPPORTED;
+  return FP8_OK;
+}
+
+extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
+                            fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream) {
+  if (!ring.history || !ring.idx || !ring.scale || !ring.scale_inv || !ring.scratch) return FP8_ERR_INVALID_ARG;
+  const int rc = check_quantize_args(in, dtype, rows, cols, layout, fmt, out, out_t, ring.scratch);
+  if (rc != FP8_OK) return rc;
+  const RingArgs r{ring.history, ring.idx, ring.scale, ring.scale_inv, ring.scratch};
+  return quantize_dispatch(in, dtype, rows, cols, layout, fmt, r, out, out_t, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int fp8_quantize_current(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
+                                    float* scale, float* scale_inv, float* amax, uint32_t* scratch, uint8_t* out,
+                                    uint8_t* out_t, fp8_stream_t stream) {
+  if (scale == nullptr || scale_inv == nullptr) return FP8_ERR_INVALID_ARG;
+  const int rc = check_quantize_args(in, dtype, rows, cols, layout, fmt, out, out_t, scratch);
+  if (rc != FP8_OK) return rc;
+  const int sms = sm_count_current();
+  if (sms <= 0) return FP8_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n = rows * cols;
+  const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
+  AmaxArgs a{};
+  a.in = static_cast<const uint8_t*>(in);
+  a.n = n;
+  const uintptr_t ia = reinterpret_cast<uintptr_t>(in);
+  a.head = std::min<int64_t>(n, int64_t(((16 - (ia & 15)) & 15) / eb));
+  a.nchunks = (n - a.head) / 16;
+  a.scratch = scratch;
+  a.scale = scale;
+  a.scale_inv = scale_inv;
+  a.amax_out = amax;
+  const int64_t want = (a.nchunks + 2 * kThreads - 1) / (2 * kThreads);
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sms) * (2048 / kThreads))));
+  cudaError_t e;
+  switch (dtype * 2 + fmt) {
+    case 0: e = launch_pdl(amax_kernel<FP8_IN_BF16, FP8_E4M3>, grid, kThreads, 0, st, 1, a); break;
+    case 1: e = launch_pdl(amax_kernel<FP8_IN_BF16, FP8_E5M2>, grid, kThreads, 0, st, 1, a); break;
+    case 2: e = launch_pdl(amax_kernel<FP8_IN_FP16, FP8_E4M3>, grid, kThreads, 0, st, 1, a); break;
+    case 3: e = launch_pdl(amax_kernel<FP8_IN_FP16, FP8_E5M2>, grid, kThreads, 0, st, 1, a); break;
+    case 4: e = launch_pdl(amax_kernel<FP8_IN_FP32, FP8_E4M3>, grid, kThreads, 0, st, 1, a); break;
+    default: e = launch_pdl(amax_kernel<FP8_IN_FP32, FP8_E5M2>, grid, kThreads, 0, st, 1, a); break;
+  }
+  if (e != cudaSuccess) return FP8_ERR_CUDA;
+  const RingArgs r{nullptr, nullptr, scale, scale_inv, scratch};
+  return quantize_dispatch(in, dtype, rows, cols, layout, fmt, r, out, out_t, st);
 }
 
 // ---- variant for callers that cannot allocate --------------------------------

@@ -70,6 +70,10 @@ def lib():
         L.fp8_device_error.restype = i32
         L.fp8_device_info.argtypes = [ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_char_p)]
         L.fp8_device_info.restype = i32
+        L.fp8_quantize_current.argtypes = [vp, i32, i64, i64, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+        L.fp8_quantize_current.restype = i32
+        L.fp8_bias_grad.argtypes = [vp, i32, i64, i64, vp, vp]
+        L.fp8_bias_grad.restype = i32
         _LIB = L
     return _LIB
 
@@ -220,6 +224,64 @@ def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream
     rc = L.fp8_mm(a3.data_ptr(), b3.data_ptr(), M, N, K, batch, strides, layout, sinv_a.data_ptr(),
                   sinv_b.data_ptr(), _ptr(bias), out3.data_ptr(), _stream(stream, a.get_device()))
     _check(rc, "fp8_mm")
+    return out
+
+
+class CurrentScale:
+    """Device state of current (dynamic) scaling: scale, scale_inv, amax and 4 scratch words."""
+
+    def __init__(self, device="cuda"):
+        self.buf = torch.zeros(8, dtype=torch.int32, device=device)
+
+    @property
+    def scale(self):
+        return self.buf[0:1].view(torch.float32)
+
+    @property
+    def scale_inv(self):
+        return self.buf[1:2].view(torch.float32)
+
+    @property
+    def amax(self):
+        return self.buf[2:3].view(torch.float32)
+
+    @property
+    def scratch(self):
+        return self.buf[4:8]
+
+
+def quantize_current(x, fmt, layout, cs, out=None, out_t=None, stream=None):
+    """fp8_quantize_current: scale from this tensor's amax (no history).
+
+    ``cs`` is a CurrentScale; after the call it holds scale, scale_inv and amax.
+    Returns (out, out_t) like ``quantize``.
+    """
+    if x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D tensor")
+    rows, cols = x.shape
+    if layout in (ROW, DUAL) and out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if layout in (TRANSPOSED, DUAL) and out_t is None:
+        out_t = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+    rc = (_LIB or lib()).fp8_quantize_current(
+        x.data_ptr(), IN_DTYPE[x.dtype], rows, cols, layout, fmt, cs.scale.data_ptr(), cs.scale_inv.data_ptr(),
+        cs.amax.data_ptr(), cs.scratch.data_ptr(), _ptr(out if layout in (ROW, DUAL) else None),
+        _ptr(out_t if layout in (TRANSPOSED, DUAL) else None), _stream(stream, x.get_device()))
+    _check(rc, "fp8_quantize_current")
+    return (out if layout in (ROW, DUAL) else None), (out_t if layout in (TRANSPOSED, DUAL) else None)
+
+
+def bias_grad(g, out=None, stream=None):
+    """fp8_bias_grad: float32 column sums of a 2-D (or flattened) gradient."""
+    g2 = g.reshape(-1, g.shape[-1])
+    if not g2.is_contiguous():
+        raise ValueError("g must be contiguous")
+    rows, cols = g2.shape
+    if out is None:
+        out = torch.empty(cols, dtype=torch.float32, device=g.device)
+    rc = (_LIB or lib()).fp8_bias_grad(g2.data_ptr(), IN_DTYPE[g2.dtype], rows, cols, out.data_ptr(),
+                                       _stream(stream, g.get_device()))
+    _check(rc, "fp8_bias_grad")
     return out
 
 

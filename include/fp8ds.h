@@ -137,6 +137,43 @@ int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layo
 int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
                                 fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);
 
+/*
+ * fp8_quantize_current -- current (dynamic) scaling cast to FP8, no ring.
+ *
+ * The DynamicScaling path of the FP8Recipe commit ("tests/extension" page:
+ * a dynamic flag, zero rings, scales measured inline): the scale comes from
+ * this tensor's own amax instead of a history of earlier ones.
+ *   amax  = max |x| over the raw values (NaN ignored)
+ *   scale = FP8_MAX / amax (fp32, round-to-nearest); 1 when amax is 0 or the
+ *           quotient is not finite
+ *   q     = saturate_rne_fp8(fp32(x) * scale)
+ *   scale_inv = 1 / scale (the GEMM's dequantisation factor)
+ * Two kernels on `stream`: an amax pass and the cast (the cast re-reads x,
+ * mostly from L2 for tensors that fit there).
+ * scale, scale_inv  device float[1] each, written (required).
+ * amax              device float[1], written, or NULL.
+ * scratch           device uint32[4], 8-byte aligned, zero before the call;
+ *                   left at zero.
+ * Other arguments and errors as fp8_quantize.
+ */
+int fp8_quantize_current(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt, float* scale,
+                         float* scale_inv, float* amax, uint32_t* scratch, uint8_t* out, uint8_t* out_t,
+                         fp8_stream_t stream);
+
+/*
+ * fp8_bias_grad -- bias gradient of the linear: db[c] = sum_r g[r, c].
+ *
+ * The _LinearFp8 backward fix ("tests/extension" page) reduces grad_b over
+ * all leading dimensions of the bf16 output gradient; callers pass G
+ * flattened to [rows, cols] (row-major, contiguous, element type `dtype`).
+ * The float32 sums are deterministic (fixed summation order, no atomics).
+ * db      device float[cols], written.
+ * Errors: FP8_ERR_INVALID_ARG (bad dtype, negative size, NULL db or g);
+ *         FP8_ERR_UNSUPPORTED (g not aligned to its element size);
+ *         FP8_ERR_CUDA (launch failed).  cols == 0 is a no-op.
+ */
+int fp8_bias_grad(const void* g, int dtype, int64_t rows, int64_t cols, float* db, fp8_stream_t stream);
+
 /* fp8_mm layout word: FP8_MM_NT plus optional operand-layout and format bits.
  * NT means A is [M, K] and B is [N, K], both with K contiguous (K-major).
  * The MN-major bits fold a transposed view into the layout tag at zero copy

@@ -74,6 +74,10 @@ def lib():
         L.fp8_quantize_current.restype = i32
         L.fp8_bias_grad.argtypes = [vp, i32, i64, i64, vp, vp]
         L.fp8_bias_grad.restype = i32
+        L.fp8_linear_forward.argtypes = [vp, i32, vp, i32, i64, i64, i64, vp, CRing, CRing, vp, vp, vp, vp]
+        L.fp8_linear_forward.restype = i32
+        L.fp8_linear_backward.argtypes = [vp, i32, i64, i64, i64, CRing, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.fp8_linear_backward.restype = i32
         _LIB = L
     return _LIB
 
@@ -283,6 +287,50 @@ def bias_grad(g, out=None, stream=None):
                                        _stream(stream, g.get_device()))
     _check(rc, "fp8_bias_grad")
     return out
+
+
+class Linear:
+    """One FP8 delayed-scaling linear through fp8_linear_forward / fp8_linear_backward.
+
+    Holds the three rings (x, w, g) and the quantized operands the backward
+    reuses; weights and bias are passed per call (they change every step).
+    """
+
+    def __init__(self, device="cuda"):
+        self.rx, self.rw, self.rg = Ring(device), Ring(device), Ring(device)
+        self.xq = self.wq = self.gq = None
+
+    def forward(self, x, w, bias=None, y=None, stream=None):
+        M, K = x.shape
+        N = w.shape[0]
+        dev = x.device
+        if self.xq is None or self.xq.shape != (M, K):
+            self.xq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        if self.wq is None or self.wq.shape != (N, K):
+            self.wq = torch.empty((N, K), dtype=torch.uint8, device=dev)
+        if y is None:
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        rc = (_LIB or lib()).fp8_linear_forward(
+            x.data_ptr(), IN_DTYPE[x.dtype], w.data_ptr(), IN_DTYPE[w.dtype], M, N, K, _ptr(bias), self.rx.c(),
+            self.rw.c(), self.xq.data_ptr(), self.wq.data_ptr(), y.data_ptr(), _stream(stream, x.get_device()))
+        _check(rc, "fp8_linear_forward")
+        return y
+
+    def backward(self, g, need_dx=True, need_dw=True, need_db=True, stream=None):
+        M, N = g.shape
+        K = self.xq.shape[1]
+        dev = g.device
+        if self.gq is None or self.gq.shape != (M, N):
+            self.gq = torch.empty((M, N), dtype=torch.uint8, device=dev)
+        dx = torch.empty((M, K), dtype=torch.bfloat16, device=dev) if need_dx else None
+        dw = torch.empty((N, K), dtype=torch.bfloat16, device=dev) if need_dw else None
+        db = torch.empty(N, dtype=torch.float32, device=dev) if need_db else None
+        rc = (_LIB or lib()).fp8_linear_backward(
+            g.data_ptr(), IN_DTYPE[g.dtype], M, N, K, self.rg.c(), self.xq.data_ptr(), self.wq.data_ptr(),
+            self.rx.scale_inv.data_ptr(), self.rw.scale_inv.data_ptr(), self.gq.data_ptr(), _ptr(dx), _ptr(dw),
+            _ptr(db), _stream(stream, g.get_device()))
+        _check(rc, "fp8_linear_backward")
+        return dx, dw, db
 
 
 def device_error(clear=True):

@@ -223,6 +223,35 @@ int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, 
            const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b,
            const float* bias, uint16_t* out_bf16, fp8_stream_t stream);
 
+/*
+ * fp8_linear_forward / fp8_linear_backward -- one FP8 delayed-scaling linear.
+ *
+ * The _LinearFp8 forward/backward pair of the "tests/extension" page (the
+ * forward captures its scales for the backward; grad_b is reduced over the
+ * leading dims), composed from the calls above on one stream:
+ *   forward:  Xq = quantize(X [M,K], E4M3, ring_x); Wq = quantize(W [N,K],
+ *             E4M3, ring_w); Y [M,N] = bf16(Xq.Wq^T * sinv_x * sinv_w + bias).
+ *   backward: Gq = quantize(G [M,N], E5M2, ring_g);
+ *             dX [M,K] = bf16(Gq.Wq * sinv_g * sinv_w)   (Wq read MN-major),
+ *             dW [N,K] = bf16(Gq^T.Xq * sinv_g * sinv_x) (Gq, Xq read MN-major),
+ *             db [N]   = column sums of G (float32, deterministic).
+ * All quantizes use the row layout: the layout tag replaces the transposed
+ * copies.  xq [M,K], wq [N,K], gq [M,N] are caller-owned uint8 buffers; the
+ * backward reads the forward's xq, wq and their scale_inv (pass ring_x.
+ * scale_inv and ring_w.scale_inv; valid while X and W are not quantized
+ * again in between).  dx, dw or db may be NULL to skip that output.
+ * Sizes: K % 16 == 0 (forward); backward also M % 16 == 0 (dW reduces over
+ * tokens) and N % 16 == 0 (MN-major row pitch).
+ * Errors: those of the calls it makes; the first failure is returned and
+ * the later steps are not launched.
+ */
+int fp8_linear_forward(const void* x, int x_dtype, const void* w, int w_dtype, int64_t M, int64_t N, int64_t K,
+                       const float* bias, fp8_ring ring_x, fp8_ring ring_w, uint8_t* xq, uint8_t* wq, uint16_t* y,
+                       fp8_stream_t stream);
+int fp8_linear_backward(const void* g, int g_dtype, int64_t M, int64_t N, int64_t K, fp8_ring ring_g,
+                        const uint8_t* xq, const uint8_t* wq, const float* sinv_x, const float* sinv_w, uint8_t* gq,
+                        uint16_t* dx, uint16_t* dw, float* db, fp8_stream_t stream);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fp8_status_string(int status);
 

@@ -84,3 +84,41 @@ def test_bias_grad_exact_on_integers_and_3d():
     db = ops.bias_grad(g.cuda())
     torch.cuda.synchronize()
     assert np.array_equal(db.cpu().numpy().astype(np.float64), OB.bias_grad(g.reshape(-1, 96)))
+
+
+def test_linear_composite_matches_the_separate_calls_and_oracle():
+    """fp8_linear_forward/backward over 3 delayed steps equal, bit for bit, the
+    same sequence of individual calls, and the last step matches the oracle."""
+    from oracle import gemm as OG
+
+    M, N, K = 256, 384, 512
+    lin = ops.Linear()
+    rx, rw, rg = ops.Ring(), ops.Ring(), ops.Ring()
+    for step in range(3):
+        x = S.normal_with_outliers((M, K), seed=60 + step, frac=0.01, mult=20.0).cuda()
+        w = S.normal_with_outliers((N, K), seed=70 + step, std=0.02).cuda()
+        g = S.normal_with_outliers((M, N), seed=80 + step, std=1e-3).cuda()
+        bias = S.uniform((N,), seed=90).cuda()
+        y = lin.forward(x, w, bias)
+        dx, dw, db = lin.backward(g)
+        xq, _ = ops.quantize(x, ops.E4M3, ops.ROW, rx)
+        wq, _ = ops.quantize(w, ops.E4M3, ops.ROW, rw)
+        y2 = ops.mm(xq, wq, rx.scale_inv, rw.scale_inv, bias)
+        gq, _ = ops.quantize(g, ops.E5M2, ops.ROW, rg)
+        dx2 = ops.mm(gq, wq, rg.scale_inv, rw.scale_inv, fmt_a=ops.E5M2, b_mn_major=True)
+        dw2 = ops.mm(gq, xq, rg.scale_inv, rx.scale_inv, fmt_a=ops.E5M2, a_mn_major=True, b_mn_major=True)
+        db2 = ops.bias_grad(g)
+        torch.cuda.synchronize()
+        for a, b in ((y, y2), (dx, dx2), (dw, dw2), (db, db2)):
+            assert torch.equal(a, b)
+        for r1, r2 in ((lin.rx, rx), (lin.rw, rw), (lin.rg, rg)):
+            assert torch.equal(r1.buf, r2.buf)
+    ref, Ssum = OG.mm_fp8(xq.cpu().numpy(), wq.cpu().numpy(), 0, 0, rx.scale_inv.item(), rw.scale_inv.item(),
+                          bias.cpu().numpy())
+    assert OG.check(y.float().cpu().numpy(), ref, Ssum)[0]
+    ref, Ssum = OG.mm_fp8(gq.cpu().numpy(), wq.cpu().numpy().T.copy(), 1, 0, rg.scale_inv.item(), rw.scale_inv.item())
+    assert OG.check(dx.float().cpu().numpy(), ref, Ssum)[0]
+    ref, Ssum = OG.mm_fp8(gq.cpu().numpy().T.copy(), xq.cpu().numpy().T.copy(), 1, 0, rg.scale_inv.item(),
+                          rx.scale_inv.item())
+    assert OG.check(dw.float().cpu().numpy(), ref, Ssum)[0]
+    assert np.all(np.abs(db.cpu().numpy().astype(np.float64) - OB.bias_grad(g.cpu())) <= OB.bound(g.cpu()))

@@ -56,6 +56,7 @@ def parse():
     ap.add_argument("--profile", action="store_true",
                     help="warm up, run exactly one step inside the NVTX range fp8_profile_step, exit (for ncu)")
     ap.add_argument("--shapes", default=None, help="sweep subset, e.g. 8192x8192x8192,64x8192x2048")
+    ap.add_argument("--ws", action="store_true", help="gemm sweep: also time each shape with a stream-K workspace")
     ap.add_argument("--qdtypes", default="bf16,fp32", help="quantize sweep input dtypes")
     ap.add_argument("--qlayouts", default="row,T,dual", help="quantize sweep layouts")
     return ap.parse_args()
@@ -157,6 +158,7 @@ class Linear:
         self.dx = torch.empty((M, HIDDEN), dtype=bf, device=dev)
         self.dw = torch.empty((n_out, HIDDEN), dtype=bf, device=dev)
         self.inputs = [(x.to(dev), g.to(dev)) for x, g in inputs]
+        self.ws = None  # stream-K workspace shared by the step's GEMMs (set by build_workload)
 
     def quantize(self, ops, x, g, ev=None):
         ops.quantize(x, ops.E4M3, ops.DUAL, self.rx, self.xq, self.xq_t)
@@ -164,9 +166,11 @@ class Linear:
         ops.quantize(g, ops.E5M2, ops.DUAL, self.rg, self.gq, self.gq_t)
 
     def gemms(self, ops):
-        ops.mm(self.xq, self.wq, self.rx.scale_inv, self.rw.scale_inv, self.bias, out=self.y)
-        ops.mm(self.gq, self.wq_t, self.rg.scale_inv, self.rw.scale_inv, None, fmt_a=ops.E5M2, out=self.dx)
-        ops.mm(self.gq_t, self.xq_t, self.rg.scale_inv, self.rx.scale_inv, None, fmt_a=ops.E5M2, out=self.dw)
+        ops.mm(self.xq, self.wq, self.rx.scale_inv, self.rw.scale_inv, self.bias, out=self.y, workspace=self.ws)
+        ops.mm(self.gq, self.wq_t, self.rg.scale_inv, self.rw.scale_inv, None, fmt_a=ops.E5M2, out=self.dx,
+               workspace=self.ws)
+        ops.mm(self.gq_t, self.xq_t, self.rg.scale_inv, self.rx.scale_inv, None, fmt_a=ops.E5M2, out=self.dw,
+               workspace=self.ws)
 
     # The same step with the layout tag: row-layout quantizes only, and the
     # backward GEMMs read W, G and X as quantized through MN-major operands.
@@ -176,11 +180,11 @@ class Linear:
         ops.quantize(g, ops.E5M2, ops.ROW, self.rg, self.gq)
 
     def gemms_mn(self, ops):
-        ops.mm(self.xq, self.wq, self.rx.scale_inv, self.rw.scale_inv, self.bias, out=self.y)
+        ops.mm(self.xq, self.wq, self.rx.scale_inv, self.rw.scale_inv, self.bias, out=self.y, workspace=self.ws)
         ops.mm(self.gq, self.wq, self.rg.scale_inv, self.rw.scale_inv, None, fmt_a=ops.E5M2, out=self.dx,
-               b_mn_major=True)
+               b_mn_major=True, workspace=self.ws)
         ops.mm(self.gq, self.xq, self.rg.scale_inv, self.rx.scale_inv, None, fmt_a=ops.E5M2, out=self.dw,
-               a_mn_major=True, b_mn_major=True)
+               a_mn_major=True, b_mn_major=True, workspace=self.ws)
 
 
 def build_workload(M, torch, ops, S, n_sets=2):
@@ -189,6 +193,16 @@ def build_workload(M, torch, ops, S, n_sets=2):
     for n_out, w, b in ((HIDDEN, w1, b1), (FFN, w2, b2)):
         sets = [S.linear_1p2b_step(M, n_out, s) for s in range(n_sets)]
         lins.append(Linear(M, n_out, w, b, sets, torch, ops))
+    # One stream-K workspace, zeroed once, for every GEMM of the step (they run
+    # one after another on one stream); sized for the largest request.
+    need = 0
+    for n in (HIDDEN, FFN):
+        for (m, nn, k) in ((M, n, HIDDEN), (M, HIDDEN, n), (n, HIDDEN, M)):
+            for amn, bmn in ((False, False), (False, True), (True, True)):
+                need = max(need, ops.mm_workspace_bytes(m, nn, k, a_mn_major=amn, b_mn_major=bmn))
+    ws = torch.zeros(max(need, 256), dtype=torch.uint8, device="cuda")
+    for L in lins:
+        L.ws = ws
     return lins
 
 
@@ -321,26 +335,38 @@ def sweep(args):
     B.build()
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     flush = torch.zeros(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
-    want = None
-    if args.shapes:
-        want = [tuple(int(v) for v in s.split("x")) for s in args.shapes.split(",")]
     if args.sweep == "gemm":
-        shapes = GEMM_SHAPES if not want else [w if len(w) == 4 else (1,) + w for w in want]
-        for bt, M, N, K in shapes:
-            a = S.fp8_codes((bt, M, K), seed=1).cuda()
-            b = S.fp8_codes((1, N, K), seed=2).cuda() if bt == 8 else S.fp8_codes((bt, N, K), seed=2).cuda()
+        # A shape is [B x]M x N x K, optionally followed by ":bmn" (B read
+        # MN-major) or ":mn" (A and B read MN-major), the backward layouts.
+        shapes = []
+        for spec in (args.shapes.split(",") if args.shapes else
+                     ["x".join(map(str, s)) for s in GEMM_SHAPES]):
+            dims, _, lay = spec.partition(":")
+            v = tuple(int(t) for t in dims.split("x"))
+            shapes.append(((1,) + v if len(v) == 3 else v, lay or "nt"))
+        for (bt, M, N, K), lay in shapes:
+            a_mn, b_mn = lay == "mn", lay in ("mn", "bmn")
+            a = S.fp8_codes((bt, K, M) if a_mn else (bt, M, K), seed=1).cuda()
+            nb = 1 if bt == 8 else bt
+            b = S.fp8_codes((nb, K, N) if b_mn else (nb, N, K), seed=2).cuda()
             one = torch.ones(1, device="cuda")
             bias = S.uniform((N,), seed=3).cuda()
             out = torch.empty((bt, M, N), dtype=torch.bfloat16, device="cuda")
-            for with_bias in (False, True):
-                fn = lambda: ops.mm(a, b, one, one, bias if with_bias else None, out=out)  # noqa: E731
-                for _ in range(3):
-                    fn()
-                ms = _kernel_ms(fn, torch, args.iters)
-                fl = 2.0 * bt * M * N * K
-                print(json.dumps({"kernel": "mm_fp8", "batch": bt, "M": M, "N": N, "K": K, "bias": with_bias,
-                                  "us": round(ms * 1e3, 2), "tflops": round(fl / ms / 1e9, 1)}))
+            need = ops.mm_workspace_bytes(M, N, K, batch=bt, a_mn_major=a_mn, b_mn_major=b_mn)
+            ws = torch.zeros(max(need, 256), dtype=torch.uint8, device="cuda") if args.ws else None
+            for use_ws in ((False, True) if args.ws and need > 0 else (False,)):
+                for with_bias in (False, True):
+                    fn = lambda: ops.mm(a, b, one, one, bias if with_bias else None, out=out,  # noqa: E731
+                                        a_mn_major=a_mn, b_mn_major=b_mn, workspace=ws if use_ws else None)
+                    for _ in range(3):
+                        fn()
+                    ms = _kernel_ms(fn, torch, args.iters)
+                    fl = 2.0 * bt * M * N * K
+                    print(json.dumps({"kernel": "mm_fp8", "batch": bt, "M": M, "N": N, "K": K, "layout": lay,
+                                      "bias": with_bias, "stream_k_ws": need if use_ws else 0,
+                                      "us": round(ms * 1e3, 2), "tflops": round(fl / ms / 1e9, 1)}))
     else:
+        want = [tuple(int(v) for v in s.split("x")) for s in args.shapes.split(",")] if args.shapes else None
         for rows, cols in (QUANT_SHAPES if not want else want):
             for dt in args.qdtypes.split(","):
                 x = S.quant_sweep_input(rows, cols, dt, 1.0).cuda()
@@ -540,6 +566,7 @@ def main():
             "data": "synthetic",
             "config": {"workload": f"1.2B-model linears fwd+bwd (hidden 1536, FFN 4096), M={M} tokens, "
                                    "X/W/G dual quantize + fwd/dX/dW mm_fp8 for both linear shapes",
+                       "stream_k_workspace_bytes": int(lins[0].ws.numel()),
                        "M": M, "linears": [[HIDDEN, HIDDEN], [FFN, HIDDEN]],
                        "l2": "no flush: 2 rotating input sets, ~320 MB per set pair > 126 MB L2",
                        "parallelism": f"replicas x{world}"},

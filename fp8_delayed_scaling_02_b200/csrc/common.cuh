@@ -27,6 +27,7 @@ enum WaitSite : uint32_t {
   kWaitEpilogueTmemFull = 4,
   kWaitDrain = 5,
   kWaitQuantizeTma = 6,
+  kWaitSplitK = 7,
 };
 
 // Library-global device error word (defined in capi.cu, relocatable device code

@@ -71,6 +71,19 @@ struct MmParams {
   int m_tiles, n_tiles, k_blocks, tiles_per_batch, tiles_total, group_m;
   int a_bcast, b_bcast;
   int a_mn, b_mn;    // operand stored MN-major ([K][M] / [K][N], M or N contiguous)
+  // Work split (data-parallel + stream-K).  Tiles [0, dp_tiles) are whole
+  // tiles, dealt round-robin to the grid's CTAs (pairs).  The k-block
+  // iterations of the remaining tiles, numbered g = (t - dp_tiles) * k_blocks
+  // + kb, form one range [0, sk_iters) cut into sk_ctas contiguous pieces;
+  // piece s = [s*sk_iters/sk_ctas, (s+1)*sk_iters/sk_ctas) runs on CTA s
+  // after its whole tiles.  A piece that starts inside a tile writes its
+  // float32 partial to slot s of `ws` and counts up flags[s]; the CTA holding
+  // the tile's k-block 0 waits for those flags, adds the partials of the
+  // following pieces in piece order and stores the tile.
+  int dp_tiles, sk_ctas;
+  int64_t sk_iters;
+  float* ws;
+  uint32_t* flags;
   int64_t c_stride;  // elements between output batches
   const float* sinv_a;
   const float* sinv_b;
@@ -310,6 +323,45 @@ __device__ __forceinline__ uint64_t sdesc_mn128(uint32_t saddr, uint32_t lbo) {
   return d;
 }
 
+// First k-block iteration of stream-K piece s (s may equal sk_ctas: the end).
+__device__ __forceinline__ int64_t sk_begin(const MmParams& p, int s) {
+  return int64_t(s) * p.sk_iters / p.sk_ctas;
+}
+
+// The piece that holds stream-K iteration g: the largest s with sk_begin(s) <= g.
+__device__ __forceinline__ int sk_owner(const MmParams& p, int64_t g) {
+  return int(((g + 1) * p.sk_ctas + p.sk_iters - 1) / p.sk_iters) - 1;
+}
+
+// Unit i of CTA (pair) s in a grid of P: tile t and k-blocks [kb0, kb1).
+// A CTA runs its stream-K piece first, then its whole tiles, so that a
+// tile's finisher (which holds the tile's first k-blocks at the end of its
+// piece) waits for partials that the next pieces wrote at their start, and
+// its partial reads overlap the mainloop of its next whole tile.
+// False past the CTA's last unit.
+__device__ __forceinline__ bool unit_at(const MmParams& p, int s, int P, int i, int& t, int& kb0, int& kb1) {
+  int n_sk = 0;
+  if (s < p.sk_ctas) {
+    const int64_t g0 = sk_begin(p, s), g1 = sk_begin(p, s + 1);
+    if (g0 < g1) {
+      const int64_t first = g0 / p.k_blocks;
+      n_sk = int((g1 - 1) / p.k_blocks - first + 1);
+      if (i < n_sk) {
+        const int64_t tb = (first + i) * p.k_blocks;
+        kb0 = g0 > tb ? int(g0 - tb) : 0;
+        kb1 = g1 - tb < p.k_blocks ? int(g1 - tb) : p.k_blocks;
+        t = p.dp_tiles + int(first + i);
+        return true;
+      }
+    }
+  }
+  t = s + (i - n_sk) * P;
+  if (t >= p.dp_tiles) return false;
+  kb0 = 0;
+  kb1 = p.k_blocks;
+  return true;
+}
+
 __device__ __forceinline__ void decode_tile(const MmParams& p, int t, int& b, int& mt, int& nt) {
   b = t / p.tiles_per_batch;
   const int r = t - b * p.tiles_per_batch;
@@ -349,8 +401,8 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
   pdl_launch_dependents();
   const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
-  const int unit0 = int(blockIdx.x) / PAIR;   // this CTA's (pair's) first tile
-  const int units = int(gridDim.x) / PAIR;    // tiles advance by the number of CTAs (pairs)
+  const int cta = int(blockIdx.x) / PAIR;  // this CTA's (pair's) index: its whole tiles and stream-K piece
+  const int ctas = int(gridDim.x) / PAIR;  // whole tiles advance by the number of CTAs (pairs)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -386,14 +438,16 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;  // bit s: stage s armed; its parity
       bool ok = true;
-      for (int t = unit0; ok && t < p.tiles_total; t += units) {
+      for (int i = 0; ok; ++i) {
+        int t, kb0, kb1;
+        if (!unit_at(p, cta, ctas, i, t, kb0, kb1)) break;
         int b, mt, nt;
         decode_tile(p, t, b, mt, nt);
         const int ba = p.a_bcast ? 0 : b;
         const int bb = p.b_bcast ? 0 : b;
         const int arow = mt * kTileM + int(rank) * kBM;
         const int brow = nt * BN + int(rank) * C::kBRows;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort, p.err, kWaitProducerEmpty)) {
             ok = false;
             break;
@@ -451,13 +505,15 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
       bool ok = true;
       const uint32_t sa0 = sbase;
       const uint32_t sb0 = sbase + C::kStages * C::kABytes;
-      for (int t = unit0; ok && t < p.tiles_total; t += units, ++i) {
+      for (; ok; ++i) {
+        int t, kb0, kb1;
+        if (!unit_at(p, cta, ctas, i, t, kb0, kb1)) break;
         const int acc = i & 1;
         const uint32_t acc_par = (i >> 1) & 1;
         if (!mbar_wait(tempty_bar(acc), acc_par ^ 1u, abort, p.err, kWaitMmaTmemEmpty)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(acc * BN);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(full_bar(stage), phase, abort, p.err, kWaitMmaFull)) {
             ok = false;
             break;
@@ -474,9 +530,9 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
 #pragma unroll
           for (int k = 0; k < kBK / kUmmaK; ++k) {
             if constexpr (PAIR == 1)
-              umma_f8(d, ad + astep * k, bd + bstep * k, p.idesc, (kb | k) != 0 ? 1u : 0u);
+              umma_f8(d, ad + astep * k, bd + bstep * k, p.idesc, (kb != kb0 || k != 0) ? 1u : 0u);
             else
-              umma_f8_pair(d, ad + astep * k, bd + bstep * k, p.idesc, (kb | k) != 0 ? 1u : 0u);
+              umma_f8_pair(d, ad + astep * k, bd + bstep * k, p.idesc, (kb != kb0 || k != 0) ? 1u : 0u);
           }
           if constexpr (PAIR == 1) umma_commit(empty_bar(stage));
           else umma_commit_pair(empty_bar(stage));
@@ -514,40 +570,79 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
     const uint32_t stage0 = sbase + C::kStagingOffset + uint32_t(ew) * 2u * kStagingBytes;
     int buf = 0;
     int i = 0;
-    for (int t = unit0; t < p.tiles_total; t += units, ++i) {
+    constexpr int kChunks = kHalfCols / 32;
+    constexpr uint32_t kPieceWarps = uint32_t(kEpiWarps * PAIR);  // arrivals of one piece's partial
+    for (;; ++i) {
+      int t, kb0, kb1;
+      if (!unit_at(p, cta, ctas, i, t, kb0, kb1)) break;
+      // A piece that starts inside the tile hands its partial on; the piece
+      // with k-block 0 of a tile it does not finish adds the later pieces'
+      // partials, pieces cta+1 .. last_piece.
+      const bool writer = kb0 > 0;
+      const bool finisher = kb0 == 0 && kb1 < p.k_blocks;
+      const int last_piece =
+          finisher ? sk_owner(p, int64_t(t - p.dp_tiles) * p.k_blocks + p.k_blocks - 1) : cta;
       const int acc = i & 1;
       const uint32_t acc_par = (i >> 1) & 1;
       if (!mbar_wait(tfull_bar(acc), acc_par, abort, p.err, kWaitEpilogueTmemFull)) break;
       tc_fence_after();
       int b, mt, nt;
       decode_tile(p, t, b, mt, nt);
+      // Chunk cc of this warp's part of piece q's float32 partial: 32 rows x
+      // 32 columns as [j][lane] float4, so each store or load instruction of
+      // the warp covers 512 contiguous bytes.
+      auto slot = [&](int q, int cc) {
+        return reinterpret_cast<float4*>(p.ws + (size_t(q) * PAIR + rank) * size_t(kBM * BN) +
+                                         size_t(ew * kChunks + cc) * 1024) + lane;
+      };
+      if (finisher && lane == 0) {
+        // Wait (bounded) until every warp of every later piece of this tile has published its partial.
+        const unsigned long long w0 = globaltimer_ns();
+        for (int q = cta + 1; q <= last_piece; ++q) {
+          uint32_t seen = 0;
+          while (true) {
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(p.flags + q) : "memory");
+            if (seen >= kPieceWarps) break;
+            if (*abort || globaltimer_ns() - w0 > kWaitBudgetNs) {
+              record_device_error(p.err, kWaitSplitK);
+              *abort = 1;
+              break;
+            }
+          }
+        }
+      }
+      if (finisher) {
+        __syncwarp();
+        __threadfence();
+      }
       const int m0 = mt * kTileM + int(rank) * kBM + quad * 32;
       const uint32_t tbase = tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + half * kHalfCols);
       const int nbase = nt * BN + half * kHalfCols;
       const uint32_t release_bar = PAIR == 1 ? tempty_bar(acc) : mapa_shared(tempty_bar(acc), 0);
       bool released = false;
-#pragma unroll 1
-      for (int c = 0; c < kHalfCols / 32; c += 2) {
-        if (nbase + c * 32 >= p.N) break;  // warp-uniform: the rest of this half is beyond N
-        uint32_t r[2][32];
-        tmem_ld32_nowait(tbase + uint32_t(c * 32), r[0]);
-        if (nbase + (c + 1) * 32 < p.N) tmem_ld32_nowait(tbase + uint32_t((c + 1) * 32), r[1]);
-        tmem_wait_ld();
-        if (c + 2 >= kHalfCols / 32 || nbase + (c + 2) * 32 >= p.N) {
-          // Last TMEM read of this tile for this warp: hand the accumulator back.
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(release_bar);
-          released = true;
-        }
+      auto release = [&]() {
+        // Last TMEM read of this tile for this warp: hand the accumulator back.
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(release_bar);
+        released = true;
+      };
+      // One 32 x 32 chunk at output columns n0 (this lane's row): scale, bias,
+      // one bf16 rounding, store.
+      auto emit = [&](int n0, const uint32_t(&v)[32]) {
+        if (m0 >= p.M) return;  // warp-uniform: rows beyond M (pair peer of a short last tile)
+        const bool full = n0 + 32 <= p.N;
+        const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
+        if (p.tma_store && lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
+        __syncwarp();
+        // 16-byte unit u of this lane's 64-byte row holds columns 8u .. 8u+7,
+        // at unit position u ^ ((lane >> 1) & 3).
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int n0 = nbase + (c + h) * 32;
-          if (n0 >= p.N) break;  // warp-uniform
-          uint32_t packed[16];
-          const bool full = n0 + 32 <= p.N;
+        for (int u = 0; u < 4; ++u) {
+          uint32_t packed[4];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
+          for (int jj = 0; jj < 2; ++jj) {
+            const int j = 2 * u + jj;
             float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
             if (p.bias != nullptr) {
               if (full && p.bias_vec) {
@@ -560,60 +655,98 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
                 bv.w = nn + 3 < p.N ? __ldg(p.bias + nn + 3) : 0.f;
               }
             }
-            const float y0 = fmaf(__uint_as_float(r[h][4 * j + 0]), sab, bv.x);
-            const float y1 = fmaf(__uint_as_float(r[h][4 * j + 1]), sab, bv.y);
-            const float y2 = fmaf(__uint_as_float(r[h][4 * j + 2]), sab, bv.z);
-            const float y3 = fmaf(__uint_as_float(r[h][4 * j + 3]), sab, bv.w);
+            const float y0 = fmaf(__uint_as_float(v[4 * j + 0]), sab, bv.x);
+            const float y1 = fmaf(__uint_as_float(v[4 * j + 1]), sab, bv.y);
+            const float y2 = fmaf(__uint_as_float(v[4 * j + 2]), sab, bv.z);
+            const float y3 = fmaf(__uint_as_float(v[4 * j + 3]), sab, bv.w);
             const __nv_bfloat162 h01 = __floats2bfloat162_rn(y0, y1);
             const __nv_bfloat162 h23 = __floats2bfloat162_rn(y2, y3);
-            packed[2 * j] = *reinterpret_cast<const uint32_t*>(&h01);
-            packed[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+            packed[2 * jj] = *reinterpret_cast<const uint32_t*>(&h01);
+            packed[2 * jj + 1] = *reinterpret_cast<const uint32_t*>(&h23);
           }
-          if (p.tma_store) {
-            if (m0 < p.M) {
-              const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
-              if (lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
-              __syncwarp();
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const uint32_t addr = sbuf + uint32_t(lane) * 64u + uint32_t((u ^ ((lane >> 1) & 3)) * 16);
-                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[4 * u]),
-                             "r"(packed[4 * u + 1]), "r"(packed[4 * u + 2]), "r"(packed[4 * u + 3])
-                             : "memory");
-              }
-              fence_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_3d(&tmC, sbuf, n0, m0, b);
-                bulk_commit();
-              }
-              buf ^= 1;
-            }
-          } else if (m0 < p.M) {
-            // Rows not 16-byte aligned: stage the 32x32 chunk in the same
-            // swizzled layout, then write it row by row, lane l taking column
-            // n0 + l, so each store instruction covers 64 contiguous bytes.
-            const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
-            __syncwarp();
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-              const uint32_t addr = sbuf + uint32_t(lane) * 64u + uint32_t((u ^ ((lane >> 1) & 3)) * 16);
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[4 * u]),
-                           "r"(packed[4 * u + 1]), "r"(packed[4 * u + 2]), "r"(packed[4 * u + 3])
-                           : "memory");
-            }
-            __syncwarp();
-            const bool col_ok = n0 + lane < p.N;
-            uint16_t* obase = p.out + int64_t(b) * p.c_stride + int64_t(m0) * p.N + n0 + lane;
+          const uint32_t addr = sbuf + uint32_t(lane) * 64u + uint32_t((u ^ ((lane >> 1) & 3)) * 16);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[0]), "r"(packed[1]),
+                       "r"(packed[2]), "r"(packed[3])
+                       : "memory");
+        }
+        if (p.tma_store) {
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_3d(&tmC, sbuf, n0, m0, b);
+            bulk_commit();
+          }
+        } else {
+          // Rows not 16-byte aligned: the chunk staged in the same swizzled
+          // layout is written row by row, lane l taking column n0 + l, so
+          // each store instruction covers 64 contiguous bytes.
+          __syncwarp();
+          const bool col_ok = n0 + lane < p.N;
+          uint16_t* obase = p.out + int64_t(b) * p.c_stride + int64_t(m0) * p.N + n0 + lane;
 #pragma unroll 4
-            for (int rr = 0; rr < 32; ++rr) {
-              const uint32_t addr = sbuf + uint32_t(rr) * 64u + uint32_t((((lane >> 3) ^ ((rr >> 1) & 3)) << 4)) +
-                                    uint32_t((lane & 7) << 1);
-              uint16_t v;
-              asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
-              if (col_ok && m0 + rr < p.M) obase[int64_t(rr) * p.N] = v;
+          for (int rr = 0; rr < 32; ++rr) {
+            const uint32_t addr = sbuf + uint32_t(rr) * 64u + uint32_t((((lane >> 3) ^ ((rr >> 1) & 3)) << 4)) +
+                                  uint32_t((lane & 7) << 1);
+            uint16_t v16;
+            asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v16) : "r"(addr) : "memory");
+            if (col_ok && m0 + rr < p.M) obase[int64_t(rr) * p.N] = v16;
+          }
+        }
+        buf ^= 1;
+      };
+      auto add4 = [](uint32_t* v, const float4& w) {
+        v[0] = __float_as_uint(__uint_as_float(v[0]) + w.x);
+        v[1] = __float_as_uint(__uint_as_float(v[1]) + w.y);
+        v[2] = __float_as_uint(__uint_as_float(v[2]) + w.z);
+        v[3] = __float_as_uint(__uint_as_float(v[3]) + w.w);
+      };
+#pragma unroll 1
+      for (int c = 0; c < kChunks; c += 2) {
+        if (nbase + c * 32 >= p.N) break;  // warp-uniform: the rest of this half is beyond N
+        const bool two = nbase + (c + 1) * 32 < p.N;
+        const bool last_pair = c + 2 >= kChunks || nbase + (c + 2) * 32 >= p.N;
+        if (finisher) {
+          // Per chunk: the next piece's partial is requested (8 independent
+          // 512-byte warp loads) before the TMEM read; any further pieces are
+          // added after it, in piece order.
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            if (h == 1 && !two) break;
+            float4 pv[8];
+            const float4* src = slot(cta + 1, c + h);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) pv[j] = __ldcg(src + 32 * j);
+            uint32_t r[32];
+            tmem_ld32_nowait(tbase + uint32_t((c + h) * 32), r);
+            tmem_wait_ld();
+            if (last_pair && (h == 1 || !two)) release();
+#pragma unroll
+            for (int j = 0; j < 8; ++j) add4(r + 4 * j, pv[j]);
+            for (int q = cta + 2; q <= last_piece; ++q) {
+              const float4* src2 = slot(q, c + h);
+#pragma unroll
+              for (int j = 0; j < 8; ++j) add4(r + 4 * j, __ldcg(src2 + 32 * j));
             }
-            buf ^= 1;
+            emit(nbase + (c + h) * 32, r);
+          }
+          continue;
+        }
+        uint32_t r[2][32];
+        tmem_ld32_nowait(tbase + uint32_t(c * 32), r[0]);
+        if (two) tmem_ld32_nowait(tbase + uint32_t((c + 1) * 32), r[1]);
+        tmem_wait_ld();
+        if (last_pair) release();
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (h == 1 && !two) break;
+          if (writer) {
+            float4* dst = slot(cta, c + h);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              __stcg(dst + 32 * j, make_float4(__uint_as_float(r[h][4 * j]), __uint_as_float(r[h][4 * j + 1]),
+                                               __uint_as_float(r[h][4 * j + 2]), __uint_as_float(r[h][4 * j + 3])));
+          } else {
+            emit(nbase + (c + h) * 32, r[h]);
           }
         }
       }
@@ -621,6 +754,21 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(release_bar);
+      }
+      if (writer) {
+        __threadfence();  // this warp's partial stores are visible before its arrival
+        __syncwarp();
+        if (lane == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(p.flags + cta) : "memory");
+      } else if (finisher) {
+        __syncwarp();
+        if (lane == 0) {
+          // Each finishing warp counts itself on every piece it read; the last
+          // of a piece's writer and reader warps clears its flag for the next call.
+          for (int q = cta + 1; q <= last_piece; ++q) {
+            const uint32_t old = atomicAdd(p.flags + q, 1u);
+            if (old == 2u * kPieceWarps - 1u) atomicExch(p.flags + q, 0u);
+          }
+        }
       }
     }
     if (p.tma_store && lane == 0) bulk_wait_all();
@@ -736,9 +884,25 @@ int max_pairs(int sms) {
   return cached[dev];
 }
 
+// Launch shape: tile width, CTA pairing, grid size in CTAs (pairs), whole
+// tiles, stream-K pieces and the workspace the pieces need.
+struct MmChoice {
+  int bn, pair, grid, dp_tiles, sk_ctas;
+  size_t ws_bytes;
+};
+
+constexpr int kMaxPieces = 256;             // flag words in the workspace's first 1024 bytes
+constexpr size_t kFlagBytes = 4 * kMaxPieces;
+
+// Workspace of a stream-K launch: 1024 bytes of per-piece arrival counters,
+// then one float32 128 x BN partial per piece and CTA of a pair.
+size_t sk_ws_bytes(int pieces, int bn, int pair) {
+  return pieces > 0 ? kFlagBytes + size_t(pieces) * size_t(pair) * kBM * size_t(bn) * 4 : 0;
+}
+
 template <int BN, int PAIR>
 int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
-              const int64_t* strides, MmParams p, int slots, cudaStream_t st) {
+              const int64_t* strides, MmParams p, const MmChoice& c, void* ws, cudaStream_t st) {
   CUtensorMap ta, tb, tc;
   const int64_t ba = (batch > 1 && strides[0] != 0) ? batch : 1;
   const int64_t bb = (batch > 1 && strides[1] != 0) ? batch : 1;
@@ -755,43 +919,79 @@ int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t 
   p.n_tiles = int((N + BN - 1) / BN);
   p.tiles_per_batch = p.m_tiles * p.n_tiles;
   p.tiles_total = int(p.tiles_per_batch * batch);
+  p.dp_tiles = c.dp_tiles;
+  p.sk_ctas = c.sk_ctas;
+  p.sk_iters = int64_t(p.tiles_total - c.dp_tiles) * p.k_blocks;
+  if (c.sk_ctas > 0) {
+    p.flags = static_cast<uint32_t*>(ws);
+    p.ws = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + kFlagBytes);
+  }
   p.group_m = 8;
   p.idesc |= (uint32_t(BN >> 3) << 17) | (uint32_t((kBM * PAIR) >> 4) << 24);
   if (!ensure_smem_attr<BN, PAIR>()) return FP8_ERR_CUDA;
-  const int units = std::max(1, std::min(p.tiles_total, slots));
-  const cudaError_t e = launch_pdl(mm_fp8_kernel<BN, PAIR>, dim3(PAIR * units), dim3(kThreadsMM),
+  const cudaError_t e = launch_pdl(mm_fp8_kernel<BN, PAIR>, dim3(PAIR * std::max(1, c.grid)), dim3(kThreadsMM),
                                    Cfg<BN, PAIR>::kSmemBytes, st, PAIR, ta, tb, tc, p);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-// Tile-shape choice: time ~ waves x per-SM tile width / relative efficiency,
-// over {one CTA, CTA pair} x {BN 256, 128}.  A pair halves each SM's share of
-// the B operand in shared memory and the L2 traffic per flop.
-struct MmChoice {
-  int bn, pair, slots;
-};
-
-MmChoice choose_mm(int64_t M, int64_t N, int64_t batch, int sms, bool b_mn) {
+// Launch-shape choice by a time model in microseconds, over {one CTA, CTA
+// pair} x {BN 256, 128} and, given a workspace, a stream-K tail:
+//   * one k-block of a 128 x 256 tile takes about 0.45 us on one SM (pairs
+//     and single CTAs alike; relative efficiencies below);
+//   * whole tiles run in waves of `slots`;
+//   * stream-K (data-parallel + two-tile stream-K): all but the last full
+//     wave stay whole tiles; the k-blocks of the rest are dealt evenly to the
+//     pieces.  A piece costs its k-blocks plus the fix-up measured on B200
+//     for a 128 x 256 float32 partial: about 4 us to write it, fence and
+//     flag it, and about 5 us per extra piece for the finisher's wait and
+//     read (half that for BN = 128).  So stream-K pays off only where a part
+//     of a wave idles for well over 10 us: small outputs with long K.
+MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool b_mn, size_t ws_limit) {
   struct Opt {
     int bn, pair;
     double eff;
   };
-  // Relative per-SM MMA efficiency measured on B200: a 128-wide MMA issues at
-  // about the rate of a 256-wide one, so BN = 128 does half the work per
-  // instruction whether or not the CTAs are paired.
+  // A 128-wide MMA issues at about the rate of a 256-wide one, so BN = 128
+  // does half the work per instruction whether or not the CTAs are paired.
   const Opt opts[4] = {{256, 2, 1.0}, {256, 1, 0.85}, {128, 2, 0.5}, {128, 1, 0.45}};
-  MmChoice best{256, 1, sms};
+  constexpr int kMinIters = 4;  // k-blocks per piece, at least
+  const int64_t kb = (K + kBK - 1) / kBK;
+  MmChoice best{256, 1, 1, 0, 0, 0};
   double best_cost = 1e300;
   for (const Opt& o : opts) {
     if (o.pair == 2 && M <= kBM) continue;  // the second CTA would hold no rows
     if (b_mn && o.bn / o.pair < 128) continue;
     const int slots = o.pair == 2 ? (o.bn == 256 ? max_pairs<256>(sms) : max_pairs<128>(sms)) : sms;
-    const int64_t units = ((M + kBM * o.pair - 1) / (kBM * o.pair)) * ((N + o.bn - 1) / o.bn) * batch;
-    const double waves = double((units + slots - 1) / slots);
-    const double cost = waves * o.bn / o.eff;
-    if (cost < best_cost) {
-      best_cost = cost;
-      best = MmChoice{o.bn, o.pair, slots};
+    const int64_t tiles = ((M + kBM * o.pair - 1) / (kBM * o.pair)) * ((N + o.bn - 1) / o.bn) * batch;
+    const double t_kb = 0.45 * (o.bn / 256.0) / o.eff;
+    const double t_write = 4.0 * (o.bn / 256.0), t_read = 5.0 * (o.bn / 256.0);
+    const double dp_cost = double((tiles + slots - 1) / slots) * double(kb) * t_kb;
+    if (dp_cost < best_cost) {
+      best_cost = dp_cost;
+      best = MmChoice{o.bn, o.pair, int(std::min<int64_t>(tiles, slots)), int(tiles), 0, 0};
+    }
+    if (ws_limit == 0 || tiles % slots == 0 || slots > kMaxPieces || kb < 2 * kMinIters) continue;
+    const int64_t full = tiles / slots;
+    const int64_t dp = full >= 1 ? (full - 1) * slots : 0;
+    const int64_t T = tiles - dp;
+    const int64_t W = T * kb;
+    int64_t cands[6] = {slots, 2 * T, 3 * T, 4 * T, 5 * T, 6 * T};
+    for (int64_t pieces : cands) {
+      pieces = std::min<int64_t>(pieces, slots);
+      pieces = std::min<int64_t>(pieces, W / kMinIters);
+      if (pieces < 2) continue;
+      const int64_t L = W / pieces;
+      if (W % pieces == 0 && L % kb == 0) continue;  // every piece whole tiles: the data-parallel case
+      const int64_t iters = (W + pieces - 1) / pieces;
+      const int64_t span = std::min<int64_t>(pieces, (kb - 1 + L - 1) / L + 1);  // pieces a tile can touch
+      const double cost = double(dp / slots) * double(kb) * t_kb + double(iters) * t_kb + t_write +
+                          double(span - 1) * t_read;
+      const size_t wsb = sk_ws_bytes(int(pieces), o.bn, o.pair);
+      if (wsb > ws_limit) continue;
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = MmChoice{o.bn, o.pair, int(dp > 0 ? slots : pieces), int(dp), int(pieces), wsb};
+      }
     }
   }
   return best;
@@ -802,9 +1002,9 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t batch, int sms, bool b_mn) {
 
 using namespace fp8ds;
 
-extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
-                      const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b,
-                      const float* bias, uint16_t* out_bf16, fp8_stream_t stream) {
+static int mm_impl(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+                   const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
+                   uint16_t* out_bf16, void* workspace, size_t ws_bytes, fp8_stream_t stream) {
   if (M < 0 || N < 0 || K < 0 || batch < 1) return FP8_ERR_INVALID_ARG;
   if ((layout & ~(FP8_MM_A_E5M2 | FP8_MM_B_E5M2 | FP8_MM_A_MN_MAJOR | FP8_MM_B_MN_MAJOR)) != FP8_MM_NT)
     return FP8_ERR_INVALID_ARG;
@@ -860,11 +1060,34 @@ extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, 
 
   // An MN-major B is loaded as boxes of 128 N-rows, so its per-CTA tile must
   // hold whole boxes (no 128-wide CTA pair).
-  const MmChoice c = choose_mm(M, N, batch, sms, b_mn);
+  if (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP8_ERR_UNSUPPORTED;
+  const MmChoice c = choose_mm(M, N, K, batch, sms, b_mn, workspace ? ws_bytes : 0);
   if (c.pair == 2) {
-    if (c.bn == 256) return launch_mm<256, 2>(A, B, M, N, K, batch, strides, p, c.slots, st);
-    return launch_mm<128, 2>(A, B, M, N, K, batch, strides, p, c.slots, st);
+    if (c.bn == 256) return launch_mm<256, 2>(A, B, M, N, K, batch, strides, p, c, workspace, st);
+    return launch_mm<128, 2>(A, B, M, N, K, batch, strides, p, c, workspace, st);
   }
-  if (c.bn == 256) return launch_mm<256, 1>(A, B, M, N, K, batch, strides, p, c.slots, st);
-  return launch_mm<128, 1>(A, B, M, N, K, batch, strides, p, c.slots, st);
+  if (c.bn == 256) return launch_mm<256, 1>(A, B, M, N, K, batch, strides, p, c, workspace, st);
+  return launch_mm<128, 1>(A, B, M, N, K, batch, strides, p, c, workspace, st);
+}
+
+extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+                      const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b,
+                      const float* bias, uint16_t* out_bf16, fp8_stream_t stream) {
+  return mm_impl(A, B, M, N, K, batch, strides, layout, sinv_a, sinv_b, bias, out_bf16, nullptr, 0, stream);
+}
+
+extern "C" int fp8_mm_ws(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+                         const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b,
+                         const float* bias, uint16_t* out_bf16, void* workspace, size_t workspace_bytes,
+                         fp8_stream_t stream) {
+  return mm_impl(A, B, M, N, K, batch, strides, layout, sinv_a, sinv_b, bias, out_bf16, workspace, workspace_bytes,
+                 stream);
+}
+
+extern "C" size_t fp8_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t batch, int layout) {
+  if (M <= 0 || N <= 0 || K <= 0 || batch < 1) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  const MmChoice c = choose_mm(M, N, K, batch, sms, (layout & FP8_MM_B_MN_MAJOR) != 0, size_t(1) << 40);
+  return c.ws_bytes;
 }

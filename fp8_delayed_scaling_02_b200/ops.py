@@ -74,6 +74,10 @@ def lib():
         L.fp8_quantize_current.restype = i32
         L.fp8_bias_grad.argtypes = [vp, i32, i64, i64, vp, vp]
         L.fp8_bias_grad.restype = i32
+        L.fp8_mm_ws.argtypes = [vp, vp, i64, i64, i64, i64, vp, i32, vp, vp, vp, vp, vp, ctypes.c_size_t, vp]
+        L.fp8_mm_ws.restype = i32
+        L.fp8_mm_workspace_bytes.argtypes = [i64, i64, i64, i64, i32]
+        L.fp8_mm_workspace_bytes.restype = ctypes.c_size_t
         L.fp8_linear_forward.argtypes = [vp, i32, vp, i32, i64, i64, i64, vp, CRing, CRing, vp, vp, vp, vp]
         L.fp8_linear_forward.restype = i32
         L.fp8_linear_backward.argtypes = [vp, i32, i64, i64, i64, CRing, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -176,15 +180,23 @@ def quantize(x, fmt, layout, ring, out=None, out_t=None, stream=None):
     return (out if layout in (ROW, DUAL) else None), (out_t if layout in (TRANSPOSED, DUAL) else None)
 
 
+def mm_workspace_bytes(M, N, K, batch=1, a_mn_major=False, b_mn_major=False):
+    """Bytes of workspace fp8_mm_ws would use (0 when whole tiles are as fast)."""
+    layout = (MM_A_MN_MAJOR if a_mn_major else 0) | (MM_B_MN_MAJOR if b_mn_major else 0)
+    return int((_LIB or lib()).fp8_mm_workspace_bytes(M, N, K, batch, layout))
+
+
 def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream=None,
-       a_mn_major=False, b_mn_major=False):
+       a_mn_major=False, b_mn_major=False, workspace=None):
     """fp8_mm: Y = bf16(A . B^T * sinv_a * sinv_b + bias).
 
     a: uint8 [M, K] or [Ba, M, K] (K contiguous), or with a_mn_major=True the
     stored [K, M] / [Ba, K, M] (M contiguous); b likewise [N, K] or, with
     b_mn_major=True, [K, N].  A size-1 (or 2-D) operand broadcasts over the
     batch at stride 0.  sinv_a / sinv_b: one-element float32 CUDA tensors.
-    bias: float32 [N] or None.
+    bias: float32 [N] or None.  workspace: optional zero-initialised uint8 CUDA
+    tensor (256-byte aligned) that lets the library spread the last waves' k-blocks
+    over all CTAs (stream-K, fp8_mm_ws).
     """
     if a.dtype != torch.uint8 or b.dtype != torch.uint8:
         raise ValueError("a and b hold FP8 codes as uint8")
@@ -205,8 +217,13 @@ def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream
             out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
         elif not out.is_contiguous() or out.shape != (M, N):
             raise ValueError("out must be a contiguous [M, N] bf16 tensor")
-        rc = L.fp8_mm(a.data_ptr(), b.data_ptr(), M, N, K, 1, None, layout, sinv_a.data_ptr(),
-                      sinv_b.data_ptr(), _ptr(bias), out.data_ptr(), _stream(stream, a.get_device()))
+        if workspace is None:
+            rc = L.fp8_mm(a.data_ptr(), b.data_ptr(), M, N, K, 1, None, layout, sinv_a.data_ptr(),
+                          sinv_b.data_ptr(), _ptr(bias), out.data_ptr(), _stream(stream, a.get_device()))
+        else:
+            rc = L.fp8_mm_ws(a.data_ptr(), b.data_ptr(), M, N, K, 1, None, layout, sinv_a.data_ptr(),
+                             sinv_b.data_ptr(), _ptr(bias), out.data_ptr(), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), _stream(stream, a.get_device()))
         _check(rc, "fp8_mm")
         return out
     a3 = a if a.dim() == 3 else a.unsqueeze(0)
@@ -225,8 +242,13 @@ def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream
         out = torch.empty((batch, M, N), dtype=torch.bfloat16, device=a.device)
     out3 = out if out.dim() == 3 else out.unsqueeze(0)
     strides = (ctypes.c_int64 * 3)(sa, sb, out3.stride(0) if batch > 1 else M * N)
-    rc = L.fp8_mm(a3.data_ptr(), b3.data_ptr(), M, N, K, batch, strides, layout, sinv_a.data_ptr(),
-                  sinv_b.data_ptr(), _ptr(bias), out3.data_ptr(), _stream(stream, a.get_device()))
+    if workspace is None:
+        rc = L.fp8_mm(a3.data_ptr(), b3.data_ptr(), M, N, K, batch, strides, layout, sinv_a.data_ptr(),
+                      sinv_b.data_ptr(), _ptr(bias), out3.data_ptr(), _stream(stream, a.get_device()))
+    else:
+        rc = L.fp8_mm_ws(a3.data_ptr(), b3.data_ptr(), M, N, K, batch, strides, layout, sinv_a.data_ptr(),
+                         sinv_b.data_ptr(), _ptr(bias), out3.data_ptr(), workspace.data_ptr(),
+                         workspace.numel() * workspace.element_size(), _stream(stream, a.get_device()))
     _check(rc, "fp8_mm")
     return out
 

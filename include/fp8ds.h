@@ -252,6 +252,38 @@ int fp8_linear_backward(const void* g, int g_dtype, int64_t M, int64_t N, int64_
                         const uint8_t* xq, const uint8_t* wq, const float* sinv_x, const float* sinv_w, uint8_t* gq,
                         uint16_t* dx, uint16_t* dw, float* db, fp8_stream_t stream);
 
+/*
+ * fp8_mm_ws -- fp8_mm with a caller-owned workspace that lets the library
+ * spread the k-blocks of the last waves' output tiles evenly over all CTAs
+ * (data-parallel whole tiles, then a stream-K tail), for outputs whose tile
+ * count leaves the GPU part-idle in its last wave (for example the dW = G^T.X
+ * GEMMs of a linear, whose output is only weight-sized).
+ * Same arguments, result and errors as fp8_mm, plus:
+ *   workspace       device memory, 256-byte aligned, all zero before its
+ *                   first use.  Its first 1024 bytes are per-piece arrival
+ *                   flags that every successful call leaves at zero, so the
+ *                   same workspace serves later calls on the same stream; the
+ *                   rest holds float32 partial tiles.  After a call that
+ *                   recorded a device error (fp8_device_error) zero it again.
+ *                   NULL (or smaller than fp8_mm_workspace_bytes) means
+ *                   whole tiles only, as fp8_mm.
+ *   workspace_bytes its size.  Calls that share a workspace must not overlap.
+ * A tile cut into pieces is finished by the CTA holding its first k-block,
+ * which adds the float32 partials of the later pieces in piece order, so
+ * results are deterministic; they may differ from the fp8_mm result in the
+ * last bits (both are within the same acceptance bound).
+ * The pages have no counterpart: it is a B200 scheduling addition for
+ * outputs whose tiles do not fill the last wave of SMs.
+ *
+ * fp8_mm_workspace_bytes -- the workspace size fp8_mm_ws would use for this
+ * problem on the current device (0 when whole tiles are as fast); at most
+ * 1024 + 148 x 128 x 256 x 4 bytes (about 19.4 MB) on a 148-SM B200.
+ */
+int fp8_mm_ws(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+              const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
+              uint16_t* out_bf16, void* workspace, size_t workspace_bytes, fp8_stream_t stream);
+size_t fp8_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t batch, int layout);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fp8_status_string(int status);
 

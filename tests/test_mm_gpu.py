@@ -179,3 +179,38 @@ def test_mn_major_batched_broadcast():
         ref, Ssum = OG.mm_fp8(a[z].numpy().T.copy(), b[0].numpy().T.copy(), 0, 0, 1.0, 1.0)
         ok, ratio = OG.check(y[z].float().cpu().numpy(), ref, Ssum)
         assert ok, (z, ratio)
+
+
+# Stream-K through a caller workspace (fp8_mm_ws): the k-blocks of the last
+# waves' tiles are dealt evenly to the CTAs, and pieces that start inside a
+# tile hand float32 partials to the CTA holding the tile's first k-block.
+# Shapes: the linear's dW GEMMs (fewer tiles than CTA pairs), wide outputs
+# with a wave of whole tiles before the stream-K tail (one ragged in M and
+# N), a tiny output cut four ways per tile, and ragged ones on 128-wide pair
+# tiles.  Checked against the oracle, deterministic across runs, flags left
+# at zero, and an undersized workspace falls back to whole tiles.
+@pytest.mark.parametrize("M,N,K,a_mn,b_mn", [(1536, 1536, 8192, False, False), (4096, 1536, 8192, True, True),
+                                             (1536, 1536, 8192, True, True), (512, 19200, 4096, False, False),
+                                             (500, 19199, 4096, False, False), (128, 256, 8192, False, False),
+                                             (1000, 1537, 8192, False, False), (130, 700, 8192, False, False)])
+def test_split_k_workspace(M, N, K, a_mn, b_mn):
+    a = S.fp8_codes((M, K), seed=M + 3)
+    b = S.fp8_codes((N, K), seed=N + 4)
+    bias = S.uniform((N,), seed=5)
+    need = ops.mm_workspace_bytes(M, N, K, a_mn_major=a_mn, b_mn_major=b_mn)
+    assert need > 0, "this shape should use stream-K pieces"
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    ad = a.t().contiguous().cuda() if a_mn else a.cuda()
+    bd = b.t().contiguous().cuda() if b_mn else b.cuda()
+    args = (ad, bd, _scalar(0.37), _scalar(0.125), bias.cuda())
+    y1 = ops.mm(*args, a_mn_major=a_mn, b_mn_major=b_mn, workspace=ws)
+    y2 = ops.mm(*args, a_mn_major=a_mn, b_mn_major=b_mn, workspace=ws)
+    small = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    y3 = ops.mm(*args, a_mn_major=a_mn, b_mn_major=b_mn, workspace=small)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2), "stream-K must be deterministic"
+    assert int(ws[:1024].count_nonzero()) == 0, "piece flags (the first 1024 bytes) must return to zero"
+    rows = np.unique(np.concatenate([np.random.default_rng(M).integers(0, M, 16), [0, M - 1]]))
+    for y in (y1, y3):
+        mm_check(y, a.numpy(), b.numpy(), ops.E4M3, ops.E4M3, np.float32(0.37), np.float32(0.125), bias.numpy(),
+                 rows)

@@ -12,8 +12,8 @@
 //     and writes one 16-byte store; loads are 16-byte vectors, realigned with
 //     funnel shifts when the input base is only element-aligned (a 2-byte
 //     offset for bf16), so the misaligned case reads HBM at full width too.
-//     Grid = a multiple of the SM count, grid-stride, two chunks in flight
-//     per thread.
+//     Grid = one wave of resident blocks, every thread taking the same
+//     number of chunks, two in flight at a time.
 //   * T / DUAL use a 128x64 tile per 256-thread block: each lane converts a
 //     4-row x 8-column patch, packs the 4 rows of each column into one 32-bit
 //     word, writes it to a padded shared tile (pitch 33 words: conflict-free
@@ -39,7 +39,9 @@
 namespace fp8ds {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;     // tile, amax and fallback kernels
+constexpr int kRowThreads = 256;  // ROW kernel block size
+constexpr int kRowMinChunks = 2;  // 16-element chunks per ROW thread, at least
 
 struct RingArgs {
   float* history;
@@ -345,15 +347,15 @@ __device__ __forceinline__ void row_chunk(const RowArgs& a, int64_t j, float s, 
 }
 
 template <int DT, int FMT, bool kAligned>
-__global__ void __launch_bounds__(kThreads) quantize_row_kernel(const RowArgs a) {
+__global__ void __launch_bounds__(kRowThreads) quantize_row_kernel(const RowArgs a) {
   constexpr int kB = In<DT>::kBytes;
   pdl_launch_dependents();
   pdl_wait_prior_grid();
   const float s = *a.ring.scale;
   const RingCache rc = prefetch_ring(a.ring);
   float amax = 0.0f;
-  const int64_t tid = int64_t(blockIdx.x) * kThreads + threadIdx.x;
-  const int64_t nthr = int64_t(gridDim.x) * kThreads;
+  const int64_t tid = int64_t(blockIdx.x) * kRowThreads + threadIdx.x;
+  const int64_t nthr = int64_t(gridDim.x) * kRowThreads;
 
   // Head and tail (fewer than 16 elements each): one element per thread.
   const int64_t tail0 = a.head + 16 * a.nchunks;
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(kThreads) quantize_row_kernel(const RowArgs a)
     row_chunk<DT, FMT, kAligned>(a, j, s, amax);
     if (j + nthr < a.nchunks) row_chunk<DT, FMT, kAligned>(a, j + nthr, s, amax);
   }
-  amax_ticket_fold<FMT>(amax, a.ring, s, rc);
+  amax_ticket_fold<FMT, kRowThreads>(amax, a.ring, s, rc);
 }
 
 // ---- T / DUAL layouts --------------------------------------------------------
@@ -397,6 +399,9 @@ template <int DT, int FMT, bool kDual>
 __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs a) {
   constexpr int kB = In<DT>::kBytes;
   __shared__ uint32_t sT[kTileC * kPitchW];
+  // DUAL with rows that are not 8-byte aligned: the tile's row-layout codes,
+  // [128 rows][64 bytes], leave as 32-byte coalesced warp stores.
+  __shared__ uint2 sR[kDual ? kTileR * kTileC / 8 : 1];
   pdl_launch_dependents();
   pdl_wait_prior_grid();
   const float s = *a.ring.scale;
@@ -428,17 +433,25 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs 
       q[i][0] = cvt4<FMT>(v[0], v[1], v[2], v[3], s);
       q[i][1] = cvt4<FMT>(v[4], v[5], v[6], v[7], s);
       if constexpr (kDual) {
-        uint8_t* o = a.out + r * a.cols + c;
-        if (interior && a.out8) {
-          *reinterpret_cast<uint2*>(o) = make_uint2(q[i][0], q[i][1]);
-        } else if (r < a.rows) {
+        if (a.out8) {
+          uint8_t* o = a.out + r * a.cols + c;
+          if (interior) {
+            *reinterpret_cast<uint2*>(o) = make_uint2(q[i][0], q[i][1]);
+          } else if (r < a.rows) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (c + j < a.cols) o[j] = uint8_t(q[i][j >> 2] >> (8 * (j & 3)));
+            for (int j = 0; j < 8; ++j)
+              if (c + j < a.cols) o[j] = uint8_t(q[i][j >> 2] >> (8 * (j & 3)));
+          }
         }
       }
     }
-    __syncthreads();  // previous tile's readers are done with sT
+    __syncthreads();  // previous tile's readers are done with sT and sR
+    if constexpr (kDual) {
+      if (!a.out8) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) sR[(lr0 + i) * (kTileC / 8) + (lc0 >> 3)] = make_uint2(q[i][0], q[i][1]);
+      }
+    }
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       uint32_t c[4];
@@ -447,6 +460,22 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs 
       for (int k = 0; k < 4; ++k) sT[(lc0 + 4 * h + k) * kPitchW + (lr0 >> 2)] = c[k];
     }
     __syncthreads();
+    if constexpr (kDual) {
+      if (!a.out8) {
+        // Warp w writes rows 16w .. 16w+15 of the tile, lane l bytes l and l+32.
+        const uint8_t* sRb = reinterpret_cast<const uint8_t*>(sR);
+#pragma unroll 4
+        for (int k = 0; k < kTileR / 8; ++k) {
+          const int rl = (kTileR / 8) * warp + k;
+          const int64_t r = r0 + rl;
+          if (r < a.rows) {
+            uint8_t* o = a.out + r * a.cols + c0;
+            if (c0 + lane < a.cols) o[lane] = sRb[rl * kTileC + lane];
+            if (c0 + lane + 32 < a.cols) o[lane + 32] = sRb[rl * kTileC + lane + 32];
+          }
+        }
+      }
+    }
 #pragma unroll
     for (int k = 0; k < kTileC / 8; ++k) {
       const int cl = 8 * warp + k;
@@ -611,7 +640,9 @@ __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __g
       uint32_t armed = 0, armed_par = 0;
       int stage = 0;
       uint32_t phase = 0;
-      uint32_t claim = atomicAdd(a.ring.scratch + 2, 1u);
+      // Tile blockIdx.x is this block's first; later tiles come from the
+      // shared counter, offset by the grid size.
+      uint32_t claim = blockIdx.x;
       while (true) {
         if (!bar_wait_bounded(empty0 + 8u * stage, phase ^ 1u)) {
           record_device_error(args.err, kWaitQuantizeTma);
@@ -619,7 +650,7 @@ __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __g
         }
         const uint32_t t = claim;
         if (t < ntiles) {
-          claim = atomicAdd(a.ring.scratch + 2, 1u);  // next claim in flight while this tile loads
+          claim = gridDim.x + atomicAdd(a.ring.scratch + 2, 1u);  // next claim in flight while this tile loads
           tile_id[stage] = t;
           issue_tile_load<DT>(&tmIn, sbase + uint32_t(stage * TT::kStageBytes), full0 + 8u * stage, t, tiles_c);
           armed |= 1u << stage;
@@ -847,30 +878,66 @@ int sm_count_current() {
   return cached[dev];
 }
 
-template <int DT, int FMT>
-int launch_row(const RowArgs& a, int grid, cudaStream_t st, bool aligned) {
-  const cudaError_t e = aligned ? launch_pdl(quantize_row_kernel<DT, FMT, true>, grid, kThreads, 0, st, 1, a)
-                                : launch_pdl(quantize_row_kernel<DT, FMT, false>, grid, kThreads, 0, st, 1, a);
+// Resident blocks per SM of a kernel without dynamic shared memory (cached
+// per device by the caller's static array).
+template <typename Kern>
+int resident_blocks(Kern kern, int threads, int (&cached)[64]) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, 0) != cudaSuccess || n < 1) return -1;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// ROW grid: one wave of resident blocks at most, and every thread takes the
+// same number of 16-element chunks (at least kRowMinChunks), so no fraction
+// of the blocks runs one more round than the rest.
+template <int DT, int FMT, bool kAligned>
+int launch_row1(const RowArgs& a, int sms, cudaStream_t st) {
+  static int cached[64] = {0};
+  const int bps = resident_blocks(quantize_row_kernel<DT, FMT, kAligned>, kRowThreads, cached);
+  if (bps <= 0) return FP8_ERR_CUDA;
+  const int64_t tmax = int64_t(bps) * sms * kRowThreads;
+  const int64_t per = std::max<int64_t>(kRowMinChunks, (a.nchunks + tmax - 1) / tmax);
+  const int grid = int(std::max<int64_t>(1, (a.nchunks + per * kRowThreads - 1) / (per * kRowThreads)));
+  const cudaError_t e = launch_pdl(quantize_row_kernel<DT, FMT, kAligned>, grid, kRowThreads, 0, st, 1, a);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 template <int DT, int FMT>
-int launch_tile(const TileArgs& a, int grid, cudaStream_t st, bool dual) {
-  const cudaError_t e = dual ? launch_pdl(quantize_tile_kernel<DT, FMT, true>, grid, kThreads, 0, st, 1, a)
-                             : launch_pdl(quantize_tile_kernel<DT, FMT, false>, grid, kThreads, 0, st, 1, a);
+int launch_row(const RowArgs& a, int sms, cudaStream_t st, bool aligned) {
+  return aligned ? launch_row1<DT, FMT, true>(a, sms, st) : launch_row1<DT, FMT, false>(a, sms, st);
+}
+
+// Element-aligned T / DUAL tiles: a grid of resident blocks (one wave).
+template <int DT, int FMT, bool kDual>
+int launch_tile1(const TileArgs& a, int sms, cudaStream_t st) {
+  static int cached[64] = {0};
+  const int bps = resident_blocks(quantize_tile_kernel<DT, FMT, kDual>, kThreads, cached);
+  if (bps <= 0) return FP8_ERR_CUDA;
+  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(a.ntiles, int64_t(bps) * sms)));
+  const cudaError_t e = launch_pdl(quantize_tile_kernel<DT, FMT, kDual>, grid, kThreads, 0, st, 1, a);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-template <int DT>
-int dispatch_fmt_row(int fmt, const RowArgs& a, int grid, cudaStream_t st, bool aligned) {
-  return fmt == FP8_E4M3 ? launch_row<DT, FP8_E4M3>(a, grid, st, aligned)
-                         : launch_row<DT, FP8_E5M2>(a, grid, st, aligned);
+template <int DT, int FMT>
+int launch_tile(const TileArgs& a, int sms, cudaStream_t st, bool dual) {
+  return dual ? launch_tile1<DT, FMT, true>(a, sms, st) : launch_tile1<DT, FMT, false>(a, sms, st);
 }
 
 template <int DT>
-int dispatch_fmt_tile(int fmt, const TileArgs& a, int grid, cudaStream_t st, bool dual) {
-  return fmt == FP8_E4M3 ? launch_tile<DT, FP8_E4M3>(a, grid, st, dual)
-                         : launch_tile<DT, FP8_E5M2>(a, grid, st, dual);
+int dispatch_fmt_row(int fmt, const RowArgs& a, int sms, cudaStream_t st, bool aligned) {
+  return fmt == FP8_E4M3 ? launch_row<DT, FP8_E4M3>(a, sms, st, aligned)
+                         : launch_row<DT, FP8_E5M2>(a, sms, st, aligned);
+}
+
+template <int DT>
+int dispatch_fmt_tile(int fmt, const TileArgs& a, int sms, cudaStream_t st, bool dual) {
+  return fmt == FP8_E4M3 ? launch_tile<DT, FP8_E4M3>(a, sms, st, dual)
+                         : launch_tile<DT, FP8_E5M2>(a, sms, st, dual);
 }
 
 // 2-D map over the input [rows, cols] with a 128-row x 128-byte box, 128B swizzle.
@@ -934,8 +1001,6 @@ int quantize_dispatch(const void* in, int dtype, int64_t rows, int64_t cols, int
   const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
   const int sms = sm_count_current();
   if (sms <= 0) return FP8_ERR_CUDA;
-  const int max_grid = sms * (2048 / kThreads);
-
   if (layout == FP8_LAYOUT_ROW) {
     RowArgs a{};
     a.in = static_cast<const uint8_t*>(in);
@@ -946,12 +1011,10 @@ int quantize_dispatch(const void* in, int dtype, int64_t rows, int64_t cols, int
     a.nchunks = (n - a.head) / 16;
     a.ring = r;
     const bool aligned = ((reinterpret_cast<uintptr_t>(in) + uintptr_t(a.head * eb)) & 15) == 0;
-    const int64_t want = (a.nchunks + 2 * kThreads - 1) / (2 * kThreads);
-    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(want, max_grid)));
     switch (dtype) {
-      case FP8_IN_BF16: return dispatch_fmt_row<FP8_IN_BF16>(fmt, a, grid, st, aligned);
-      case FP8_IN_FP16: return dispatch_fmt_row<FP8_IN_FP16>(fmt, a, grid, st, aligned);
-      default: return dispatch_fmt_row<FP8_IN_FP32>(fmt, a, grid, st, aligned);
+      case FP8_IN_BF16: return dispatch_fmt_row<FP8_IN_BF16>(fmt, a, sms, st, aligned);
+      case FP8_IN_FP16: return dispatch_fmt_row<FP8_IN_FP16>(fmt, a, sms, st, aligned);
+      default: return dispatch_fmt_row<FP8_IN_FP32>(fmt, a, sms, st, aligned);
     }
   }
 
@@ -978,11 +1041,10 @@ int quantize_dispatch(const void* in, int dtype, int64_t rows, int64_t cols, int
       default: return dispatch_fmt_tile_tma<FP8_IN_FP32>(fmt, a, map, sms, st, dual);
     }
   }
-  const int grid = int(std::max<int64_t>(1, std::min<int64_t>(a.ntiles, max_grid)));
   switch (dtype) {
-    case FP8_IN_BF16: return dispatch_fmt_tile<FP8_IN_BF16>(fmt, a, grid, st, dual);
-    case FP8_IN_FP16: return dispatch_fmt_tile<FP8_IN_FP16>(fmt, a, grid, st, dual);
-    default: return dispatch_fmt_tile<FP8_IN_FP32>(fmt, a, grid, st, dual);
+    case FP8_IN_BF16: return dispatch_fmt_tile<FP8_IN_BF16>(fmt, a, sms, st, dual);
+    case FP8_IN_FP16: return dispatch_fmt_tile<FP8_IN_FP16>(fmt, a, sms, st, dual);
+    default: return dispatch_fmt_tile<FP8_IN_FP32>(fmt, a, sms, st, dual);
   }
 }
 

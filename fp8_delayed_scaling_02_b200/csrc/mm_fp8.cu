@@ -632,41 +632,42 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
       auto emit = [&](int n0, const uint32_t(&v)[32]) {
         if (m0 >= p.M) return;  // warp-uniform: rows beyond M (pair peer of a short last tile)
         const bool full = n0 + 32 <= p.N;
+        uint32_t packed[16];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (p.bias != nullptr) {
+            if (full && p.bias_vec) {
+              bv = __ldg(reinterpret_cast<const float4*>(p.bias + n0) + j);
+            } else {
+              const int nn = n0 + 4 * j;
+              bv.x = nn < p.N ? __ldg(p.bias + nn) : 0.f;
+              bv.y = nn + 1 < p.N ? __ldg(p.bias + nn + 1) : 0.f;
+              bv.z = nn + 2 < p.N ? __ldg(p.bias + nn + 2) : 0.f;
+              bv.w = nn + 3 < p.N ? __ldg(p.bias + nn + 3) : 0.f;
+            }
+          }
+          const float y0 = fmaf(__uint_as_float(v[4 * j + 0]), sab, bv.x);
+          const float y1 = fmaf(__uint_as_float(v[4 * j + 1]), sab, bv.y);
+          const float y2 = fmaf(__uint_as_float(v[4 * j + 2]), sab, bv.z);
+          const float y3 = fmaf(__uint_as_float(v[4 * j + 3]), sab, bv.w);
+          const __nv_bfloat162 h01 = __floats2bfloat162_rn(y0, y1);
+          const __nv_bfloat162 h23 = __floats2bfloat162_rn(y2, y3);
+          packed[2 * j] = *reinterpret_cast<const uint32_t*>(&h01);
+          packed[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+        }
         const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
-        if (p.tma_store && lane == 0) bulk_wait_read_le1();  // this buffer's previous store has read it
+        // The buffer's previous TMA store has read it (checked after the math,
+        // so the wait overlaps it).
+        if (p.tma_store && lane == 0) bulk_wait_read_le1();
         __syncwarp();
         // 16-byte unit u of this lane's 64-byte row holds columns 8u .. 8u+7,
         // at unit position u ^ ((lane >> 1) & 3).
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          uint32_t packed[4];
-#pragma unroll
-          for (int jj = 0; jj < 2; ++jj) {
-            const int j = 2 * u + jj;
-            float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (p.bias != nullptr) {
-              if (full && p.bias_vec) {
-                bv = __ldg(reinterpret_cast<const float4*>(p.bias + n0) + j);
-              } else {
-                const int nn = n0 + 4 * j;
-                bv.x = nn < p.N ? __ldg(p.bias + nn) : 0.f;
-                bv.y = nn + 1 < p.N ? __ldg(p.bias + nn + 1) : 0.f;
-                bv.z = nn + 2 < p.N ? __ldg(p.bias + nn + 2) : 0.f;
-                bv.w = nn + 3 < p.N ? __ldg(p.bias + nn + 3) : 0.f;
-              }
-            }
-            const float y0 = fmaf(__uint_as_float(v[4 * j + 0]), sab, bv.x);
-            const float y1 = fmaf(__uint_as_float(v[4 * j + 1]), sab, bv.y);
-            const float y2 = fmaf(__uint_as_float(v[4 * j + 2]), sab, bv.z);
-            const float y3 = fmaf(__uint_as_float(v[4 * j + 3]), sab, bv.w);
-            const __nv_bfloat162 h01 = __floats2bfloat162_rn(y0, y1);
-            const __nv_bfloat162 h23 = __floats2bfloat162_rn(y2, y3);
-            packed[2 * jj] = *reinterpret_cast<const uint32_t*>(&h01);
-            packed[2 * jj + 1] = *reinterpret_cast<const uint32_t*>(&h23);
-          }
           const uint32_t addr = sbuf + uint32_t(lane) * 64u + uint32_t((u ^ ((lane >> 1) & 3)) * 16);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[0]), "r"(packed[1]),
-                       "r"(packed[2]), "r"(packed[3])
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[4 * u]),
+                       "r"(packed[4 * u + 1]), "r"(packed[4 * u + 2]), "r"(packed[4 * u + 3])
                        : "memory");
         }
         if (p.tma_store) {

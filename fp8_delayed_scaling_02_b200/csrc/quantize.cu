@@ -43,12 +43,17 @@ constexpr int kThreads = 256;     // tile, amax and fallback kernels
 constexpr int kRowThreads = 256;  // ROW kernel block size
 constexpr int kRowMinChunks = 2;  // 16-element chunks per ROW thread, at least
 
+// Three modes: fold (history set, amax_out null), local (amax_out set: the
+// last block writes the grid's amax and scale_inv and does not fold; the
+// fold follows after a cross-rank MAX of the amax) and fixed scale (both
+// null: current scaling's cast pass).
 struct RingArgs {
   float* history;
   int32_t* idx;
   float* scale;
   float* scale_inv;
   uint32_t* scratch;
+  float* amax_out;
 };
 
 // ---- element loads -----------------------------------------------------------
@@ -249,7 +254,7 @@ struct RingCache {
 
 __device__ __forceinline__ RingCache prefetch_ring(const RingArgs& ring) {
   RingCache c{0.0f, 0};
-  if (ring.history == nullptr) return c;  // fixed scale (current scaling's cast pass)
+  if (ring.history == nullptr || ring.amax_out != nullptr) return c;  // no fold in this call
   if (threadIdx.x < kHistoryLen) c.hist = ring.history[threadIdx.x];
   if (threadIdx.x == kHistoryLen) c.idx = *ring.idx;
   return c;
@@ -269,7 +274,7 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
   if (threadIdx.x < kHistoryLen) hist_s[threadIdx.x] = rc.hist;
   if (threadIdx.x == kHistoryLen) idx_s = rc.idx;
   __syncthreads();
-  if (ring.history == nullptr) {
+  if (ring.history == nullptr && ring.amax_out == nullptr) {
     // Fixed scale: no amax to publish; the last block clears the scratch
     // words (the tile counter is shared by every kernel that claims tiles).
     if (threadIdx.x == 0) {
@@ -302,6 +307,13 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
       const float a = __uint_as_float(bits);
       asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ring.scratch + 1) : "memory");
       asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ring.scratch + 2) : "memory");  // tile counter
+      if (ring.amax_out != nullptr) {
+        // Local mode: this rank's amax for the cross-rank MAX; the scale the
+        // call used is already known, so its inverse is published now.
+        *ring.amax_out = a;
+        *ring.scale_inv = __frcp_rn(s_used);
+        return;
+      }
       int idx = idx_s;
       idx = ((idx % kHistoryLen) + kHistoryLen) % kHistoryLen;
       hist_s[idx] = a;
@@ -1078,6 +1090,59 @@ extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t col
   if (rc != FP8_OK) return rc;
   const RingArgs r{ring.history, ring.idx, ring.scale, ring.scale_inv, ring.scratch};
   return quantize_dispatch(in, dtype, rows, cols, layout, fmt, r, out, out_t, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int fp8_quantize_local(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
+                                  fp8_ring ring, float* amax_out, uint8_t* out, uint8_t* out_t,
+                                  fp8_stream_t stream) {
+  if (!ring.scale || !ring.scale_inv || !ring.scratch || !amax_out) return FP8_ERR_INVALID_ARG;
+  const int rc = check_quantize_args(in, dtype, rows, cols, layout, fmt, out, out_t, ring.scratch);
+  if (rc != FP8_OK) return rc;
+  const RingArgs r{ring.history, ring.idx, ring.scale, ring.scale_inv, ring.scratch, amax_out};
+  return quantize_dispatch(in, dtype, rows, cols, layout, fmt, r, out, out_t, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace fp8ds {
+namespace {
+// The ring fold alone, of a given amax: one thread.  Same arithmetic as the
+// last block of a quantize call (history write, max over the window, scale =
+// FP8_MAX / max when positive, finite and finite in quotient; scale_inv =
+// 1 / the scale in effect before the fold).
+template <int FMT>
+__global__ void ring_fold_kernel(float* history, int32_t* idx_p, float* scale, float* scale_inv, const float* amax) {
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
+  if (threadIdx.x != 0) return;
+  const float a = *amax;
+  const float s_used = *scale;
+  int idx = *idx_p;
+  idx = ((idx % kHistoryLen) + kHistoryLen) % kHistoryLen;
+  history[idx] = a;
+  float mx = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kHistoryLen; ++i) mx = fmaxf(mx, history[i]);
+  *idx_p = (idx + 1) % kHistoryLen;
+  const float fmax = FMT == FP8_E4M3 ? kE4M3Max : kE5M2Max;
+  if (mx > 0.0f && isfinite(mx)) {
+    const float c = __fdiv_rn(fmax, mx);
+    if (isfinite(c) && c > 0.0f) *scale = c;
+  }
+  *scale_inv = __frcp_rn(s_used);
+}
+}  // namespace
+}  // namespace fp8ds
+
+extern "C" int fp8_ring_fold(fp8_ring ring, int fmt, const float* amax, fp8_stream_t stream) {
+  if (!ring.history || !ring.idx || !ring.scale || !ring.scale_inv || !amax) return FP8_ERR_INVALID_ARG;
+  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const cudaError_t e =
+      fmt == FP8_E4M3
+          ? launch_pdl(ring_fold_kernel<FP8_E4M3>, dim3(1), dim3(32), 0, st, 1, ring.history, ring.idx, ring.scale,
+                       ring.scale_inv, amax)
+          : launch_pdl(ring_fold_kernel<FP8_E5M2>, dim3(1), dim3(32), 0, st, 1, ring.history, ring.idx, ring.scale,
+                       ring.scale_inv, amax);
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 extern "C" int fp8_quantize_current(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,

@@ -82,6 +82,10 @@ def lib():
         L.fp8_linear_forward.restype = i32
         L.fp8_linear_backward.argtypes = [vp, i32, i64, i64, i64, CRing, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.fp8_linear_backward.restype = i32
+        L.fp8_quantize_local.argtypes = [vp, i32, i64, i64, i32, i32, CRing, vp, vp, vp, vp]
+        L.fp8_quantize_local.restype = i32
+        L.fp8_ring_fold.argtypes = [CRing, i32, vp, vp]
+        L.fp8_ring_fold.restype = i32
         _LIB = L
     return _LIB
 
@@ -178,6 +182,37 @@ def quantize(x, fmt, layout, ring, out=None, out_t=None, stream=None):
                                       _stream(stream, x.get_device()))
     _check(rc, "fp8_quantize")
     return (out if layout in (ROW, DUAL) else None), (out_t if layout in (TRANSPOSED, DUAL) else None)
+
+
+def quantize_local(x, fmt, layout, ring, amax=None, out=None, out_t=None, stream=None):
+    """fp8_quantize_local: the cast of ``quantize`` without the ring fold.
+
+    Writes ring.scale_inv (1 / the scale used) and this shard's amax into
+    ``amax`` (a one-element float32 CUDA tensor, allocated when None).
+    Returns (out, out_t, amax); fold later with ``ring_fold`` after the
+    ranks have MAX-reduced ``amax``.
+    """
+    if x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous 2-D tensor")
+    rows, cols = x.shape
+    if layout in (ROW, DUAL) and out is None:
+        out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+    if layout in (TRANSPOSED, DUAL) and out_t is None:
+        out_t = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+    if amax is None:
+        amax = torch.zeros(1, dtype=torch.float32, device=x.device)
+    rc = (_LIB or lib()).fp8_quantize_local(x.data_ptr(), IN_DTYPE[x.dtype], rows, cols, layout, fmt, ring.c(),
+                                            amax.data_ptr(), _ptr(out if layout in (ROW, DUAL) else None),
+                                            _ptr(out_t if layout in (TRANSPOSED, DUAL) else None),
+                                            _stream(stream, x.get_device()))
+    _check(rc, "fp8_quantize_local")
+    return (out if layout in (ROW, DUAL) else None), (out_t if layout in (TRANSPOSED, DUAL) else None), amax
+
+
+def ring_fold(ring, fmt, amax, stream=None):
+    """fp8_ring_fold: fold the amax in the one-element float32 CUDA tensor ``amax`` into ``ring``."""
+    rc = (_LIB or lib()).fp8_ring_fold(ring.c(), fmt, amax.data_ptr(), _stream(stream, amax.get_device()))
+    _check(rc, "fp8_ring_fold")
 
 
 def mm_workspace_bytes(M, N, K, batch=1, a_mn_major=False, b_mn_major=False):

@@ -138,6 +138,37 @@ int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t
                                 fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);
 
 /*
+ * fp8_quantize_local / fp8_ring_fold -- delayed scaling of a tensor sharded
+ * across data-parallel ranks: one scale for all shards.
+ *
+ * The pages fold each quantize's amax into the ring in the same kernel
+ * ("tests/extension" page, ring commit).  With a tensor split across ranks
+ * the fold needs the amax of the whole tensor, so the call is split in two
+ * around a cross-rank MAX of one float (the reading of the multi-GPU scale
+ * consistency item; the pages give no detail):
+ *   1. fp8_quantize_local casts with ring.scale exactly as fp8_quantize does
+ *      (same codes), writes 1/ring.scale to ring.scale_inv (the GEMM can run
+ *      at once) and this rank's amax over the raw values to *amax_out.  It
+ *      leaves history, idx and scale untouched (they may be NULL).
+ *   2. The caller MAX-reduces *amax_out over the ranks (NCCL or gloo).
+ *   3. fp8_ring_fold folds *amax into the ring (history[idx] = amax,
+ *      idx = (idx + 1) mod 16, scale = FP8_MAX / max(history) when positive
+ *      and finite, else kept; scale_inv = 1 / the scale before the fold).
+ * Every rank that starts from the same ring and folds the same global amax
+ * keeps an identical ring.  fp8_quantize_local followed by fp8_ring_fold of
+ * its own amax equals one fp8_quantize call bit for bit.
+ *
+ *   amax_out  device float, written by the last block of the call.
+ *   amax      device float read by the fold (device memory, never host).
+ * Other arguments, layouts and errors as fp8_quantize; ring.scratch follows
+ * the same rules.  fp8_ring_fold launches one single-thread kernel and
+ * returns FP8_ERR_INVALID_ARG for a NULL ring pointer or amax or a bad fmt.
+ */
+int fp8_quantize_local(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt, fp8_ring ring,
+                       float* amax_out, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);
+int fp8_ring_fold(fp8_ring ring, int fmt, const float* amax, fp8_stream_t stream);
+
+/*
  * fp8_quantize_current -- current (dynamic) scaling cast to FP8, no ring.
  *
  * The DynamicScaling path of the FP8Recipe commit ("tests/extension" page:

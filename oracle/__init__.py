@@ -29,7 +29,8 @@ Sources (the AstrAI commit-log pages):
 
 Modules:
   fp8_formats -- decode table and encoder (RNE + saturation) per format.
-  recipe      -- amax, quantize in row/transposed/dual layout, ring fold.
+  recipe      -- amax, quantize in row/transposed/dual layout, ring fold,
+                 current scaling, and the shard cast of data-parallel scaling.
   gemm        -- fp64 scaled GEMM, |a.b| sums and the acceptance bound.
   bias_grad   -- column sums of the output gradient (the bias gradient).
 

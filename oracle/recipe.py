@@ -147,3 +147,28 @@ def quantize_current(x, fmt, layout):
     out = q if layout in (ROW, DUAL) else None
     out_t = np.ascontiguousarray(q.T) if layout in (TRANSPOSED, DUAL) else None
     return out, out_t, a, s, np.float32(np.float32(1.0) / s)
+
+
+def quantize_local(x, fmt, layout, ring):
+    """One shard's cast without the fold (data-parallel delayed scaling).
+
+    Steps 1-4 above with the ring left untouched: the codes use ``ring.scale``
+    and the shard's amax is returned for a cross-rank MAX.  The fold of that
+    MAX with ``fold`` is the ring update of the whole tensor, because amax of
+    a union is the max of the shards' amaxes (reading of the data-parallel
+    scale-consistency item; the pages give no detail beyond the per-tensor
+    ring of the "tests/extension" ring commit).
+
+    Returns (out or None, out_t or None, amax, scale_inv) with
+    scale_inv = fp32(1 / ring.scale).
+    """
+    xf = to_float32(x)
+    assert xf.ndim == 2
+    s = np.float32(ring.scale)
+    a = amax(xf)
+    q = scaled_codes(xf, s, fmt)
+    out = q if layout in (ROW, DUAL) else None
+    out_t = np.ascontiguousarray(q.T) if layout in (TRANSPOSED, DUAL) else None
+    with np.errstate(divide="ignore"):
+        sinv = np.float32(np.float32(1.0) / s)
+    return out, out_t, a, sinv

@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
     assert declared_functions() == sorted(
         ["fp8_quantize", "fp8_mm", "fp8_status_string", "fp8_device_error", "fp8_device_info",
          "fp8_quantize_static_scratch", "fp8_quantize_current", "fp8_bias_grad", "fp8_linear_forward",
-         "fp8_linear_backward", "fp8_mm_ws", "fp8_mm_workspace_bytes"])
+         "fp8_linear_backward", "fp8_mm_ws", "fp8_mm_workspace_bytes", "fp8_quantize_local", "fp8_ring_fold"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -65,6 +65,20 @@ def test_quantize_rejects_bad_arguments_without_cuda(L):
     assert _q(L, dtype=2, inp=0x4002) == ops.FP8_ERR_UNSUPPORTED   # fp32 needs 4-byte alignment
     assert _q(L, dtype=0, inp=0x4001) == ops.FP8_ERR_UNSUPPORTED   # bf16 needs 2-byte alignment
     assert _q(L, ring=ops.CRing(0x1000, 0x1040, 0x1044, 0x1048, 0x104C)) == ops.FP8_ERR_UNSUPPORTED  # scratch % 8
+
+
+def test_local_quantize_and_ring_fold_reject_bad_arguments_without_cuda(L):
+    def ql(amax=0x5000, fmt=0, layout=0, ring=None, out=0x2000):
+        return L.fp8_quantize_local(ctypes.c_void_p(0x4000), 0, 4, 4, layout, fmt, ring or _ring(),
+                                    ctypes.c_void_p(amax), ctypes.c_void_p(out), ctypes.c_void_p(0x3000), None)
+    assert ql(amax=0) == ops.FP8_ERR_INVALID_ARG
+    assert ql(fmt=2) == ops.FP8_ERR_INVALID_ARG
+    assert ql(layout=0, out=0) == ops.FP8_ERR_INVALID_ARG
+    assert ql(ring=ops.CRing(0x1000, 0x1040, 0, 0x1048, 0x1050)) == ops.FP8_ERR_INVALID_ARG  # no scale
+    assert L.fp8_ring_fold(_ring(), 0, None, None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_ring_fold(_ring(), 2, ctypes.c_void_p(0x5000), None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_ring_fold(ops.CRing(0, 0x1040, 0x1044, 0x1048, 0x1050), 0, ctypes.c_void_p(0x5000),
+                           None) == ops.FP8_ERR_INVALID_ARG
 
 
 def _mm(L, M=128, N=128, K=128, batch=1, strides=None, layout=0, A=0x10000, B=0x20000, out=0x30000,

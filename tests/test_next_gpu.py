@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from fp8_delayed_scaling_02_b200 import ops, synthetic as S
-from gpu_helpers import assert_bytes_equal, require_gpu
+from gpu_helpers import assert_bytes_equal, assert_ring_equal, require_gpu
 from oracle import bias_grad as OB
 from oracle import recipe as OR
 
@@ -122,3 +122,47 @@ def test_linear_composite_matches_the_separate_calls_and_oracle():
                           rx.scale_inv.item())
     assert OG.check(dw.float().cpu().numpy(), ref, Ssum)[0]
     assert np.all(np.abs(db.cpu().numpy().astype(np.float64) - OB.bias_grad(g.cpu())) <= OB.bound(g.cpu()))
+
+
+@pytest.mark.parametrize("dtype,fmt", [("bf16", ops.E4M3), ("fp32", ops.E5M2)])
+@pytest.mark.parametrize("layout", [ops.ROW, ops.TRANSPOSED, ops.DUAL])
+def test_quantize_local_then_fold_equals_quantize(dtype, fmt, layout):
+    """fp8_quantize_local + fp8_ring_fold of its own amax = fp8_quantize, bit for bit, over 4 steps."""
+    r1, r2 = ops.Ring(), ops.Ring()
+    for step, (rows, cols) in enumerate([(256, 512), (130, 70), (8192, 1536), (7, 33)]):
+        x = S.quant_sweep_input(rows, cols, dtype, [1.0, 1e-3, 1e3, 1.0][step], seed=400 + step).cuda()
+        o1, t1 = ops.quantize(x, fmt, layout, r1)
+        o2, t2, amax = ops.quantize_local(x, fmt, layout, r2)
+        assert torch.equal(r2.scale_inv, r1.scale_inv), "scale_inv is published by the local cast"
+        ops.ring_fold(r2, fmt, amax)
+        torch.cuda.synchronize()
+        for a, b in ((o1, o2), (t1, t2)):
+            if a is not None:
+                assert torch.equal(a, b)
+        assert torch.equal(r1.buf, r2.buf)
+        assert _bits(amax.item()) == _bits(OR.amax(OR.to_float32(x.cpu())))
+
+
+def test_dp_two_shards_match_the_whole_tensor():
+    """Two ranks emulated on one GPU: each casts its shard, the MAX of the two
+    amaxes (taken on the device, as the collective would) is folded into both
+    rings; codes and rings equal one quantize of the whole tensor and the oracle."""
+    rows, cols = 2048, 1536
+    r0, r1, rr = ops.Ring(), ops.Ring(), ops.Ring()
+    ref = OR.Ring()
+    for step in range(5):
+        full = S.normal_with_outliers((rows, cols), seed=500 + step, frac=0.005, mult=10.0 * (1 + step % 3))
+        x = full.cuda()
+        o0, t0, a0 = ops.quantize_local(x[: rows // 2].contiguous(), ops.E4M3, ops.DUAL, r0)
+        o1, t1, a1 = ops.quantize_local(x[rows // 2:].contiguous(), ops.E4M3, ops.DUAL, r1)
+        g = torch.maximum(a0, a1)
+        ops.ring_fold(r0, ops.E4M3, g)
+        ops.ring_fold(r1, ops.E4M3, g)
+        o, t = ops.quantize(x, ops.E4M3, ops.DUAL, rr)
+        torch.cuda.synchronize()
+        assert torch.equal(torch.cat([o0, o1]), o)
+        assert torch.equal(torch.cat([t0, t1], dim=1), t)
+        assert torch.equal(r0.buf, rr.buf) and torch.equal(r1.buf, rr.buf)
+        r_out, r_out_t, _ = OR.quantize(full, OR.F.E4M3, OR.DUAL, ref)
+        assert_bytes_equal(o, r_out, "out")
+    assert_ring_equal(rr, ref)

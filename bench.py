@@ -8,7 +8,9 @@ workload (hidden 1536, FFN 4096) at M = 8192 tokens, for both linear shapes
   fwd  Y  = Xq . Wq^T * sx*sw + b      (M x N x 1536)
   dX   = Gq . (W^T)q^T * sg*sw          (M x 1536 x N, A = E5M2)
   dW   = (G^T)q . (X^T)q^T * sg*sx      (N x 1536 x M, A = E5M2)
-12 kernel launches per step (6 quantize, 6 GEMM).  The device-timed steps
+dX and dW of a linear go through fp8_mm_pair (one launch when the library's
+time model pairs them), so a step is 10 to 12 kernel launches, counted with
+fp8_launch_count while the step's graph is captured.  The device-timed steps
 replay a CUDA graph of the step; the end-to-end figure calls the C ABI
 directly every step with host copies in and out.
 
@@ -167,10 +169,11 @@ class Linear:
 
     def gemms(self, ops):
         ops.mm(self.xq, self.wq, self.rx.scale_inv, self.rw.scale_inv, self.bias, out=self.y, workspace=self.ws)
-        ops.mm(self.gq, self.wq_t, self.rg.scale_inv, self.rw.scale_inv, None, fmt_a=ops.E5M2, out=self.dx,
-               workspace=self.ws)
-        ops.mm(self.gq_t, self.xq_t, self.rg.scale_inv, self.rx.scale_inv, None, fmt_a=ops.E5M2, out=self.dw,
-               workspace=self.ws)
+        # dX and dW are independent: one fp8_mm_pair launch shares the GPU between them.
+        ops.mm_pair(dict(a=self.gq, b=self.wq_t, sinv_a=self.rg.scale_inv, sinv_b=self.rw.scale_inv,
+                         fmt_a=ops.E5M2, out=self.dx),
+                    dict(a=self.gq_t, b=self.xq_t, sinv_a=self.rg.scale_inv, sinv_b=self.rx.scale_inv,
+                         fmt_a=ops.E5M2, out=self.dw), workspace=self.ws)
 
     # The same step with the layout tag: row-layout quantizes only, and the
     # backward GEMMs read W, G and X as quantized through MN-major operands.
@@ -181,10 +184,10 @@ class Linear:
 
     def gemms_mn(self, ops):
         ops.mm(self.xq, self.wq, self.rx.scale_inv, self.rw.scale_inv, self.bias, out=self.y, workspace=self.ws)
-        ops.mm(self.gq, self.wq, self.rg.scale_inv, self.rw.scale_inv, None, fmt_a=ops.E5M2, out=self.dx,
-               b_mn_major=True, workspace=self.ws)
-        ops.mm(self.gq, self.xq, self.rg.scale_inv, self.rx.scale_inv, None, fmt_a=ops.E5M2, out=self.dw,
-               a_mn_major=True, b_mn_major=True, workspace=self.ws)
+        ops.mm_pair(dict(a=self.gq, b=self.wq, sinv_a=self.rg.scale_inv, sinv_b=self.rw.scale_inv,
+                         fmt_a=ops.E5M2, out=self.dx, b_mn_major=True),
+                    dict(a=self.gq, b=self.xq, sinv_a=self.rg.scale_inv, sinv_b=self.rx.scale_inv,
+                         fmt_a=ops.E5M2, out=self.dw, a_mn_major=True, b_mn_major=True), workspace=self.ws)
 
 
 def build_workload(M, torch, ops, S, n_sets=2):
@@ -459,17 +462,21 @@ def main():
     torch.cuda.synchronize()
     if args.profile:
         torch.cuda.nvtx.range_push("fp8_profile_step")
+        n0 = ops.launch_count()
         run_step(lins, ops, 0)
+        n1 = ops.launch_count()
         torch.cuda.nvtx.range_pop()
         torch.cuda.synchronize()
-        print(json.dumps({"profile_step": "done", "M": M, "launches": 12}))
+        print(json.dumps({"profile_step": "done", "M": M, "launches": n1 - n0}))
         return 0
     q_ms, g_ms = time_split(lins, ops, torch, 50)
 
     # The timed steps replay a CUDA graph of two consecutive steps (one per
     # input set), so the host launch cost is off the measured device time.
     steps = args.steps + (args.steps % 2)
+    n0 = ops.launch_count()
     graph = capture(torch, lambda: (run_step(lins, ops, 0), run_step(lins, ops, 1)))
+    launches_per_step = (ops.launch_count() - n0) // 2
     graph.replay()
     st = torch.cuda.current_stream()
     if pg:
@@ -578,12 +585,12 @@ def main():
             "roofline": {"bound": "tensor", "achieved": round(gemm_tf, 2), "peak": round(fp8_peak, 1),
                          "unit": "TFLOP/s", "frac": round(gemm_tf / fp8_peak, 4),
                          "traffic": traffic if M == 8192 else None,
-                         "kernel": "mm_fp8_kernel (all 6 GEMM launches of the step)", "peak_source": peak_src},
+                         "kernel": "mm_fp8 (all GEMM launches of the step: fwd, and dX + dW through fp8_mm_pair)", "peak_source": peak_src},
             "quantize_roofline": {"bound": "hbm", "achieved": round(quant_gbs, 1), "peak": hbm_peak, "unit": "GB/s",
                                   "frac": round(quant_gbs / hbm_peak, 4), "peak_source": "of measured hbm_gbs"},
             "clocks": clk.summary(t_clk0, t_clk1),
-            "gpu_launches": 12 * steps,
-            "timing": "device events around CUDA-graph replays of the step (12 kernels per step)",
+            "gpu_launches": launches_per_step * steps,
+            "timing": f"device events around CUDA-graph replays of the step ({launches_per_step} kernels per step)",
             "e2e": e2e,
         }
         if world == 1 and not args.no_cpu_baseline:

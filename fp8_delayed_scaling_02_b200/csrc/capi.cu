@@ -2,6 +2,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -109,6 +110,15 @@ bool encode_tiled_cached(void* map, int data_type, int rank, const void* base, c
   return true;
 }
 }  // namespace fp8ds
+
+namespace fp8ds {
+namespace {
+std::atomic<unsigned long long> g_launches{0};
+}  // namespace
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace fp8ds
+
+extern "C" uint64_t fp8_launch_count(void) { return fp8ds::g_launches.load(std::memory_order_relaxed); }
 
 extern "C" const char* fp8_status_string(int status) {
   switch (status) {

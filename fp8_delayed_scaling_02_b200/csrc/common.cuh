@@ -69,6 +69,10 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Counts one successful kernel launch (the library-wide launch counter read
+// by fp8_launch_count).
+void note_launch();
+
 // cudaLaunchKernelEx with programmatic stream serialisation (and a cluster
 // shape when cluster_x > 1).
 template <typename... KArgs, typename... Args>
@@ -93,7 +97,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e == cudaSuccess) note_launch();
+  return e;
 }
 
 }  // namespace fp8ds

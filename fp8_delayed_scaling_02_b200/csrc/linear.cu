@@ -11,6 +11,7 @@
 //   backward  Gq = quantize(G, E5M2, ring_g)        (row layout)
 //             dX = bf16(Gq . Wq * sinv_g * sinv_w)  (Wq read MN-major: [K=N, N=K_in])
 //             dW = bf16(Gq^T . Xq * sinv_g * sinv_x)  (Gq and Xq read MN-major)
+//             (dX and dW in one fp8_mm_pair launch when both are wanted)
 //             db = column sums of G (float32, deterministic)
 // The backward's sinv_x / sinv_w are the forward's ring_x / ring_w
 // scale_inv: valid as long as X and W are not quantized again between the
@@ -36,17 +37,21 @@ extern "C" int fp8_linear_backward(const void* g, int g_dtype, int64_t M, int64_
   int rc = fp8_quantize(g, g_dtype, M, N, FP8_LAYOUT_ROW, FP8_E5M2, ring_g, gq, nullptr, stream);
   if (rc != FP8_OK) return rc;
   // dX [M, K] = G [M, N] . W [N, K]: A = Gq K-major (K = N), B = Wq stored [N, K] = MN-major.
-  if (dx != nullptr) {
-    rc = fp8_mm(gq, wq, M, K, N, 1, nullptr, FP8_MM_B_MN_MAJOR | FP8_MM_A_E5M2, ring_g.scale_inv, sinv_w, nullptr,
-                dx, stream);
-    if (rc != FP8_OK) return rc;
-  }
+  const fp8_mm_args ax{gq, wq, M, K, N, 1, nullptr, FP8_MM_B_MN_MAJOR | FP8_MM_A_E5M2, ring_g.scale_inv, sinv_w,
+                       nullptr, dx};
   // dW [N, K] = G^T [N, M] . X [M, K]: A = Gq stored [M, N] = MN-major, B = Xq stored [M, K] = MN-major.
-  if (dw != nullptr) {
-    rc = fp8_mm(gq, xq, N, K, M, 1, nullptr, FP8_MM_A_MN_MAJOR | FP8_MM_B_MN_MAJOR | FP8_MM_A_E5M2,
-                ring_g.scale_inv, sinv_x, nullptr, dw, stream);
-    if (rc != FP8_OK) return rc;
+  const fp8_mm_args aw{gq, xq, N, K, M, 1, nullptr, FP8_MM_A_MN_MAJOR | FP8_MM_B_MN_MAJOR | FP8_MM_A_E5M2,
+                       ring_g.scale_inv, sinv_x, nullptr, dw};
+  // Both wanted: one launch shares the GPU between them (the weight-sized dW
+  // output alone leaves SMs idle).
+  if (dx != nullptr && dw != nullptr) {
+    rc = fp8_mm_pair(&ax, &aw, nullptr, 0, stream);
+  } else if (dx != nullptr) {
+    rc = fp8_mm(ax.A, ax.B, ax.M, ax.N, ax.K, 1, nullptr, ax.layout, ax.sinv_a, ax.sinv_b, nullptr, dx, stream);
+  } else if (dw != nullptr) {
+    rc = fp8_mm(aw.A, aw.B, aw.M, aw.N, aw.K, 1, nullptr, aw.layout, aw.sinv_a, aw.sinv_b, nullptr, dw, stream);
   }
+  if (rc != FP8_OK) return rc;
   if (db != nullptr) return fp8_bias_grad(g, g_dtype, M, N, db, stream);
   return FP8_OK;
 }

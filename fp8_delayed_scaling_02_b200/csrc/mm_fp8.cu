@@ -374,10 +374,11 @@ __device__ __forceinline__ void decode_tile(const MmParams& p, int t, int& b, in
   nt = rr / gm;
 }
 
+// One CTA's (pair's) whole life: problem `p` with maps tmA / tmB / tmC, as
+// CTA (pair) `cta` of the `ctas` that work on this problem.
 template <int BN, int PAIR>
-__global__ void __launch_bounds__(kThreadsMM, 1)
-    mm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const __grid_constant__ CUtensorMap tmC, const MmParams p) {
+__device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmC,
+                                        const MmParams& p, const int cta, const int ctas) {
   using C = Cfg<BN, PAIR>;
   constexpr int kTileM = kBM * PAIR;
   extern __shared__ uint8_t smem_raw[];
@@ -401,8 +402,6 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
   pdl_launch_dependents();
   const uint32_t rank = PAIR == 2 ? cluster_ctarank() : 0u;
   const bool leader = rank == 0;
-  const int cta = int(blockIdx.x) / PAIR;  // this CTA's (pair's) index: its whole tiles and stream-K piece
-  const int ctas = int(gridDim.x) / PAIR;  // whole tiles advance by the number of CTAs (pairs)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
@@ -419,9 +418,9 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
-    if (p.tma_store) prefetch_tmap(&tmC);
+    prefetch_tmap(tmA);
+    prefetch_tmap(tmB);
+    if (p.tma_store) prefetch_tmap(tmC);
   }
   if constexpr (PAIR == 2) cluster_sync();  // the peer's barriers exist before any remote arrive
   if (warp == 1) tmem_alloc_g<PAIR>(smem_u32(tmem_slot), C::kTmemCols);
@@ -469,13 +468,13 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
             if constexpr (PAIR == 1) tma_load_3d(dst, tm, c0, c1, c2, bar);
             else tma_load_3d_pair(dst, tm, c0, c1, c2, bar);
           };
-          if (p.a_mn) load(sa, &tmA, arow, kb * kBK, ba);
-          else load(sa, &tmA, kb * kBK, arow, ba);
+          if (p.a_mn) load(sa, tmA, arow, kb * kBK, ba);
+          else load(sa, tmA, kb * kBK, arow, ba);
           if (p.b_mn) {
 #pragma unroll
-            for (int g = 0; g < C::kBRows / 128; ++g) load(sb + g * 16384u, &tmB, brow + 128 * g, kb * kBK, bb);
+            for (int g = 0; g < C::kBRows / 128; ++g) load(sb + g * 16384u, tmB, brow + 128 * g, kb * kBK, bb);
           } else {
-            load(sb, &tmB, kb * kBK, brow, bb);
+            load(sb, tmB, kb * kBK, brow, bb);
           }
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
@@ -674,7 +673,7 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
           fence_async_smem();
           __syncwarp();
           if (lane == 0) {
-            tma_store_3d(&tmC, sbuf, n0, m0, b);
+            tma_store_3d(tmC, sbuf, n0, m0, b);
             bulk_commit();
           }
         } else {
@@ -785,6 +784,28 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
   if (warp == 1) tmem_dealloc_g<PAIR>(tmem_base, C::kTmemCols);
 }
 
+template <int BN, int PAIR>
+__global__ void __launch_bounds__(kThreadsMM, 1)
+    mm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmC, const __grid_constant__ MmParams p) {
+  mm_body<BN, PAIR>(&tmA, &tmB, &tmC, p, int(blockIdx.x) / PAIR, int(gridDim.x) / PAIR);
+}
+
+// Two independent GEMMs in one persistent launch (the dX and dW GEMMs of a
+// linear's backward): CTAs (pairs) [0, split) work on problem 0 and the rest
+// on problem 1, each set over its own tiles, so a problem with too few tiles
+// to fill the GPU shares it with the other instead of leaving SMs idle.
+template <int BN, int PAIR>
+__global__ void __launch_bounds__(kThreadsMM, 1)
+    mm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                       const __grid_constant__ CUtensorMap tmC0, const __grid_constant__ MmParams p0,
+                       const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                       const __grid_constant__ CUtensorMap tmC1, const __grid_constant__ MmParams p1, const int split) {
+  const int g = int(blockIdx.x) / PAIR;
+  if (g < split) mm_body<BN, PAIR>(&tmA0, &tmB0, &tmC0, p0, g, split);
+  else mm_body<BN, PAIR>(&tmA1, &tmB1, &tmC1, p1, g - split, int(gridDim.x) / PAIR - split);
+}
+
 // K == 0: Y = bf16(bias) or 0.
 __global__ void mm_bias_only_kernel(uint16_t* out, const float* bias, int64_t M, int64_t N, int64_t batch,
                                     int64_t c_stride) {
@@ -890,6 +911,7 @@ int max_pairs(int sms) {
 struct MmChoice {
   int bn, pair, grid, dp_tiles, sk_ctas;
   size_t ws_bytes;
+  double cost;  // modelled time, microseconds
 };
 
 constexpr int kMaxPieces = 256;             // flag words in the workspace's first 1024 bytes
@@ -901,10 +923,22 @@ size_t sk_ws_bytes(int pieces, int bn, int pair) {
   return pieces > 0 ? kFlagBytes + size_t(pieces) * size_t(pair) * kBM * size_t(bn) * 4 : 0;
 }
 
+// One validated GEMM: its arguments and the parameters that do not depend on
+// the launch shape.
+struct MmProblem {
+  const uint8_t* A;
+  const uint8_t* B;
+  int64_t M, N, K, batch;
+  const int64_t* strides;
+  bool nothing;  // M == 0 or N == 0: no output
+  MmParams p;
+};
+
+// Tensor maps and tile parameters of problem q for the launch shape c.
 template <int BN, int PAIR>
-int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
-              const int64_t* strides, MmParams p, const MmChoice& c, void* ws, cudaStream_t st) {
-  CUtensorMap ta, tb, tc;
+int prepare_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+               const int64_t* strides, MmParams& p, const MmChoice& c, void* ws, CUtensorMap& ta, CUtensorMap& tb,
+               CUtensorMap& tc) {
   const int64_t ba = (batch > 1 && strides[0] != 0) ? batch : 1;
   const int64_t bb = (batch > 1 && strides[1] != 0) ? batch : 1;
   const bool okA = p.a_mn ? make_map_mn(&ta, A, K, M, ba, ba > 1 ? strides[0] : 0)
@@ -929,9 +963,49 @@ int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t 
   }
   p.group_m = 8;
   p.idesc |= (uint32_t(BN >> 3) << 17) | (uint32_t((kBM * PAIR) >> 4) << 24);
+  return FP8_OK;
+}
+
+template <int BN, int PAIR>
+int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+              const int64_t* strides, MmParams p, const MmChoice& c, void* ws, cudaStream_t st) {
+  CUtensorMap ta, tb, tc;
+  const int rc = prepare_mm<BN, PAIR>(A, B, M, N, K, batch, strides, p, c, ws, ta, tb, tc);
+  if (rc != FP8_OK) return rc;
   if (!ensure_smem_attr<BN, PAIR>()) return FP8_ERR_CUDA;
   const cudaError_t e = launch_pdl(mm_fp8_kernel<BN, PAIR>, dim3(PAIR * std::max(1, c.grid)), dim3(kThreadsMM),
                                    Cfg<BN, PAIR>::kSmemBytes, st, PAIR, ta, tb, tc, p);
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+template <int BN, int PAIR>
+bool ensure_pair_smem_attr() {
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!done[dev]) {
+    if (cudaFuncSetAttribute(mm_fp8_pair_kernel<BN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg<BN, PAIR>::kSmemBytes) != cudaSuccess)
+      return false;
+    done[dev] = true;
+  }
+  return true;
+}
+
+// Two problems in one launch: c0.grid CTAs (pairs) on problem 0, c1.grid on
+// problem 1, whole tiles only.
+template <int BN, int PAIR>
+int launch_pair(MmProblem& q0, const MmChoice& c0, MmProblem& q1, const MmChoice& c1, cudaStream_t st) {
+  CUtensorMap ta0, tb0, tc0, ta1, tb1, tc1;
+  MmParams p0 = q0.p, p1 = q1.p;
+  int rc = prepare_mm<BN, PAIR>(q0.A, q0.B, q0.M, q0.N, q0.K, q0.batch, q0.strides, p0, c0, nullptr, ta0, tb0, tc0);
+  if (rc != FP8_OK) return rc;
+  rc = prepare_mm<BN, PAIR>(q1.A, q1.B, q1.M, q1.N, q1.K, q1.batch, q1.strides, p1, c1, nullptr, ta1, tb1, tc1);
+  if (rc != FP8_OK) return rc;
+  if (!ensure_pair_smem_attr<BN, PAIR>()) return FP8_ERR_CUDA;
+  const cudaError_t e =
+      launch_pdl(mm_fp8_pair_kernel<BN, PAIR>, dim3(PAIR * (c0.grid + c1.grid)), dim3(kThreadsMM),
+                 Cfg<BN, PAIR>::kSmemBytes, st, PAIR, ta0, tb0, tc0, p0, ta1, tb1, tc1, p1, c0.grid);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
@@ -957,7 +1031,7 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool
   const Opt opts[4] = {{256, 2, 1.0}, {256, 1, 0.85}, {128, 2, 0.5}, {128, 1, 0.45}};
   constexpr int kMinIters = 4;  // k-blocks per piece, at least
   const int64_t kb = (K + kBK - 1) / kBK;
-  MmChoice best{256, 1, 1, 0, 0, 0};
+  MmChoice best{256, 1, 1, 0, 0, 0, 0.0};
   double best_cost = 1e300;
   for (const Opt& o : opts) {
     if (o.pair == 2 && M <= kBM) continue;  // the second CTA would hold no rows
@@ -969,7 +1043,7 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool
     const double dp_cost = double((tiles + slots - 1) / slots) * double(kb) * t_kb;
     if (dp_cost < best_cost) {
       best_cost = dp_cost;
-      best = MmChoice{o.bn, o.pair, int(std::min<int64_t>(tiles, slots)), int(tiles), 0, 0};
+      best = MmChoice{o.bn, o.pair, int(std::min<int64_t>(tiles, slots)), int(tiles), 0, 0, dp_cost};
     }
     if (ws_limit == 0 || tiles % slots == 0 || slots > kMaxPieces || kb < 2 * kMinIters) continue;
     const int64_t full = tiles / slots;
@@ -991,7 +1065,7 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool
       if (wsb > ws_limit) continue;
       if (cost < best_cost) {
         best_cost = cost;
-        best = MmChoice{o.bn, o.pair, int(dp > 0 ? slots : pieces), int(dp), int(pieces), wsb};
+        best = MmChoice{o.bn, o.pair, int(dp > 0 ? slots : pieces), int(dp), int(pieces), wsb, cost};
       }
     }
   }
@@ -1003,9 +1077,12 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool
 
 using namespace fp8ds;
 
-static int mm_impl(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
-                   const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
-                   uint16_t* out_bf16, void* workspace, size_t ws_bytes, fp8_stream_t stream) {
+namespace fp8ds {
+namespace {
+
+int mm_validate(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+                const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
+                uint16_t* out_bf16, MmProblem& q) {
   if (M < 0 || N < 0 || K < 0 || batch < 1) return FP8_ERR_INVALID_ARG;
   if ((layout & ~(FP8_MM_A_E5M2 | FP8_MM_B_E5M2 | FP8_MM_A_MN_MAJOR | FP8_MM_B_MN_MAJOR)) != FP8_MM_NT)
     return FP8_ERR_INVALID_ARG;
@@ -1013,30 +1090,29 @@ static int mm_impl(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int
   const bool b_mn = (layout & FP8_MM_B_MN_MAJOR) != 0;
   if (batch > 1 && strides == nullptr) return FP8_ERR_INVALID_ARG;
   if (batch > 1 && (strides[0] < 0 || strides[1] < 0 || strides[2] < 0)) return FP8_ERR_INVALID_ARG;
-  if (M == 0 || N == 0) return FP8_OK;
+  q = MmProblem{};
+  q.A = A;
+  q.B = B;
+  q.M = M;
+  q.N = N;
+  q.K = K;
+  q.batch = batch;
+  q.strides = strides;
+  q.nothing = M == 0 || N == 0;
+  if (q.nothing) return FP8_OK;
   if (out_bf16 == nullptr || sinv_a == nullptr || sinv_b == nullptr) return FP8_ERR_INVALID_ARG;
   if (K > 0 && (A == nullptr || B == nullptr)) return FP8_ERR_INVALID_ARG;
   if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2 || batch > 65535) return FP8_ERR_UNSUPPORTED;
   if (K % 16 != 0) return FP8_ERR_UNSUPPORTED;
   if ((a_mn && M % 16 != 0) || (b_mn && N % 16 != 0)) return FP8_ERR_UNSUPPORTED;  // MN-major row pitch
   if (reinterpret_cast<uintptr_t>(out_bf16) % 2 != 0) return FP8_ERR_UNSUPPORTED;
-  const int64_t c_stride = batch > 1 ? strides[2] : M * N;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-
-  if (K == 0) {
-    const int64_t total = batch * M * N;
-    const int grid = int(std::min<int64_t>((total + 255) / 256, 4096));
-    const cudaError_t e = launch_pdl(mm_bias_only_kernel, dim3(grid), dim3(256), 0, st, 1, out_bf16, bias, M, N,
-                                     batch, c_stride);
-    return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+  if (K > 0) {
+    if (reinterpret_cast<uintptr_t>(A) % 16 != 0 || reinterpret_cast<uintptr_t>(B) % 16 != 0)
+      return FP8_ERR_UNSUPPORTED;
+    if (batch > 1 && ((strides[0] % 16) != 0 || (strides[1] % 16) != 0)) return FP8_ERR_UNSUPPORTED;
   }
-  if (reinterpret_cast<uintptr_t>(A) % 16 != 0 || reinterpret_cast<uintptr_t>(B) % 16 != 0) return FP8_ERR_UNSUPPORTED;
-  if (batch > 1 && ((strides[0] % 16) != 0 || (strides[1] % 16) != 0)) return FP8_ERR_UNSUPPORTED;
-
-  const int sms = sm_count();
-  if (sms <= 0) return FP8_ERR_CUDA;
-
-  MmParams p{};
+  const int64_t c_stride = batch > 1 ? strides[2] : M * N;
+  MmParams& p = q.p;
   p.M = int(M);
   p.N = int(N);
   p.K = int(K);
@@ -1058,17 +1134,42 @@ static int mm_impl(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int
   p.b_mn = b_mn;
   p.idesc = (1u << 4) | (fa << 7) | (fb << 10) | (a_mn ? 1u << 15 : 0u) | (b_mn ? 1u << 16 : 0u);
   p.err = error_word_ptr();
+  return FP8_OK;
+}
 
-  // An MN-major B is loaded as boxes of 128 N-rows, so its per-CTA tile must
-  // hold whole boxes (no 128-wide CTA pair).
+int launch_bias_only(const MmProblem& q, cudaStream_t st) {
+  const int64_t total = q.batch * q.M * q.N;
+  const int grid = int(std::min<int64_t>((total + 255) / 256, 4096));
+  const cudaError_t e = launch_pdl(mm_bias_only_kernel, dim3(grid), dim3(256), 0, st, 1, q.p.out, q.p.bias, q.M, q.N,
+                                   q.batch, q.p.c_stride);
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+int mm_run(MmProblem& q, void* workspace, size_t ws_bytes, cudaStream_t st) {
+  if (q.nothing) return FP8_OK;
+  if (q.K == 0) return launch_bias_only(q, st);
+  const int sms = sm_count();
+  if (sms <= 0) return FP8_ERR_CUDA;
   if (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP8_ERR_UNSUPPORTED;
-  const MmChoice c = choose_mm(M, N, K, batch, sms, b_mn, workspace ? ws_bytes : 0);
+  const MmChoice c = choose_mm(q.M, q.N, q.K, q.batch, sms, q.p.b_mn, workspace ? ws_bytes : 0);
   if (c.pair == 2) {
-    if (c.bn == 256) return launch_mm<256, 2>(A, B, M, N, K, batch, strides, p, c, workspace, st);
-    return launch_mm<128, 2>(A, B, M, N, K, batch, strides, p, c, workspace, st);
+    if (c.bn == 256) return launch_mm<256, 2>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, c, workspace, st);
+    return launch_mm<128, 2>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, c, workspace, st);
   }
-  if (c.bn == 256) return launch_mm<256, 1>(A, B, M, N, K, batch, strides, p, c, workspace, st);
-  return launch_mm<128, 1>(A, B, M, N, K, batch, strides, p, c, workspace, st);
+  if (c.bn == 256) return launch_mm<256, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, c, workspace, st);
+  return launch_mm<128, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, c, workspace, st);
+}
+
+}  // namespace
+}  // namespace fp8ds
+
+static int mm_impl(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+                   const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
+                   uint16_t* out_bf16, void* workspace, size_t ws_bytes, fp8_stream_t stream) {
+  MmProblem q;
+  const int rc = mm_validate(A, B, M, N, K, batch, strides, layout, sinv_a, sinv_b, bias, out_bf16, q);
+  if (rc != FP8_OK) return rc;
+  return mm_run(q, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
@@ -1083,6 +1184,53 @@ extern "C" int fp8_mm_ws(const uint8_t* A, const uint8_t* B, int64_t M, int64_t 
                          fp8_stream_t stream) {
   return mm_impl(A, B, M, N, K, batch, strides, layout, sinv_a, sinv_b, bias, out_bf16, workspace, workspace_bytes,
                  stream);
+}
+
+extern "C" int fp8_mm_pair(const fp8_mm_args* a0, const fp8_mm_args* a1, void* workspace, size_t workspace_bytes,
+                           fp8_stream_t stream) {
+  if (a0 == nullptr || a1 == nullptr) return FP8_ERR_INVALID_ARG;
+  MmProblem q0, q1;
+  int rc = mm_validate(a0->A, a0->B, a0->M, a0->N, a0->K, a0->batch, a0->strides, a0->layout, a0->sinv_a,
+                       a0->sinv_b, a0->bias, a0->out_bf16, q0);
+  if (rc != FP8_OK) return rc;
+  rc = mm_validate(a1->A, a1->B, a1->M, a1->N, a1->K, a1->batch, a1->strides, a1->layout, a1->sinv_a, a1->sinv_b,
+                   a1->bias, a1->out_bf16, q1);
+  if (rc != FP8_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  auto separately = [&]() {
+    int r = mm_run(q0, workspace, workspace_bytes, st);
+    return r != FP8_OK ? r : mm_run(q1, workspace, workspace_bytes, st);
+  };
+  if (q0.nothing || q1.nothing || q0.K == 0 || q1.K == 0) return separately();
+  const int sms = sm_count();
+  if (sms <= 0) return FP8_ERR_CUDA;
+  if (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP8_ERR_UNSUPPORTED;
+  // Shared launch shape: 256-wide tiles, CTA pairs when both problems have
+  // more than 128 rows.  CTAs go one at a time to the problem whose whole
+  // tiles take longer with the CTAs it has.
+  const int pair = (q0.M > kBM && q1.M > kBM) ? 2 : 1;
+  const int slots = pair == 2 ? max_pairs<256>(sms) : sms;
+  if (slots < 2) return separately();
+  const int64_t t0 = ((q0.M + kBM * pair - 1) / (kBM * pair)) * ((q0.N + 255) / 256) * q0.batch;
+  const int64_t t1 = ((q1.M + kBM * pair - 1) / (kBM * pair)) * ((q1.N + 255) / 256) * q1.batch;
+  const int64_t kb0 = (q0.K + kBK - 1) / kBK, kb1 = (q1.K + kBK - 1) / kBK;
+  int64_t c0 = 1, c1 = 1;
+  auto span = [](int64_t tiles, int64_t c, int64_t kb) { return ((tiles + c - 1) / c) * kb; };
+  while (c0 + c1 < slots) {
+    const bool grow0 = c0 < t0 && (span(t0, c0, kb0) >= span(t1, c1, kb1) || c1 >= t1);
+    if (grow0) ++c0;
+    else if (c1 < t1) ++c1;
+    else break;
+  }
+  const double t_kb = 0.45 / (pair == 2 ? 1.0 : 0.85);
+  const double paired = double(std::max(span(t0, c0, kb0), span(t1, c1, kb1))) * t_kb;
+  const size_t wl = workspace ? workspace_bytes : 0;
+  const double apart = choose_mm(q0.M, q0.N, q0.K, q0.batch, sms, q0.p.b_mn, wl).cost +
+                       choose_mm(q1.M, q1.N, q1.K, q1.batch, sms, q1.p.b_mn, wl).cost;
+  if (paired > 0.97 * apart) return separately();
+  const MmChoice ch0{256, pair, int(c0), int(t0), 0, 0, 0.0};
+  const MmChoice ch1{256, pair, int(c1), int(t1), 0, 0, 0.0};
+  return pair == 2 ? launch_pair<256, 2>(q0, ch0, q1, ch1, st) : launch_pair<256, 1>(q0, ch0, q1, ch1, st);
 }
 
 extern "C" size_t fp8_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t batch, int layout) {

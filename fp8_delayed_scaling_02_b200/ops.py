@@ -86,6 +86,10 @@ def lib():
         L.fp8_quantize_local.restype = i32
         L.fp8_ring_fold.argtypes = [CRing, i32, vp, vp]
         L.fp8_ring_fold.restype = i32
+        L.fp8_mm_pair.argtypes = [vp, vp, vp, ctypes.c_size_t, vp]
+        L.fp8_mm_pair.restype = i32
+        L.fp8_launch_count.argtypes = []
+        L.fp8_launch_count.restype = ctypes.c_uint64
         _LIB = L
     return _LIB
 
@@ -215,10 +219,72 @@ def ring_fold(ring, fmt, amax, stream=None):
     _check(rc, "fp8_ring_fold")
 
 
+def launch_count():
+    """Kernels launched through the library by this process so far (fp8_launch_count)."""
+    return int((_LIB or lib()).fp8_launch_count())
+
+
 def mm_workspace_bytes(M, N, K, batch=1, a_mn_major=False, b_mn_major=False):
     """Bytes of workspace fp8_mm_ws would use (0 when whole tiles are as fast)."""
     layout = (MM_A_MN_MAJOR if a_mn_major else 0) | (MM_B_MN_MAJOR if b_mn_major else 0)
     return int((_LIB or lib()).fp8_mm_workspace_bytes(M, N, K, batch, layout))
+
+
+def _shape2d(a, b, a_mn_major, b_mn_major, out):
+    """(M, N, K, out) of a 2-D fp8_mm call; checks strides and allocates out."""
+    if (a_mn_major or b_mn_major) and not (a.is_contiguous() and b.is_contiguous()):
+        raise ValueError("operands must be contiguous")
+    K, M = a.shape if a_mn_major else (a.shape[1], a.shape[0])
+    Kb, N = b.shape if b_mn_major else (b.shape[1], b.shape[0])
+    if Kb != K:
+        raise ValueError("K mismatch")
+    if not (a_mn_major or b_mn_major) and K > 0 and (
+            (M > 1 and a.stride(0) != K) or a.stride(1) != 1 or (N > 1 and b.stride(0) != K) or b.stride(1) != 1):
+        raise ValueError("operands must be K-contiguous")
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    elif not out.is_contiguous() or out.shape != (M, N):
+        raise ValueError("out must be a contiguous [M, N] bf16 tensor")
+    return M, N, K, out
+
+
+def _layout(fmt_a, fmt_b, a_mn_major, b_mn_major):
+    return (MM_NT | (MM_A_E5M2 if fmt_a == E5M2 else 0) | (MM_B_E5M2 if fmt_b == E5M2 else 0)
+            | (MM_A_MN_MAJOR if a_mn_major else 0) | (MM_B_MN_MAJOR if b_mn_major else 0))
+
+
+class CMmArgs(ctypes.Structure):
+    """Mirror of ``fp8_mm_args``."""
+
+    _fields_ = [("A", ctypes.c_void_p), ("B", ctypes.c_void_p), ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("batch", ctypes.c_int64), ("strides", ctypes.c_void_p),
+                ("layout", ctypes.c_int), ("sinv_a", ctypes.c_void_p), ("sinv_b", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("out_bf16", ctypes.c_void_p)]
+
+
+def mm_pair(p0, p1, workspace=None, stream=None):
+    """fp8_mm_pair: two independent 2-D GEMMs in one launch (e.g. dX and dW).
+
+    p0, p1: dicts of ``mm`` keyword arguments (a, b, sinv_a, sinv_b and
+    optionally bias, fmt_a, fmt_b, out, a_mn_major, b_mn_major).  Returns
+    (out0, out1).
+    """
+    args, outs = [], []
+    for q in (p0, p1):
+        a, b = q["a"], q["b"]
+        if a.dtype != torch.uint8 or b.dtype != torch.uint8 or a.dim() != 2 or b.dim() != 2:
+            raise ValueError("a and b are 2-D uint8 FP8 codes")
+        amn, bmn = q.get("a_mn_major", False), q.get("b_mn_major", False)
+        M, N, K, out = _shape2d(a, b, amn, bmn, q.get("out"))
+        outs.append(out)
+        args.append(CMmArgs(a.data_ptr(), b.data_ptr(), M, N, K, 1, None,
+                            _layout(q.get("fmt_a", E4M3), q.get("fmt_b", E4M3), amn, bmn),
+                            q["sinv_a"].data_ptr(), q["sinv_b"].data_ptr(), _ptr(q.get("bias")), out.data_ptr()))
+    ws, wsb = (workspace.data_ptr(), workspace.numel() * workspace.element_size()) if workspace is not None else (None, 0)
+    rc = (_LIB or lib()).fp8_mm_pair(ctypes.byref(args[0]), ctypes.byref(args[1]), ws, wsb,
+                                     _stream(stream, p0["a"].get_device()))
+    _check(rc, "fp8_mm_pair")
+    return outs[0], outs[1]
 
 
 def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream=None,
@@ -239,19 +305,7 @@ def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream
               | (MM_A_MN_MAJOR if a_mn_major else 0) | (MM_B_MN_MAJOR if b_mn_major else 0))
     L = _LIB or lib()
     if a.dim() == 2 and b.dim() == 2:
-        if (a_mn_major or b_mn_major) and not (a.is_contiguous() and b.is_contiguous()):
-            raise ValueError("operands must be contiguous")
-        K, M = a.shape if a_mn_major else (a.shape[1], a.shape[0])
-        Kb, N = b.shape if b_mn_major else (b.shape[1], b.shape[0])
-        if Kb != K:
-            raise ValueError("K mismatch")
-        if not (a_mn_major or b_mn_major) and K > 0 and (
-                (M > 1 and a.stride(0) != K) or a.stride(1) != 1 or (N > 1 and b.stride(0) != K) or b.stride(1) != 1):
-            raise ValueError("operands must be K-contiguous")
-        if out is None:
-            out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
-        elif not out.is_contiguous() or out.shape != (M, N):
-            raise ValueError("out must be a contiguous [M, N] bf16 tensor")
+        M, N, K, out = _shape2d(a, b, a_mn_major, b_mn_major, out)
         if workspace is None:
             rc = L.fp8_mm(a.data_ptr(), b.data_ptr(), M, N, K, 1, None, layout, sinv_a.data_ptr(),
                           sinv_b.data_ptr(), _ptr(bias), out.data_ptr(), _stream(stream, a.get_device()))

@@ -315,6 +315,43 @@ int fp8_mm_ws(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t 
               uint16_t* out_bf16, void* workspace, size_t workspace_bytes, fp8_stream_t stream);
 size_t fp8_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t batch, int layout);
 
+/*
+ * fp8_mm_pair -- two independent GEMMs (each exactly an fp8_mm call) in one
+ * launch, such as the dX and dW GEMMs of a linear's backward.
+ *
+ * The persistent grid is split: one set of CTAs works through problem 0's
+ * output tiles and the rest through problem 1's, sized so both sets finish
+ * together.  A problem whose tiles cannot fill the GPU (the weight-sized dW
+ * output) then shares it with the other instead of leaving SMs idle.  When
+ * the library's time model says one launch per problem is as fast (or a
+ * problem is empty or has K = 0), the two run one after the other on
+ * `stream` as fp8_mm_ws calls with `workspace` (which may be NULL; see
+ * fp8_mm_ws; a paired launch does not use it).
+ *   a0, a1  host structs; each field as the fp8_mm argument of that name.
+ * Each output equals the corresponding fp8_mm result within the fp8_mm
+ * bound; errors as fp8_mm (the first problem's error is reported first).
+ * The pages have no counterpart (a B200 scheduling addition).
+ */
+typedef struct {
+  const uint8_t* A;
+  const uint8_t* B;
+  int64_t M, N, K, batch;
+  const int64_t* strides;
+  int layout;
+  const float* sinv_a;
+  const float* sinv_b;
+  const float* bias;
+  uint16_t* out_bf16;
+} fp8_mm_args;
+int fp8_mm_pair(const fp8_mm_args* a0, const fp8_mm_args* a1, void* workspace, size_t workspace_bytes,
+                fp8_stream_t stream);
+
+/* Number of kernels this process has launched through the library so far
+ * (every entry point, every device; a host-side counter, safe to call from
+ * any thread, never synchronises).  Tracing aid: the difference across a
+ * region is the kernel count of that region, e.g. of a captured CUDA graph. */
+uint64_t fp8_launch_count(void);
+
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fp8_status_string(int status);
 

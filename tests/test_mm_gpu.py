@@ -214,3 +214,52 @@ def test_split_k_workspace(M, N, K, a_mn, b_mn):
     for y in (y1, y3):
         mm_check(y, a.numpy(), b.numpy(), ops.E4M3, ops.E4M3, np.float32(0.37), np.float32(0.125), bias.numpy(),
                  rows)
+
+
+# fp8_mm_pair: two independent GEMMs in one launch (the dX and dW of a
+# linear), CTAs split between them.  Shapes: both linears' backward GEMMs
+# (paired with CTA pairs), a single-CTA pairing (one problem with M <= 128),
+# a ragged pair, and pairs the library runs one after the other (K = 0 on
+# one side).  Each output is checked against the oracle on sampled rows.
+PAIR_CASES = [
+    ((8192, 1536, 1536, False, True), (1536, 1536, 8192, True, True)),
+    ((8192, 1536, 4096, False, True), (4096, 1536, 8192, True, True)),
+    ((128, 512, 4096, False, False), (2048, 2048, 1024, False, False)),
+    ((1000, 1537, 512, False, False), (130, 700, 8192, False, False)),
+    ((512, 256, 0, False, False), (256, 384, 1024, False, False)),
+]
+
+
+@pytest.mark.parametrize("c0,c1", PAIR_CASES)
+def test_mm_pair_matches_the_oracle(c0, c1):
+    probs, refs = [], []
+    for i, (M, N, K, a_mn, b_mn) in enumerate((c0, c1)):
+        a = S.fp8_codes((M, K), seed=M + K + i, fmt=ops.E5M2 if i == 1 else ops.E4M3)
+        b = S.fp8_codes((N, K), seed=N + K + 7 * i)
+        bias = S.uniform((N,), seed=11 + i) if i == 0 else None
+        ad = a.t().contiguous().cuda() if a_mn else a.cuda()
+        bd = b.t().contiguous().cuda() if b_mn else b.cuda()
+        probs.append(dict(a=ad, b=bd, sinv_a=_scalar(0.5 + i), sinv_b=_scalar(0.25), bias=None if bias is None else
+                          bias.cuda(), fmt_a=ops.E5M2 if i == 1 else ops.E4M3, a_mn_major=a_mn, b_mn_major=b_mn))
+        refs.append((a, b, bias, M, i))
+    y0, y1 = ops.mm_pair(probs[0], probs[1])
+    torch.cuda.synchronize()
+    for y, (a, b, bias, M, i) in zip((y0, y1), refs):
+        rows = np.unique(np.concatenate([np.random.default_rng(M + i).integers(0, M, 12), [0, M - 1]]))
+        mm_check(y, a.numpy(), b.numpy(), ops.E5M2 if i == 1 else ops.E4M3, ops.E4M3, np.float32(0.5 + i),
+                 np.float32(0.25), None if bias is None else bias.numpy(), rows)
+
+
+def test_mm_pair_equals_separate_calls_when_the_shapes_match():
+    """With one launch shape for both (256-wide CTA pairs, whole tiles) the
+    paired results equal the single calls bit for bit."""
+    # 24 long tiles (K = 8192) beside 256 short ones (K = 1024): paired, and
+    # each alone also runs 256-wide CTA pairs over whole tiles.
+    a0, b0 = S.fp8_codes((1024, 8192), seed=1).cuda(), S.fp8_codes((1536, 8192), seed=2).cuda()
+    a1, b1 = S.fp8_codes((8192, 1024), seed=3).cuda(), S.fp8_codes((2048, 1024), seed=4).cuda()
+    s = _scalar(1.0)
+    y0, y1 = ops.mm_pair(dict(a=a0, b=b0, sinv_a=s, sinv_b=s), dict(a=a1, b=b1, sinv_a=s, sinv_b=s))
+    z0 = ops.mm(a0, b0, s, s)
+    z1 = ops.mm(a1, b1, s, s)
+    torch.cuda.synchronize()
+    assert torch.equal(y0, z0) and torch.equal(y1, z1)

@@ -8,9 +8,10 @@ workload (hidden 1536, FFN 4096) at M = 8192 tokens, for both linear shapes
   fwd  Y  = Xq . Wq^T * sx*sw + b      (M x N x 1536)
   dX   = Gq . (W^T)q^T * sg*sw          (M x 1536 x N, A = E5M2)
   dW   = (G^T)q . (X^T)q^T * sg*sx      (N x 1536 x M, A = E5M2)
-dX and dW of a linear go through fp8_mm_pair (one launch when the library's
-time model pairs them), so a step is 10 to 12 kernel launches, counted with
-fp8_launch_count while the step's graph is captured.  The device-timed steps
+X and W of a linear go through fp8_quantize_pair and its dX and dW through
+fp8_mm_pair (one launch each when the library pairs them), so a step is 8 to
+12 kernel launches, counted with fp8_launch_count while the step's graph is
+captured.  The device-timed steps
 replay a CUDA graph of the step; the end-to-end figure calls the C ABI
 directly every step with host copies in and out.
 
@@ -163,8 +164,9 @@ class Linear:
         self.ws = None  # stream-K workspace shared by the step's GEMMs (set by build_workload)
 
     def quantize(self, ops, x, g, ev=None):
-        ops.quantize(x, ops.E4M3, ops.DUAL, self.rx, self.xq, self.xq_t)
-        ops.quantize(self.w, ops.E4M3, ops.DUAL, self.rw, self.wq, self.wq_t)
+        # X and W (both needed by the forward GEMM) in one fp8_quantize_pair launch.
+        ops.quantize_pair(dict(x=x, fmt=ops.E4M3, layout=ops.DUAL, ring=self.rx, out=self.xq, out_t=self.xq_t),
+                          dict(x=self.w, fmt=ops.E4M3, layout=ops.DUAL, ring=self.rw, out=self.wq, out_t=self.wq_t))
         ops.quantize(g, ops.E5M2, ops.DUAL, self.rg, self.gq, self.gq_t)
 
     def gemms(self, ops):
@@ -178,8 +180,8 @@ class Linear:
     # The same step with the layout tag: row-layout quantizes only, and the
     # backward GEMMs read W, G and X as quantized through MN-major operands.
     def quantize_row(self, ops, x, g):
-        ops.quantize(x, ops.E4M3, ops.ROW, self.rx, self.xq)
-        ops.quantize(self.w, ops.E4M3, ops.ROW, self.rw, self.wq)
+        ops.quantize_pair(dict(x=x, fmt=ops.E4M3, layout=ops.ROW, ring=self.rx, out=self.xq),
+                          dict(x=self.w, fmt=ops.E4M3, layout=ops.ROW, ring=self.rw, out=self.wq))
         ops.quantize(g, ops.E5M2, ops.ROW, self.rg, self.gq)
 
     def gemms_mn(self, ops):

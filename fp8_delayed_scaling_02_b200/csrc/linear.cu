@@ -6,7 +6,7 @@
 // library's kernels, all launched on one stream with programmatic dependent
 // launch between them:
 //   forward   Xq = quantize(X, E4M3, ring_x)        (row layout)
-//             Wq = quantize(W, E4M3, ring_w)        (row layout)
+//             Wq = quantize(W, E4M3, ring_w)        (row layout; one fp8_quantize_pair launch with X)
 //             Y  = bf16(Xq . Wq^T * sinv_x * sinv_w + b)
 //   backward  Gq = quantize(G, E5M2, ring_g)        (row layout)
 //             dX = bf16(Gq . Wq * sinv_g * sinv_w)  (Wq read MN-major: [K=N, N=K_in])
@@ -22,9 +22,10 @@ extern "C" int fp8_linear_forward(const void* x, int x_dtype, const void* w, int
                                   int64_t K, const float* bias, fp8_ring ring_x, fp8_ring ring_w, uint8_t* xq,
                                   uint8_t* wq, uint16_t* y, fp8_stream_t stream) {
   if (M < 0 || N < 0 || K < 0) return FP8_ERR_INVALID_ARG;
-  int rc = fp8_quantize(x, x_dtype, M, K, FP8_LAYOUT_ROW, FP8_E4M3, ring_x, xq, nullptr, stream);
-  if (rc != FP8_OK) return rc;
-  rc = fp8_quantize(w, w_dtype, N, K, FP8_LAYOUT_ROW, FP8_E4M3, ring_w, wq, nullptr, stream);
+  // X and W in one launch (each with its own ring).
+  const fp8_quantize_args qx{x, x_dtype, M, K, FP8_LAYOUT_ROW, FP8_E4M3, ring_x, xq, nullptr};
+  const fp8_quantize_args qw{w, w_dtype, N, K, FP8_LAYOUT_ROW, FP8_E4M3, ring_w, wq, nullptr};
+  const int rc = fp8_quantize_pair(&qx, &qw, stream);
   if (rc != FP8_OK) return rc;
   return fp8_mm(xq, wq, M, N, K, 1, nullptr, FP8_MM_NT, ring_x.scale_inv, ring_w.scale_inv, bias, y, stream);
 }

@@ -242,7 +242,8 @@ __device__ __forceinline__ void transpose4x4(uint32_t r0, uint32_t r1, uint32_t 
 // ---- amax + ring fold --------------------------------------------------------
 
 // Block-reduce the per-thread amax, publish it with one atomicMax, draw a
-// ticket; the last block folds the ring.  Must be called by every thread.
+// ticket; the last of the `nblocks` blocks working on this ring folds it.
+// Must be called by every thread of the block.
 // The ring's history and idx are not written until the last block runs, so
 // each block reads them early (prefetch_ring at kernel start, one lane per
 // word) and the fold itself needs no dependent global reads besides the
@@ -262,7 +263,7 @@ __device__ __forceinline__ RingCache prefetch_ring(const RingArgs& ring) {
 
 template <int FMT, int NT = kThreads>
 __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& ring, float s_used,
-                                                 const RingCache& rc) {
+                                                 const RingCache& rc, const unsigned nblocks) {
   __shared__ float warp_max[NT / 32];
   __shared__ float hist_s[kHistoryLen];
   __shared__ int idx_s;
@@ -280,7 +281,7 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
     if (threadIdx.x == 0) {
       unsigned t;
       asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(ring.scratch + 1) : "memory");
-      if (t == gridDim.x - 1) {
+      if (t == nblocks - 1) {
         asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ring.scratch + 1) : "memory");
         asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(ring.scratch + 2) : "memory");
       }
@@ -300,7 +301,7 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
     // finishing together made its retries quadratic.)
     unsigned t;
     asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(ring.scratch + 1) : "memory");
-    last = (t == gridDim.x - 1);
+    last = (t == nblocks - 1);
     if (last) {
       uint32_t bits;
       asm volatile("atom.relaxed.gpu.global.exch.b32 %0, [%1], 0;" : "=r"(bits) : "l"(ring.scratch) : "memory");
@@ -358,16 +359,17 @@ __device__ __forceinline__ void row_chunk(const RowArgs& a, int64_t j, float s, 
   *reinterpret_cast<uint4*>(a.out + e) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
+// Block `blk` of the `nblk` blocks that work on tensor a.
 template <int DT, int FMT, bool kAligned>
-__global__ void __launch_bounds__(kRowThreads) quantize_row_kernel(const RowArgs a) {
+__device__ __forceinline__ void row_body(const RowArgs& a, const unsigned blk, const unsigned nblk) {
   constexpr int kB = In<DT>::kBytes;
   pdl_launch_dependents();
   pdl_wait_prior_grid();
   const float s = *a.ring.scale;
   const RingCache rc = prefetch_ring(a.ring);
   float amax = 0.0f;
-  const int64_t tid = int64_t(blockIdx.x) * kRowThreads + threadIdx.x;
-  const int64_t nthr = int64_t(gridDim.x) * kRowThreads;
+  const int64_t tid = int64_t(blk) * kRowThreads + threadIdx.x;
+  const int64_t nthr = int64_t(nblk) * kRowThreads;
 
   // Head and tail (fewer than 16 elements each): one element per thread.
   const int64_t tail0 = a.head + 16 * a.nchunks;
@@ -387,7 +389,21 @@ __global__ void __launch_bounds__(kRowThreads) quantize_row_kernel(const RowArgs
     row_chunk<DT, FMT, kAligned>(a, j, s, amax);
     if (j + nthr < a.nchunks) row_chunk<DT, FMT, kAligned>(a, j + nthr, s, amax);
   }
-  amax_ticket_fold<FMT, kRowThreads>(amax, a.ring, s, rc);
+  amax_ticket_fold<FMT, kRowThreads>(amax, a.ring, s, rc, nblk);
+}
+
+template <int DT, int FMT, bool kAligned>
+__global__ void __launch_bounds__(kRowThreads) quantize_row_kernel(const __grid_constant__ RowArgs a) {
+  row_body<DT, FMT, kAligned>(a, blockIdx.x, gridDim.x);
+}
+
+// Two tensors in one launch: blocks [0, split) cast a0, the rest a1.
+template <int DT, int FMT, bool kAligned>
+__global__ void __launch_bounds__(kRowThreads)
+    quantize_row_pair_kernel(const __grid_constant__ RowArgs a0, const __grid_constant__ RowArgs a1,
+                             const unsigned split) {
+  if (blockIdx.x < split) row_body<DT, FMT, kAligned>(a0, blockIdx.x, split);
+  else row_body<DT, FMT, kAligned>(a1, blockIdx.x - split, gridDim.x - split);
 }
 
 // ---- T / DUAL layouts --------------------------------------------------------
@@ -506,7 +522,7 @@ __global__ void __launch_bounds__(kThreads) quantize_tile_kernel(const TileArgs 
       }
     }
   }
-  amax_ticket_fold<FMT>(amax, a.ring, s, rc);
+  amax_ticket_fold<FMT>(amax, a.ring, s, rc, gridDim.x);
 }
 
 // ---- T / DUAL layouts, warp-specialised TMA pipeline (16-byte aligned rows) -------
@@ -614,8 +630,8 @@ __device__ __forceinline__ void issue_tile_load(const CUtensorMap* tm, uint32_t 
 __device__ __forceinline__ int tbuf_unit(int c, int v) { return c * 128 + ((v ^ ((c >> 2) & 6)) << 4); }
 
 template <int DT, int FMT, bool kDual>
-__global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __grid_constant__ CUtensorMap tmIn,
-                                                                        const TmaTileArgs args) {
+__device__ __forceinline__ void tile_tma_body(const CUtensorMap* tmIn, const TmaTileArgs& args, const unsigned blk,
+                                              const unsigned nblk) {
   using TT = TmaTile<DT>;
   constexpr int kB = In<DT>::kBytes;
   constexpr int S = TT::kStages;
@@ -637,7 +653,7 @@ __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __g
     }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmIn)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmIn)) : "memory");
   }
   __syncthreads();
   pdl_wait_prior_grid();
@@ -652,9 +668,9 @@ __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __g
       uint32_t armed = 0, armed_par = 0;
       int stage = 0;
       uint32_t phase = 0;
-      // Tile blockIdx.x is this block's first; later tiles come from the
-      // shared counter, offset by the grid size.
-      uint32_t claim = blockIdx.x;
+      // Tile blk is this block's first; later tiles come from the shared
+      // counter, offset by the number of blocks on this tensor.
+      uint32_t claim = blk;
       while (true) {
         if (!bar_wait_bounded(empty0 + 8u * stage, phase ^ 1u)) {
           record_device_error(args.err, kWaitQuantizeTma);
@@ -662,9 +678,9 @@ __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __g
         }
         const uint32_t t = claim;
         if (t < ntiles) {
-          claim = gridDim.x + atomicAdd(a.ring.scratch + 2, 1u);  // next claim in flight while this tile loads
+          claim = nblk + atomicAdd(a.ring.scratch + 2, 1u);  // next claim in flight while this tile loads
           tile_id[stage] = t;
-          issue_tile_load<DT>(&tmIn, sbase + uint32_t(stage * TT::kStageBytes), full0 + 8u * stage, t, tiles_c);
+          issue_tile_load<DT>(tmIn, sbase + uint32_t(stage * TT::kStageBytes), full0 + 8u * stage, t, tiles_c);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
         } else {
@@ -799,7 +815,25 @@ __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __g
     if constexpr (kB == 2) amax = fmaxf(amax, absmax2_to_float<DT>(amax2));
   }
   __syncthreads();
-  amax_ticket_fold<FMT, kWsThreads>(amax, a.ring, s, rc);
+  amax_ticket_fold<FMT, kWsThreads>(amax, a.ring, s, rc, nblk);
+}
+
+template <int DT, int FMT, bool kDual>
+__global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __grid_constant__ CUtensorMap tmIn,
+                                                                        const __grid_constant__ TmaTileArgs args) {
+  tile_tma_body<DT, FMT, kDual>(&tmIn, args, blockIdx.x, gridDim.x);
+}
+
+// Two tensors in one launch (a linear's X and W): blocks [0, split) work on
+// tensor 0, the rest on tensor 1, each set with its own ring, ticket and
+// tile counter.
+template <int DT, int FMT, bool kDual>
+__global__ void __launch_bounds__(kWsThreads)
+    quantize_tile_tma_pair_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ TmaTileArgs a0,
+                                  const __grid_constant__ CUtensorMap tm1, const __grid_constant__ TmaTileArgs a1,
+                                  const unsigned split) {
+  if (blockIdx.x < split) tile_tma_body<DT, FMT, kDual>(&tm0, a0, blockIdx.x, split);
+  else tile_tma_body<DT, FMT, kDual>(&tm1, a1, blockIdx.x - split, gridDim.x - split);
 }
 
 // ---- current scaling: amax pass ---------------------------------------------------
@@ -1007,14 +1041,27 @@ namespace fp8ds {
 namespace {
 // Launches the cast kernel for the layout (and the ring fold unless r.history
 // is null).  Arguments are already validated.
-int quantize_dispatch(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt, const RingArgs& r,
-                      uint8_t* out, uint8_t* out_t, cudaStream_t st) {
+// One quantize call resolved to its kernel: ROW, TMA tiles (16-byte aligned
+// rows) or element-aligned tiles, with the kernel arguments.
+enum QKind { kQRow = 0, kQTma = 1, kQTile = 2 };
+struct QPlan {
+  int kind, dtype, fmt, layout;
+  bool aligned;  // ROW: chunks start 16-byte aligned in the input
+  RowArgs ra;
+  TileArgs ta;
+  CUtensorMap map;
+};
+
+int quantize_plan(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt, const RingArgs& r,
+                  uint8_t* out, uint8_t* out_t, QPlan& q) {
   const int64_t n = rows * cols;
   const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
-  const int sms = sm_count_current();
-  if (sms <= 0) return FP8_ERR_CUDA;
+  q = QPlan{};
+  q.dtype = dtype;
+  q.fmt = fmt;
+  q.layout = layout;
   if (layout == FP8_LAYOUT_ROW) {
-    RowArgs a{};
+    RowArgs& a = q.ra;
     a.in = static_cast<const uint8_t*>(in);
     a.out = out;
     a.n = n;
@@ -1022,15 +1069,11 @@ int quantize_dispatch(const void* in, int dtype, int64_t rows, int64_t cols, int
     a.head = std::min<int64_t>(n, int64_t((16 - (oa & 15)) & 15));
     a.nchunks = (n - a.head) / 16;
     a.ring = r;
-    const bool aligned = ((reinterpret_cast<uintptr_t>(in) + uintptr_t(a.head * eb)) & 15) == 0;
-    switch (dtype) {
-      case FP8_IN_BF16: return dispatch_fmt_row<FP8_IN_BF16>(fmt, a, sms, st, aligned);
-      case FP8_IN_FP16: return dispatch_fmt_row<FP8_IN_FP16>(fmt, a, sms, st, aligned);
-      default: return dispatch_fmt_row<FP8_IN_FP32>(fmt, a, sms, st, aligned);
-    }
+    q.aligned = ((reinterpret_cast<uintptr_t>(in) + uintptr_t(a.head * eb)) & 15) == 0;
+    q.kind = kQRow;
+    return FP8_OK;
   }
-
-  TileArgs a{};
+  TileArgs& a = q.ta;
   a.in = static_cast<const uint8_t*>(in);
   a.out = out;
   a.out_t = out_t;
@@ -1041,22 +1084,134 @@ int quantize_dispatch(const void* in, int dtype, int64_t rows, int64_t cols, int
   a.out8 = (layout == FP8_LAYOUT_DUAL) && (reinterpret_cast<uintptr_t>(out) % 8 == 0) && (cols % 8 == 0);
   a.outt4 = (reinterpret_cast<uintptr_t>(out_t) % 4 == 0) && (rows % 4 == 0);
   a.ring = r;
-  const bool dual = layout == FP8_LAYOUT_DUAL;
   if (n > 0 && reinterpret_cast<uintptr_t>(in) % 16 == 0 && (cols * eb) % 16 == 0 && a.ntiles < (int64_t(1) << 30) &&
       rows < (int64_t(1) << 30) && cols < (int64_t(1) << 30)) {
-    CUtensorMap map;
-    std::memset(&map, 0, sizeof(map));
-    if (!make_input_map(&map, in, dtype, rows, cols)) return FP8_ERR_CUDA;
-    switch (dtype) {
-      case FP8_IN_BF16: return dispatch_fmt_tile_tma<FP8_IN_BF16>(fmt, a, map, sms, st, dual);
-      case FP8_IN_FP16: return dispatch_fmt_tile_tma<FP8_IN_FP16>(fmt, a, map, sms, st, dual);
-      default: return dispatch_fmt_tile_tma<FP8_IN_FP32>(fmt, a, map, sms, st, dual);
+    if (!make_input_map(&q.map, in, dtype, rows, cols)) return FP8_ERR_CUDA;
+    q.kind = kQTma;
+  } else {
+    q.kind = kQTile;
+  }
+  return FP8_OK;
+}
+
+int quantize_launch(const QPlan& q, int sms, cudaStream_t st) {
+  const bool dual = q.layout == FP8_LAYOUT_DUAL;
+  if (q.kind == kQRow) {
+    switch (q.dtype) {
+      case FP8_IN_BF16: return dispatch_fmt_row<FP8_IN_BF16>(q.fmt, q.ra, sms, st, q.aligned);
+      case FP8_IN_FP16: return dispatch_fmt_row<FP8_IN_FP16>(q.fmt, q.ra, sms, st, q.aligned);
+      default: return dispatch_fmt_row<FP8_IN_FP32>(q.fmt, q.ra, sms, st, q.aligned);
     }
   }
-  switch (dtype) {
-    case FP8_IN_BF16: return dispatch_fmt_tile<FP8_IN_BF16>(fmt, a, sms, st, dual);
-    case FP8_IN_FP16: return dispatch_fmt_tile<FP8_IN_FP16>(fmt, a, sms, st, dual);
-    default: return dispatch_fmt_tile<FP8_IN_FP32>(fmt, a, sms, st, dual);
+  if (q.kind == kQTma) {
+    switch (q.dtype) {
+      case FP8_IN_BF16: return dispatch_fmt_tile_tma<FP8_IN_BF16>(q.fmt, q.ta, q.map, sms, st, dual);
+      case FP8_IN_FP16: return dispatch_fmt_tile_tma<FP8_IN_FP16>(q.fmt, q.ta, q.map, sms, st, dual);
+      default: return dispatch_fmt_tile_tma<FP8_IN_FP32>(q.fmt, q.ta, q.map, sms, st, dual);
+    }
+  }
+  switch (q.dtype) {
+    case FP8_IN_BF16: return dispatch_fmt_tile<FP8_IN_BF16>(q.fmt, q.ta, sms, st, dual);
+    case FP8_IN_FP16: return dispatch_fmt_tile<FP8_IN_FP16>(q.fmt, q.ta, sms, st, dual);
+    default: return dispatch_fmt_tile<FP8_IN_FP32>(q.fmt, q.ta, sms, st, dual);
+  }
+}
+
+// Launches the cast kernel for the layout (and the ring fold unless r.history
+// is null).  Arguments are already validated.
+int quantize_dispatch(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt, const RingArgs& r,
+                      uint8_t* out, uint8_t* out_t, cudaStream_t st) {
+  const int sms = sm_count_current();
+  if (sms <= 0) return FP8_ERR_CUDA;
+  QPlan q;
+  const int rc = quantize_plan(in, dtype, rows, cols, layout, fmt, r, out, out_t, q);
+  return rc != FP8_OK ? rc : quantize_launch(q, sms, st);
+}
+
+// ---- two tensors in one launch -----------------------------------------------
+
+// Blocks for side 0 out of g, in proportion to the work w0 : w1, at least one
+// each side.
+int64_t share0(int64_t g, int64_t w0, int64_t w1) {
+  const int64_t s = (g * w0 + (w0 + w1) / 2) / std::max<int64_t>(1, w0 + w1);
+  return std::min<int64_t>(std::max<int64_t>(s, 1), g - 1);
+}
+
+template <int DT, int FMT, bool kAligned>
+int launch_row_pair1(const RowArgs& a0, const RowArgs& a1, int sms, cudaStream_t st) {
+  static int cached[64] = {0};
+  const int bps = resident_blocks(quantize_row_pair_kernel<DT, FMT, kAligned>, kRowThreads, cached);
+  if (bps <= 0) return FP8_ERR_CUDA;
+  const int64_t G = int64_t(bps) * sms;
+  const int64_t g0max = share0(G, a0.nchunks + 1, a1.nchunks + 1);
+  // Each side sized as a single launch with its share of the wave.
+  auto size = [](const RowArgs& a, int64_t gmax) {
+    const int64_t tmax = gmax * kRowThreads;
+    const int64_t per = std::max<int64_t>(kRowMinChunks, (a.nchunks + tmax - 1) / tmax);
+    return std::max<int64_t>(1, (a.nchunks + per * kRowThreads - 1) / (per * kRowThreads));
+  };
+  const int64_t g0 = size(a0, g0max), g1 = size(a1, G - g0max);
+  const cudaError_t e = launch_pdl(quantize_row_pair_kernel<DT, FMT, kAligned>, dim3(unsigned(g0 + g1)), kRowThreads, 0,
+                                   st, 1, a0, a1, unsigned(g0));
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+template <int DT, int FMT, bool kDual>
+int launch_tile_tma_pair1(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
+  static int cached[64] = {0};
+  auto kern = quantize_tile_tma_pair_kernel<DT, FMT, kDual>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
+  if (cached[dev] == 0) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TmaTile<DT>::kSmem) != cudaSuccess)
+      return FP8_ERR_CUDA;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kWsThreads, TmaTile<DT>::kSmem) != cudaSuccess || n < 1)
+      return FP8_ERR_CUDA;
+    cached[dev] = n;
+  }
+  const int64_t G = int64_t(cached[dev]) * sms;
+  const int64_t t0 = q0.ta.ntiles, t1 = q1.ta.ntiles;
+  const int64_t g0 = std::min<int64_t>(share0(G, t0, t1), t0);
+  const int64_t g1 = std::min<int64_t>(G - g0, t1);
+  const TmaTileArgs a0{q0.ta, error_word_ptr()}, a1{q1.ta, error_word_ptr()};
+  const cudaError_t e = launch_pdl(kern, dim3(unsigned(g0 + g1)), kWsThreads, TmaTile<DT>::kSmem, st, 1, q0.map, a0,
+                                   q1.map, a1, unsigned(g0));
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+template <int DT, int FMT>
+int launch_pair_dt_fmt(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
+  if (q0.kind == kQRow)
+    return q0.aligned ? launch_row_pair1<DT, FMT, true>(q0.ra, q1.ra, sms, st)
+                      : launch_row_pair1<DT, FMT, false>(q0.ra, q1.ra, sms, st);
+  return q0.layout == FP8_LAYOUT_DUAL ? launch_tile_tma_pair1<DT, FMT, true>(q0, q1, sms, st)
+                                      : launch_tile_tma_pair1<DT, FMT, false>(q0, q1, sms, st);
+}
+
+template <int DT>
+int launch_pair_dt(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
+  return q0.fmt == FP8_E4M3 ? launch_pair_dt_fmt<DT, FP8_E4M3>(q0, q1, sms, st)
+                            : launch_pair_dt_fmt<DT, FP8_E5M2>(q0, q1, sms, st);
+}
+
+// Both calls in one launch when they resolve to the same kernel (ROW with
+// the same alignment, or TMA tiles with the same layout) and neither is
+// empty; otherwise one launch each, in order.
+int quantize_pair_dispatch(QPlan& q0, QPlan& q1, cudaStream_t st) {
+  const int sms = sm_count_current();
+  if (sms <= 0) return FP8_ERR_CUDA;
+  const bool same = q0.kind == q1.kind && q0.dtype == q1.dtype && q0.fmt == q1.fmt && q0.layout == q1.layout &&
+                    (q0.kind == kQTma || (q0.kind == kQRow && q0.aligned == q1.aligned));
+  const bool nonempty = q0.kind == kQRow ? (q0.ra.n > 0 && q1.ra.n > 0) : (q0.ta.ntiles > 0 && q1.ta.ntiles > 0);
+  if (!same || !nonempty) {
+    const int rc = quantize_launch(q0, sms, st);
+    return rc != FP8_OK ? rc : quantize_launch(q1, sms, st);
+  }
+  switch (q0.dtype) {
+    case FP8_IN_BF16: return launch_pair_dt<FP8_IN_BF16>(q0, q1, sms, st);
+    case FP8_IN_FP16: return launch_pair_dt<FP8_IN_FP16>(q0, q1, sms, st);
+    default: return launch_pair_dt<FP8_IN_FP32>(q0, q1, sms, st);
   }
 }
 
@@ -1090,6 +1245,35 @@ extern "C" int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t col
   if (rc != FP8_OK) return rc;
   const RingArgs r{ring.history, ring.idx, ring.scale, ring.scale_inv, ring.scratch};
   return quantize_dispatch(in, dtype, rows, cols, layout, fmt, r, out, out_t, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int fp8_quantize_pair(const fp8_quantize_args* q0, const fp8_quantize_args* q1, fp8_stream_t stream) {
+  if (q0 == nullptr || q1 == nullptr) return FP8_ERR_INVALID_ARG;
+  QPlan p[2];
+  const fp8_quantize_args* qs[2] = {q0, q1};
+  for (int i = 0; i < 2; ++i) {
+    const fp8_quantize_args& q = *qs[i];
+    const fp8_ring& ring = q.ring;
+    if (!ring.history || !ring.idx || !ring.scale || !ring.scale_inv || !ring.scratch) return FP8_ERR_INVALID_ARG;
+    const int rc = check_quantize_args(q.in, q.dtype, q.rows, q.cols, q.layout, q.fmt, q.out, q.out_t, ring.scratch);
+    if (rc != FP8_OK) return rc;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  for (int i = 0; i < 2; ++i) {
+    const fp8_quantize_args& q = *qs[i];
+    const RingArgs r{q.ring.history, q.ring.idx, q.ring.scale, q.ring.scale_inv, q.ring.scratch};
+    const int rc = quantize_plan(q.in, q.dtype, q.rows, q.cols, q.layout, q.fmt, r, q.out, q.out_t, p[i]);
+    if (rc != FP8_OK) return rc;
+  }
+  // One ring for both: two calls in order, as the caller wrote them.
+  const bool shared = q0->ring.scratch == q1->ring.scratch || q0->ring.history == q1->ring.history;
+  if (shared) {
+    const int sms = sm_count_current();
+    if (sms <= 0) return FP8_ERR_CUDA;
+    const int rc = quantize_launch(p[0], sms, st);
+    return rc != FP8_OK ? rc : quantize_launch(p[1], sms, st);
+  }
+  return quantize_pair_dispatch(p[0], p[1], st);
 }
 
 extern "C" int fp8_quantize_local(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,

@@ -88,6 +88,8 @@ def lib():
         L.fp8_ring_fold.restype = i32
         L.fp8_mm_pair.argtypes = [vp, vp, vp, ctypes.c_size_t, vp]
         L.fp8_mm_pair.restype = i32
+        L.fp8_quantize_pair.argtypes = [vp, vp, vp]
+        L.fp8_quantize_pair.restype = i32
         L.fp8_launch_count.argtypes = []
         L.fp8_launch_count.restype = ctypes.c_uint64
         _LIB = L
@@ -186,6 +188,42 @@ def quantize(x, fmt, layout, ring, out=None, out_t=None, stream=None):
                                       _stream(stream, x.get_device()))
     _check(rc, "fp8_quantize")
     return (out if layout in (ROW, DUAL) else None), (out_t if layout in (TRANSPOSED, DUAL) else None)
+
+
+class CQuantArgs(ctypes.Structure):
+    """Mirror of ``fp8_quantize_args``."""
+
+    _fields_ = [("in_", ctypes.c_void_p), ("dtype", ctypes.c_int), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("layout", ctypes.c_int), ("fmt", ctypes.c_int), ("ring", CRing), ("out", ctypes.c_void_p),
+                ("out_t", ctypes.c_void_p)]
+
+
+def quantize_pair(q0, q1, stream=None):
+    """fp8_quantize_pair: two quantize calls (own rings) in one launch, e.g. a linear's X and W.
+
+    q0, q1: dicts of ``quantize`` arguments (x, fmt, layout, ring and
+    optionally out, out_t).  Returns ((out0, out_t0), (out1, out_t1)).
+    """
+    args, res = [], []
+    for q in (q0, q1):
+        x, layout = q["x"], q["layout"]
+        if x.dim() != 2 or not x.is_contiguous():
+            raise ValueError("x must be a contiguous 2-D tensor")
+        rows, cols = x.shape
+        out, out_t = q.get("out"), q.get("out_t")
+        if layout in (ROW, DUAL) and out is None:
+            out = torch.empty((rows, cols), dtype=torch.uint8, device=x.device)
+        if layout in (TRANSPOSED, DUAL) and out_t is None:
+            out_t = torch.empty((cols, rows), dtype=torch.uint8, device=x.device)
+        out = out if layout in (ROW, DUAL) else None
+        out_t = out_t if layout in (TRANSPOSED, DUAL) else None
+        args.append(CQuantArgs(x.data_ptr(), IN_DTYPE[x.dtype], rows, cols, layout, q["fmt"], q["ring"].c(),
+                               _ptr(out), _ptr(out_t)))
+        res.append((out, out_t))
+    rc = (_LIB or lib()).fp8_quantize_pair(ctypes.byref(args[0]), ctypes.byref(args[1]),
+                                           _stream(stream, q0["x"].get_device()))
+    _check(rc, "fp8_quantize_pair")
+    return res[0], res[1]
 
 
 def quantize_local(x, fmt, layout, ring, amax=None, out=None, out_t=None, stream=None):

@@ -138,6 +138,33 @@ int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t
                                 fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);
 
 /*
+ * fp8_quantize_pair -- two fp8_quantize calls (each on its own ring) in one
+ * launch, such as a linear's X and W before its forward GEMM.
+ *
+ * When both resolve to the same kernel (same dtype, fmt and layout; ROW
+ * inputs with the same 16-byte alignment, or T/DUAL inputs with 16-byte rows
+ * on TMA) and neither is empty, one grid is split between them in proportion
+ * to their sizes; each set of blocks has its own amax ticket and folds its
+ * own ring.  Otherwise the two run one after the other on `stream`.  Each
+ * result (codes, ring, scales) is exactly that of the fp8_quantize call with
+ * the same arguments.  If both name the same ring the two calls run in order
+ * (a ring cannot serve two calls at once).
+ *   q0, q1  host structs; each field as the fp8_quantize argument of that name.
+ * Errors as fp8_quantize (the first call's checked first).
+ * The pages have no counterpart (a B200 scheduling addition).
+ */
+typedef struct {
+  const void* in;
+  int dtype;
+  int64_t rows, cols;
+  int layout, fmt;
+  fp8_ring ring;
+  uint8_t* out;
+  uint8_t* out_t;
+} fp8_quantize_args;
+int fp8_quantize_pair(const fp8_quantize_args* q0, const fp8_quantize_args* q1, fp8_stream_t stream);
+
+/*
  * fp8_quantize_local / fp8_ring_fold -- delayed scaling of a tensor sharded
  * across data-parallel ranks: one scale for all shards.
  *

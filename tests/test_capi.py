@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
         ["fp8_quantize", "fp8_mm", "fp8_status_string", "fp8_device_error", "fp8_device_info",
          "fp8_quantize_static_scratch", "fp8_quantize_current", "fp8_bias_grad", "fp8_linear_forward",
          "fp8_linear_backward", "fp8_mm_ws", "fp8_mm_workspace_bytes", "fp8_quantize_local", "fp8_ring_fold",
-         "fp8_mm_pair", "fp8_launch_count"])
+         "fp8_mm_pair", "fp8_launch_count", "fp8_quantize_pair"])
 
 
 def test_library_exports_every_declared_symbol(L):

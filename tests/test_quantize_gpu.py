@@ -141,3 +141,62 @@ def test_nan_inputs_do_not_reach_amax(dtype, layout):
         g = out_t.cpu().numpy()
         assert np.array_equal(g[~nan.T], r_out_t[~nan.T])
     assert_ring_equal(ring, r_ring)
+
+
+# fp8_quantize_pair: two quantize calls (own rings) in one launch.  Each case
+# runs 3 delayed steps and must equal the two separate fp8_quantize calls bit
+# for bit (codes, rings).  Cases: paired TMA tiles (dual, transposed), paired
+# ROW (aligned; element-offset bases), and the sequential fallbacks (different
+# kernels, different formats, an empty side).
+QPAIR = [
+    (((8192, 1536), "bf16", 0, False), ((1536, 1536), "bf16", 0, False), ops.DUAL),
+    (((2048, 1536), "fp32", 1, False), ((130, 64), "fp32", 1, False), ops.TRANSPOSED),
+    (((8192, 1536), "bf16", 0, False), ((4096, 1536), "bf16", 0, False), ops.ROW),
+    (((1000, 1537), "bf16", 0, True), ((7, 33), "bf16", 0, True), ops.ROW),
+    (((2048, 1537), "bf16", 0, False), ((256, 512), "bf16", 0, False), ops.DUAL),
+    (((256, 512), "bf16", 0, False), ((256, 512), "bf16", 1, False), ops.DUAL),
+    (((0, 9), "bf16", 0, False), ((64, 64), "bf16", 0, False), ops.DUAL),
+]
+
+
+def _dev(x, misalign):
+    if not misalign:
+        return x.cuda()
+    flat = torch.empty(x.numel() + 1, dtype=x.dtype, device="cuda")
+    flat[1:].copy_(x.reshape(-1))
+    return flat[1:].view(x.shape)
+
+
+@pytest.mark.parametrize("s0,s1,layout", QPAIR)
+def test_quantize_pair_equals_two_calls(s0, s1, layout):
+    rings = [ops.Ring(), ops.Ring()]
+    refs = [ops.Ring(), ops.Ring()]
+    for step in range(3):
+        qs, expect = [], []
+        for i, ((rows, cols), dt, fmt, mis) in enumerate((s0, s1)):
+            x = _dev(S.quant_sweep_input(rows, cols, dt, [1.0, 1e3, 1e-3][step], seed=600 + 10 * step + i), mis)
+            qs.append(dict(x=x, fmt=fmt, layout=layout, ring=rings[i]))
+            expect.append(ops.quantize(x, fmt, layout, refs[i]))
+        got = ops.quantize_pair(qs[0], qs[1])
+        torch.cuda.synchronize()
+        for (o, t), (eo, et) in zip(got, expect):
+            for a, b in ((o, eo), (t, et)):
+                assert (a is None) == (b is None)
+                if a is not None:
+                    assert torch.equal(a, b)
+        for r, e in zip(rings, refs):
+            assert torch.equal(r.buf, e.buf)
+
+
+def test_quantize_pair_with_one_ring_runs_in_order():
+    """Naming the same ring twice is two calls in order (the second sees the
+    scale the first published)."""
+    ring, ref = ops.Ring(), ops.Ring()
+    x0 = S.quant_sweep_input(512, 256, "bf16", 1.0, seed=1).cuda()
+    x1 = S.quant_sweep_input(512, 256, "bf16", 1e3, seed=2).cuda()
+    (o0, _), (o1, _) = ops.quantize_pair(dict(x=x0, fmt=ops.E4M3, layout=ops.ROW, ring=ring),
+                                         dict(x=x1, fmt=ops.E4M3, layout=ops.ROW, ring=ring))
+    e0, _ = ops.quantize(x0, ops.E4M3, ops.ROW, ref)
+    e1, _ = ops.quantize(x1, ops.E4M3, ops.ROW, ref)
+    torch.cuda.synchronize()
+    assert torch.equal(o0, e0) and torch.equal(o1, e1) and torch.equal(ring.buf, ref.buf)

@@ -515,41 +515,78 @@ def main():
     flops = gemm_flops(M)
     value = world * flops / (ms * 1e-3) / 1e12
 
-    # End to end through the C ABI: pinned host X and G copied in, Y, dX, dW copied out, every step.
+    # End to end through the C ABI: every step copies its X and G in from pinned
+    # host memory and its Y, dX and dW out to pinned host memory.  As a
+    # training loop would, it overlaps step i's compute with the copy-in of
+    # step i+1 and the copy-out of step i-1 (three streams; inputs, outputs
+    # and host outputs double-buffered; events order every reuse).
     e2e = None
     if not args.no_e2e:
         host_in = [[(x.cpu().pin_memory(), g.cpu().pin_memory()) for x, g in L.inputs] for L in lins]
-        host_out = [(torch.empty(L.y.shape, dtype=L.y.dtype).pin_memory(),
-                     torch.empty(L.dx.shape, dtype=L.dx.dtype).pin_memory(),
-                     torch.empty(L.dw.shape, dtype=L.dw.dtype).pin_memory()) for L in lins]
+        outs = [[(L.y, L.dx, L.dw), (torch.empty_like(L.y), torch.empty_like(L.dx), torch.empty_like(L.dw))]
+                for L in lins]
+        host_out = [[tuple(torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in o) for o in lo] for lo in outs]
         h2d = sum(x.numel() * x.element_size() + g.numel() * g.element_size() for x, g in (h[0] for h in host_in))
-        d2h = sum(sum(t.numel() * t.element_size() for t in ho) for ho in host_out)
+        d2h = sum(sum(t.numel() * t.element_size() for t in lo[0]) for lo in outs)
         steps_e2e = max(3, min(200, args.steps // 5))
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        ev = lambda: torch.cuda.Event()  # noqa: E731
+        in_ready = [ev(), ev()]      # inputs of buffer set b copied in
+        in_free = [ev(), ev()]       # compute done reading buffer set b
+        out_ready = [ev(), ev()]     # outputs of buffer set b computed
+        out_free = [ev(), ev()]      # outputs of buffer set b copied out
+        for e in in_free + out_free:
+            e.record(st)
         if pg:
             pg.barrier()
         torch.cuda.synchronize()
         a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def copy_in(i):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                s_in.wait_event(in_free[b])
+                for L, hin in zip(lins, host_in):
+                    hx, hg = hin[i % len(hin)]
+                    x, g = L.inputs[b]
+                    x.copy_(hx, non_blocking=True)
+                    g.copy_(hg, non_blocking=True)
+                in_ready[b].record(s_in)
+
         a0.record(st)
+        copy_in(0)
         for i in range(steps_e2e):
-            for L, hin, hout in zip(lins, host_in, host_out):
-                hx, hg = hin[i % len(hin)]
-                x, g = L.inputs[i % len(L.inputs)]
-                x.copy_(hx, non_blocking=True)
-                g.copy_(hg, non_blocking=True)
+            b = i % 2
+            if i + 1 < steps_e2e:
+                copy_in(i + 1)
+            st.wait_event(in_ready[b])
+            st.wait_event(out_free[b])
+            for L, lo in zip(lins, outs):
+                x, g = L.inputs[b]
+                L.y, L.dx, L.dw = lo[b]
                 L.quantize(ops, x, g)
                 L.gemms(ops)
-                hout[0].copy_(L.y, non_blocking=True)
-                hout[1].copy_(L.dx, non_blocking=True)
-                hout[2].copy_(L.dw, non_blocking=True)
+            in_free[b].record(st)
+            out_ready[b].record(st)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(out_ready[b])
+                for lo, ho in zip(outs, host_out):
+                    for t, h in zip(lo[b], ho[b]):
+                        h.copy_(t, non_blocking=True)
+                out_free[b].record(s_out)
+        st.wait_stream(s_out)
         a1.record(st)
         torch.cuda.synchronize()
+        for L, lo in zip(lins, outs):
+            L.y, L.dx, L.dw = lo[0]
         ms_e2e = a0.elapsed_time(a1) / steps_e2e
         if pg:
             t = torch.tensor([ms_e2e], device="cuda")
             pg.all_reduce(t, op=pg.ReduceOp.MAX)
             ms_e2e = float(t.item())
         e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s", "ms_per_step": ms_e2e,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "overlap": "copy-in of step i+1 and copy-out of step i-1 run beside step i's kernels"}
 
     peaks = {}
     try:

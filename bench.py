@@ -340,6 +340,27 @@ def _kernel_ms(fn, torch, iters, flush=None):
     return t / iters
 
 
+def pair_sweep(spec, args, torch, ops, S):
+    """Time two 2-D GEMMs ("MxNxK[:lay]+MxNxK[:lay]") as one fp8_mm_pair call."""
+    probs, fl = [], 0.0
+    for i, part in enumerate(spec.split("+")):
+        dims, _, lay = part.partition(":")
+        M, N, K = (int(t) for t in dims.split("x"))
+        a_mn, b_mn = lay == "mn", lay in ("mn", "bmn")
+        a = S.fp8_codes((K, M) if a_mn else (M, K), seed=1 + 2 * i).cuda()
+        b = S.fp8_codes((K, N) if b_mn else (N, K), seed=2 + 2 * i).cuda()
+        one = torch.ones(1, device="cuda")
+        out = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        probs.append(dict(a=a, b=b, sinv_a=one, sinv_b=one, out=out, a_mn_major=a_mn, b_mn_major=b_mn))
+        fl += 2.0 * M * N * K
+    fn = lambda: ops.mm_pair(probs[0], probs[1])  # noqa: E731
+    for _ in range(3):
+        fn()
+    ms = _kernel_ms(fn, torch, args.iters)
+    print(json.dumps({"kernel": "mm_fp8_pair", "pair": spec, "us": round(ms * 1e3, 2),
+                      "tflops": round(fl / ms / 1e9, 1)}))
+
+
 def sweep(args):
     import torch
 
@@ -352,9 +373,13 @@ def sweep(args):
     if args.sweep == "gemm":
         # A shape is [B x]M x N x K, optionally followed by ":bmn" (B read
         # MN-major) or ":mn" (A and B read MN-major), the backward layouts.
+        # Two 2-D shapes joined by "+" are timed as one fp8_mm_pair call.
         shapes = []
         for spec in (args.shapes.split(",") if args.shapes else
                      ["x".join(map(str, s)) for s in GEMM_SHAPES]):
+            if "+" in spec:
+                pair_sweep(spec, args, torch, ops, S)
+                continue
             dims, _, lay = spec.partition(":")
             v = tuple(int(t) for t in dims.split("x"))
             shapes.append(((1,) + v if len(v) == 3 else v, lay or "nt"))

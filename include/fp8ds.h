@@ -7,8 +7,16 @@
  *                 held in a delayed-scaling ring, reduce amax over the raw
  *                 values, and fold that amax into the ring in the same kernel.
  *   fp8_mm        Y = bf16(sinv_a * sinv_b * A.B^T + bias), A and B FP8 with K
- *                 contiguous ("NT"), fp32 accumulation, optional fp32 bias,
- *                 optional batch with stride-0 broadcast.
+ *                 contiguous ("NT") or MN-major, fp32 accumulation, optional
+ *                 fp32 bias, optional batch with stride-0 broadcast.
+ *
+ * Around them: fp8_quantize_pair / fp8_mm_pair (two calls in one launch),
+ * fp8_mm_ws (stream-K tail through a caller workspace), fp8_quantize_current
+ * (current scaling), fp8_quantize_local + fp8_ring_fold (data-parallel
+ * delayed scaling), fp8_bias_grad and fp8_linear_forward / _backward (the
+ * linear composites), fp8_quantize_static_scratch (no caller scratch), and
+ * the utilities fp8_status_string, fp8_device_error, fp8_device_info and
+ * fp8_launch_count.
  *
  * Sources: the AstrAI commit-log pages "AstrAI commits, branch main,
  * tests/extension" (ring commit, quantize split commit, snapshot commit,

@@ -82,6 +82,35 @@ def test_saturation_and_specials():
             _run_and_compare(vals, fmt, layout, ring)
 
 
+def _all_16bit_patterns(dtype, with_inf=True):
+    """Every non-NaN bf16 or fp16 bit pattern (both zeros, subnormals, infinities
+    unless left out), zero-padded to [rows, 256] so the aligned kernels run."""
+    bits = torch.from_numpy(np.arange(1 << 16, dtype=np.uint16).view(np.int16).copy())
+    x = bits.view(torch.bfloat16 if dtype == "bf16" else torch.float16)
+    xf = x.float()
+    x = x[~torch.isnan(xf) & (torch.isfinite(xf) | with_inf)]
+    pad = (-x.numel()) % 256
+    return torch.cat([x, torch.zeros(pad, dtype=x.dtype)]).view(-1, 256)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("layout", LAYOUTS)
+def test_every_16bit_input_pattern(dtype, fmt, layout):
+    """All 16-bit inputs at scale 1 (subnormal, normal, saturating and infinite
+    inputs), at two scales that are not powers of two (the scaled product rounds
+    in float32 before the cast), then two delayed steps on the finite patterns:
+    the second uses the scale the first folded from the largest finite value."""
+    x = _all_16bit_patterns(dtype)
+    for s in (1.0, 0.3, 3.0 * 2.0 ** -7):
+        _run_and_compare(x, fmt, layout, ops.Ring(scale=s))
+    ring = ops.Ring()
+    finite = _all_16bit_patterns(dtype, with_inf=False)
+    for _ in range(2):
+        _run_and_compare(finite, fmt, layout, ring)
+    assert ring.state()[2] != 1.0
+
+
 # Full sizes of the quantize bandwidth sweep, in the launch configuration the
 # bench times; bytes compared on sampled rows, amax / ring / scales in full.
 FULL = [(128, 1536), (2048, 1536), (8192, 1536), (16384, 4096), (2048, 1537), (8192, 1537)]

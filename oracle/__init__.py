@@ -16,7 +16,9 @@ Sources (the AstrAI commit-log pages):
   next scale), the quantize split commit (E4M3/E5M2 fmt enum, bf16/fp16/fp32
   inputs), the snapshot commit (the GEMM dequantises with the scale that
   quantize used), the bias-fusion commit (fp32 bias added before one bf16
-  rounding) and the batched commit (stride-0 broadcast).
+  rounding), the batched commit (stride-0 broadcast), the bias_scale commit
+  (FP8 bias storage dequantised in the epilogue) and the FP8-in/FP8-out
+  GEMM commit.
 * "AstrAI commit 69f35c46 csrc/kernels/fp8_mm.cu" -- amax is taken over the
   raw, unscaled values.
 * "AstrAI commit 5244f1a8 (te-style scaled fp8 training)" on the same page
@@ -31,7 +33,9 @@ Modules:
   fp8_formats -- decode table and encoder (RNE + saturation) per format.
   recipe      -- amax, quantize in row/transposed/dual layout, ring fold,
                  current scaling, and the shard cast of data-parallel scaling.
-  gemm        -- fp64 scaled GEMM, |a.b| sums and the acceptance bound.
+  gemm        -- fp64 scaled GEMM, |a.b| sums and the acceptance bound;
+                 FP8 bias dequantisation and the acceptance interval of
+                 FP8 output codes and of the output amax.
   bias_grad   -- column sums of the output gradient (the bias gradient).
 
 Parity status: every function is pinned by ``tests/test_oracle_*.py``

@@ -91,3 +91,67 @@ def check(y, ref, S):
     b = bound(ref, S)
     ratio = float(np.max(err / b)) if err.size else 0.0
     return bool(np.all(err <= b)), ratio
+
+
+# ---- FP8 bias storage and FP8 output (epilogue variants) -------------------
+#
+# "AstrAI commits, branch main, tests/extension" page: the bias_scale commit
+# (FP8Params.bias becomes untyped with a bias_scale slot: without a scale the
+# bias is used as stored, with one it is FP8 storage dequantised in the
+# epilogue after the operand scaling and before any output quantisation) and
+# the FP8-in/FP8-out GEMM commit (fp8_mm_prequant_fp8).  The pages fix no
+# formula for either; the readings here are the plainest ones that match the
+# rest of the recipe:
+#   bias value  = fp32(decode(code) * bias_scale)        (one float32 multiply)
+#   y           = sinv_a * sinv_b * sum_k a.b + bias     (the float32 epilogue value)
+#   output code = encode(fp32(y * s)), s = out_ring.scale (the output tensor's
+#                 delayed scale, one float32 multiply, saturating RNE)
+#   out_ring    folds amax = max |y| over the output (NaN ignored) exactly as
+#                 a quantize call folds the amax of its input.
+
+
+def bias_from_fp8(codes, fmt, bias_scale):
+    """float32 [N] bias of FP8 bias storage: fp32(decode(code) * bias_scale)."""
+    vals = F.decode(np.asarray(codes, dtype=np.uint8), fmt).astype(np.float32)  # exact: FP8 values fit in float32
+    return np.multiply(vals, np.float32(bias_scale), dtype=np.float32)
+
+
+def bound_f32(ref, S):
+    """Allowed |y - ref| for the float32 epilogue value y itself (no bf16 rounding):
+    the accumulation allowance 2^-20 * S plus one float32 ulp of ref for the
+    epilogue's fused multiply-add, plus the smallest float32 subnormal."""
+    ref = np.abs(np.asarray(ref, dtype=np.float64))
+    return np.ldexp(np.asarray(S, dtype=np.float64), -20) + np.ldexp(ref, -23) + 2.0 ** -149
+
+
+def out8_code_range(ref, S, scale, fmt):
+    """(lo, hi) uint8 codes: every float32 y within ``bound_f32`` of ``ref`` has
+    encode(fp32(y * scale)) between the two (both encode steps are monotone in
+    y, and a float32 y >= lo_end is >= fp32(lo_end)).  Where lo == hi the code
+    is fixed exactly."""
+    b = bound_f32(ref, S)
+    lo_end = np.asarray(ref, dtype=np.float64) - b
+    hi_end = np.asarray(ref, dtype=np.float64) + b
+    with np.errstate(over="ignore"):
+        lo32 = lo_end.astype(np.float32)
+        hi32 = hi_end.astype(np.float32)
+    s = np.float32(scale)
+    with np.errstate(over="ignore"):
+        lo = F.encode(np.multiply(lo32, s, dtype=np.float32), fmt)
+        hi = F.encode(np.multiply(hi32, s, dtype=np.float32), fmt)
+    return lo, hi
+
+
+def codes_within(codes, lo, hi, fmt):
+    """Boolean array: decode(lo) <= decode(codes) <= decode(hi), element-wise."""
+    v = F.decode(np.asarray(codes, dtype=np.uint8), fmt)
+    return (F.decode(lo, fmt) <= v) & (v <= F.decode(hi, fmt))
+
+
+def amax_range(ref, S):
+    """(amax_exact, tolerance) of max |y| over the output: the exact max |ref|
+    and the largest per-element ``bound_f32`` (0, 0 for an empty output)."""
+    ref = np.asarray(ref, dtype=np.float64)
+    if ref.size == 0:
+        return 0.0, 0.0
+    return float(np.max(np.abs(ref))), float(np.max(bound_f32(ref, S)))

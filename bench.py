@@ -60,6 +60,8 @@ def parse():
                     help="warm up, run exactly one step inside the NVTX range fp8_profile_step, exit (for ncu)")
     ap.add_argument("--shapes", default=None, help="sweep subset, e.g. 8192x8192x8192,64x8192x2048")
     ap.add_argument("--ws", action="store_true", help="gemm sweep: also time each shape with a stream-K workspace")
+    ap.add_argument("--mm-out", default="bf16",
+                    help="gemm sweep: output kinds to time, of bf16,e4m3,e5m2 (FP8 outputs fold an output ring)")
     ap.add_argument("--qdtypes", default="bf16,fp32", help="quantize sweep input dtypes")
     ap.add_argument("--qlayouts", default="row,T,dual", help="quantize sweep layouts")
     return ap.parse_args()
@@ -393,17 +395,28 @@ def sweep(args):
             out = torch.empty((bt, M, N), dtype=torch.bfloat16, device="cuda")
             need = ops.mm_workspace_bytes(M, N, K, batch=bt, a_mn_major=a_mn, b_mn_major=b_mn)
             ws = torch.zeros(max(need, 256), dtype=torch.uint8, device="cuda") if args.ws else None
+            out8 = torch.empty((bt, M, N), dtype=torch.uint8, device="cuda")
+            ring = ops.Ring()
+            kinds = {"bf16": None, "e4m3": ops.E4M3, "e5m2": ops.E5M2}
             for use_ws in ((False, True) if args.ws and need > 0 else (False,)):
-                for with_bias in (False, True):
-                    fn = lambda: ops.mm(a, b, one, one, bias if with_bias else None, out=out,  # noqa: E731
-                                        a_mn_major=a_mn, b_mn_major=b_mn, workspace=ws if use_ws else None)
-                    for _ in range(3):
-                        fn()
-                    ms = _kernel_ms(fn, torch, args.iters)
-                    fl = 2.0 * bt * M * N * K
-                    print(json.dumps({"kernel": "mm_fp8", "batch": bt, "M": M, "N": N, "K": K, "layout": lay,
-                                      "bias": with_bias, "stream_k_ws": need if use_ws else 0,
-                                      "us": round(ms * 1e3, 2), "tflops": round(fl / ms / 1e9, 1)}))
+                for kind in args.mm_out.split(","):
+                    for with_bias in (False, True):
+                        bb = bias if with_bias else None
+                        w = ws if use_ws else None
+                        if kinds[kind] is None:
+                            fn = lambda: ops.mm(a, b, one, one, bb, out=out,  # noqa: E731
+                                                a_mn_major=a_mn, b_mn_major=b_mn, workspace=w)
+                        else:
+                            fn = lambda: ops.mm_ex(a, b, one, one, bias=bb, out_fmt=kinds[kind],  # noqa: E731
+                                                   out_ring=ring, out=out8, a_mn_major=a_mn, b_mn_major=b_mn,
+                                                   workspace=w)
+                        for _ in range(3):
+                            fn()
+                        ms = _kernel_ms(fn, torch, args.iters)
+                        fl = 2.0 * bt * M * N * K
+                        print(json.dumps({"kernel": "mm_fp8", "batch": bt, "M": M, "N": N, "K": K, "layout": lay,
+                                          "out": kind, "bias": with_bias, "stream_k_ws": need if use_ws else 0,
+                                          "us": round(ms * 1e3, 2), "tflops": round(fl / ms / 1e9, 1)}))
     else:
         want = [tuple(int(v) for v in s.split("x")) for s in args.shapes.split(",")] if args.shapes else None
         for rows, cols in (QUANT_SHAPES if not want else want):

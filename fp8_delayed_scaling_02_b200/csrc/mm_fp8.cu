@@ -30,6 +30,8 @@
 //     run replicas.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -37,6 +39,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "fp8_ring.cuh"
 
 namespace fp8ds {
 namespace {
@@ -63,7 +66,7 @@ struct Cfg {
   static constexpr int kBarOffset = kStagingOffset + kEpiWarps * 2 * kStagingBytes;
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(2 * kStages + 5 <= 28, "barrier area");
+  static_assert((2 * kStages + 5) * 8 + 16 + 4 * kEpiWarps <= 256, "barrier area: barriers, TMEM slot, abort, amax");
 };
 
 struct MmParams {
@@ -94,7 +97,65 @@ struct MmParams {
   int bias_vec;      // bias is 16-byte aligned
   uint32_t idesc;
   uint32_t* err;
+  // Epilogue variants (kernel template EPI): an FP8 bias, dequantised as
+  // fp32(code * *bias_scale), and FP8 output codes of fp32(y * *r_scale) with
+  // max |y| folded into the output's ring by the CTA that finishes last.
+  const uint8_t* bias8;
+  const float* bias_scale;
+  int bias_fmt;
+  int out_fmt;
+  uint8_t* out8;
+  int out8_vec;      // code rows are 16-byte aligned: codes leave through TMA stores
+  float* r_history;
+  int32_t* r_idx;
+  float* r_scale;
+  float* r_scale_inv;
+  uint32_t* r_scratch;  // [0] amax bits, [1] CTA ticket; zero between calls
 };
+
+constexpr int kEpiOut8 = 1;   // EPI bit: FP8 output codes + output ring fold
+constexpr int kEpiBias8 = 2;  // EPI bit: FP8 bias codes
+
+// Value of one FP8 code (exact in fp32; NaN codes give NaN).
+__device__ __forceinline__ float fp8_value(uint8_t c, int fmt) {
+  const __half_raw h = __nv_cvt_fp8_to_halfraw(c, fmt == FP8_E5M2 ? __NV_E5M2 : __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// Dequantised FP8 bias of columns n .. n+3, 0 beyond N.
+__device__ __forceinline__ float4 bias8_4(const MmParams& p, int n, float bsc) {
+  float e[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) e[q] = n + q < p.N ? __fmul_rn(fp8_value(__ldg(p.bias8 + n + q), p.bias_fmt), bsc) : 0.f;
+  return make_float4(e[0], e[1], e[2], e[3]);
+}
+
+// FP8 output: this CTA's max |y| (per epilogue warp in amax_s) joins the
+// ring's scratch word; the CTA that draws the last of gridDim.x tickets takes
+// the grid's amax, clears the scratch words and commits the ring.  The
+// acq_rel ticket orders each CTA's amax before its increment and gives the
+// last CTA every other CTA's.  Run by one thread after the CTA's epilogue.
+__device__ __noinline__ void out8_ticket_fold(const MmParams& p, const float* amax_s) {
+  float m = 0.0f;
+#pragma unroll
+  for (int w = 0; w < kEpiWarps; ++w) m = fmaxf(m, amax_s[w]);
+  if (m > 0.0f)
+    asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p.r_scratch), "r"(__float_as_uint(m)) : "memory");
+  unsigned t;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.r_scratch + 1) : "memory");
+  if (t != gridDim.x - 1) return;
+  uint32_t bits;
+  asm volatile("atom.relaxed.gpu.global.exch.b32 %0, [%1], 0;" : "=r"(bits) : "l"(p.r_scratch) : "memory");
+  asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(p.r_scratch + 1) : "memory");
+  float hist[kHistoryLen];
+#pragma unroll
+  for (int i = 0; i < kHistoryLen; ++i) hist[i] = p.r_history[i];
+  const float a = __uint_as_float(bits);
+  if (p.out_fmt == FP8_E5M2)
+    ring_commit<FP8_E5M2>(a, hist, *p.r_idx, p.r_history, p.r_idx, p.r_scale, p.r_scale_inv, *p.r_scale);
+  else
+    ring_commit<FP8_E4M3>(a, hist, *p.r_idx, p.r_history, p.r_idx, p.r_scale, p.r_scale_inv, *p.r_scale);
+}
 
 // ---- PTX wrappers (written from the PTX ISA description) -----------------------
 
@@ -363,10 +424,12 @@ __device__ __forceinline__ void decode_tile(const MmParams& p, int t, int& b, in
 
 // One CTA's (pair's) whole life: problem `p` with maps tmA / tmB / tmC, as
 // CTA (pair) `cta` of the `ctas` that work on this problem.
-template <int BN, int PAIR>
+template <int BN, int PAIR, int EPI>
 __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMap* tmB, const CUtensorMap* tmC,
                                         const MmParams& p, const int cta, const int ctas) {
   using C = Cfg<BN, PAIR>;
+  constexpr bool kOut8 = (EPI & kEpiOut8) != 0;
+  constexpr bool kBias8 = (EPI & kEpiBias8) != 0;
   constexpr int kTileM = kBM * PAIR;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled tiles (the same offset in both CTAs of a pair).
@@ -377,6 +440,7 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
   // bars[0, S) full, [S, 2S) empty, [2S, 2S+2) tmem_full, [2S+2, 2S+4) tmem_empty, [2S+4] mma_done
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * C::kStages + 5);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* amax_s = reinterpret_cast<float*>(tmem_slot + 4);  // FP8 output: max |y| per epilogue warp
   const uint32_t bar0 = smem_u32(bars);
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
@@ -553,6 +617,9 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
     const int half = ew >> 2;
     constexpr int kHalfCols = BN / 2;
     const float sab = __fmul_rn(*p.sinv_a, *p.sinv_b);
+    const float bsc = kBias8 ? *p.bias_scale : 0.0f;  // FP8 bias dequantisation factor
+    const float s_out = kOut8 ? *p.r_scale : 0.0f;    // FP8 output: the output ring's scale
+    float amax = 0.0f;                                 // FP8 output: max |y| of this lane's elements
     const uint32_t stage0 = sbase + C::kStagingOffset + uint32_t(ew) * 2u * kStagingBytes;
     int buf = 0;
     int i = 0;
@@ -604,6 +671,25 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
       const int m0 = mt * kTileM + int(rank) * kBM + quad * 32;
       const uint32_t tbase = tmem_base + (uint32_t(quad * 32) << 16) + uint32_t(acc * BN + half * kHalfCols);
       const int nbase = nt * BN + half * kHalfCols;
+      // This warp's bias, four columns per lane (lane l: nbase + 4l .. 4l+3),
+      // read once per tile; emit() takes a chunk's 32 values from 8 lanes by
+      // shuffle.  (Broadcast loads of the same values in every chunk cost a
+      // K=1536 GEMM about 28% of its time.)
+      const bool has_bias = kBias8 || p.bias != nullptr;
+      float4 bias_l = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (has_bias && lane < kHalfCols / 4) {
+        const int c4 = nbase + 4 * lane;
+        if constexpr (kBias8) {
+          bias_l = bias8_4(p, c4, bsc);
+        } else if (p.bias_vec && c4 + 3 < p.N) {
+          bias_l = __ldg(reinterpret_cast<const float4*>(p.bias + c4));
+        } else {
+          bias_l.x = c4 < p.N ? __ldg(p.bias + c4) : 0.f;
+          bias_l.y = c4 + 1 < p.N ? __ldg(p.bias + c4 + 1) : 0.f;
+          bias_l.z = c4 + 2 < p.N ? __ldg(p.bias + c4 + 2) : 0.f;
+          bias_l.w = c4 + 3 < p.N ? __ldg(p.bias + c4 + 3) : 0.f;
+        }
+      }
       const uint32_t release_bar = PAIR == 1 ? tempty_bar(acc) : mapa_shared(tempty_bar(acc), 0);
       bool released = false;
       auto release = [&]() {
@@ -618,29 +704,72 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
       auto emit = [&](int n0, const uint32_t(&v)[32]) {
         if (m0 >= p.M) return;  // warp-uniform: rows beyond M (pair peer of a short last tile)
         const bool full = n0 + 32 <= p.N;
-        uint32_t packed[16];
+        const bool row_ok = m0 + lane < p.M;
+        uint32_t packed[16];  // bf16 pairs, or (FP8 output) code quads in [0, 8)
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-          if (p.bias != nullptr) {
-            if (full && p.bias_vec) {
-              bv = __ldg(reinterpret_cast<const float4*>(p.bias + n0) + j);
-            } else {
-              const int nn = n0 + 4 * j;
-              bv.x = nn < p.N ? __ldg(p.bias + nn) : 0.f;
-              bv.y = nn + 1 < p.N ? __ldg(p.bias + nn + 1) : 0.f;
-              bv.z = nn + 2 < p.N ? __ldg(p.bias + nn + 2) : 0.f;
-              bv.w = nn + 3 < p.N ? __ldg(p.bias + nn + 3) : 0.f;
-            }
+          if (has_bias) {  // warp-uniform
+            const int src = ((n0 - nbase) >> 5) * 8 + j;
+            bv.x = __shfl_sync(0xFFFFFFFFu, bias_l.x, src);
+            bv.y = __shfl_sync(0xFFFFFFFFu, bias_l.y, src);
+            bv.z = __shfl_sync(0xFFFFFFFFu, bias_l.z, src);
+            bv.w = __shfl_sync(0xFFFFFFFFu, bias_l.w, src);
           }
           const float y0 = fmaf(__uint_as_float(v[4 * j + 0]), sab, bv.x);
           const float y1 = fmaf(__uint_as_float(v[4 * j + 1]), sab, bv.y);
           const float y2 = fmaf(__uint_as_float(v[4 * j + 2]), sab, bv.z);
           const float y3 = fmaf(__uint_as_float(v[4 * j + 3]), sab, bv.w);
-          const __nv_bfloat162 h01 = __floats2bfloat162_rn(y0, y1);
-          const __nv_bfloat162 h23 = __floats2bfloat162_rn(y2, y3);
-          packed[2 * j] = *reinterpret_cast<const uint32_t*>(&h01);
-          packed[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+          if constexpr (kOut8) {
+            // amax over this lane's in-range elements (NaN ignored), then the
+            // codes of y * s_out.
+            if (row_ok) {
+              const int nn = n0 + 4 * j;
+              amax = fmaxf(amax, nn < p.N ? fabsf(y0) : 0.f);
+              amax = fmaxf(amax, nn + 1 < p.N ? fabsf(y1) : 0.f);
+              amax = fmaxf(amax, nn + 2 < p.N ? fabsf(y2) : 0.f);
+              amax = fmaxf(amax, nn + 3 < p.N ? fabsf(y3) : 0.f);
+            }
+            packed[j] = p.out_fmt == FP8_E5M2 ? cvt4<FP8_E5M2>(y0, y1, y2, y3, s_out)
+                                              : cvt4<FP8_E4M3>(y0, y1, y2, y3, s_out);
+          } else {
+            const __nv_bfloat162 h01 = __floats2bfloat162_rn(y0, y1);
+            const __nv_bfloat162 h23 = __floats2bfloat162_rn(y2, y3);
+            packed[2 * j] = *reinterpret_cast<const uint32_t*>(&h01);
+            packed[2 * j + 1] = *reinterpret_cast<const uint32_t*>(&h23);
+          }
+        }
+        if constexpr (kOut8) {
+          if (p.tma_store) {
+            // 32 x 32 codes through a TMA store (clipped to M and N) from the
+            // first 1 KB of a staging buffer, 32B swizzle: 16-byte unit u of
+            // row r at unit u ^ ((r >> 2) & 1), conflict-free for the warp.
+            const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
+            if (lane == 0) bulk_wait_read_le1();
+            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const uint32_t addr = sbuf + uint32_t(lane) * 32u + uint32_t((u ^ ((lane >> 2) & 1)) * 16);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[4 * u]),
+                           "r"(packed[4 * u + 1]), "r"(packed[4 * u + 2]), "r"(packed[4 * u + 3])
+                           : "memory");
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(tmC, sbuf, n0, m0, b);
+              bulk_commit();
+            }
+            buf ^= 1;
+            return;
+          }
+          // Rows not 16-byte aligned: guarded byte stores of this lane's row.
+          if (!row_ok) return;
+          uint8_t* o = p.out8 + int64_t(b) * p.c_stride + int64_t(m0 + lane) * p.N + n0;
+#pragma unroll 4
+          for (int k = 0; k < 32; ++k)
+            if (n0 + k < p.N) o[k] = uint8_t(packed[k >> 2] >> (8 * (k & 3)));
+          return;
         }
         const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
         // The buffer's previous TMA store has read it (checked after the math,
@@ -758,12 +887,20 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
         }
       }
     }
+    if constexpr (kOut8) {
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      if (lane == 0) amax_s[ew] = amax;
+    }
     if (p.tma_store && lane == 0) bulk_wait_all();
     __syncwarp();
   }
 
   tc_fence_before();
   __syncthreads();
+  if constexpr (kOut8) {
+    if (threadIdx.x == 0) out8_ticket_fold(p, amax_s);
+  }
   // A pair leaves together: the leader's MMAs read the peer's shared memory
   // and write the peer's TMEM until done_bar fired.
   if constexpr (PAIR == 2) cluster_sync();
@@ -771,11 +908,11 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
   if (warp == 1) tmem_dealloc_g<PAIR>(tmem_base, C::kTmemCols);
 }
 
-template <int BN, int PAIR>
+template <int BN, int PAIR, int EPI>
 __global__ void __launch_bounds__(kThreadsMM, 1)
     mm_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmC, const __grid_constant__ MmParams p) {
-  mm_body<BN, PAIR>(&tmA, &tmB, &tmC, p, int(blockIdx.x) / PAIR, int(gridDim.x) / PAIR);
+  mm_body<BN, PAIR, EPI>(&tmA, &tmB, &tmC, p, int(blockIdx.x) / PAIR, int(gridDim.x) / PAIR);
 }
 
 // Two independent GEMMs in one persistent launch (the dX and dW GEMMs of a
@@ -789,21 +926,59 @@ __global__ void __launch_bounds__(kThreadsMM, 1)
                        const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                        const __grid_constant__ CUtensorMap tmC1, const __grid_constant__ MmParams p1, const int split) {
   const int g = int(blockIdx.x) / PAIR;
-  if (g < split) mm_body<BN, PAIR>(&tmA0, &tmB0, &tmC0, p0, g, split);
-  else mm_body<BN, PAIR>(&tmA1, &tmB1, &tmC1, p1, g - split, int(gridDim.x) / PAIR - split);
+  if (g < split) mm_body<BN, PAIR, 0>(&tmA0, &tmB0, &tmC0, p0, g, split);
+  else mm_body<BN, PAIR, 0>(&tmA1, &tmB1, &tmC1, p1, g - split, int(gridDim.x) / PAIR - split);
 }
 
 // K == 0: Y = bf16(bias) or 0.
-__global__ void mm_bias_only_kernel(uint16_t* out, const float* bias, int64_t M, int64_t N, int64_t batch,
-                                    int64_t c_stride) {
+// Bias value of column n: float32, dequantised FP8, or 0 without a bias.
+__device__ __forceinline__ float bias_at(const MmParams& p, int64_t n) {
+  if (p.bias8 != nullptr) return __fmul_rn(fp8_value(p.bias8[n], p.bias_fmt), *p.bias_scale);
+  return p.bias != nullptr ? p.bias[n] : 0.0f;
+}
+
+__global__ void mm_bias_only_kernel(const MmParams p, int64_t M, int64_t N, int64_t batch) {
   pdl_launch_dependents();
   pdl_wait_prior_grid();
   const int64_t total = batch * M * N;
   for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < total; i += int64_t(gridDim.x) * blockDim.x) {
     const int64_t b = i / (M * N), r = i - b * M * N, n = r % N;
-    const __nv_bfloat16 h = __float2bfloat16_rn(bias ? bias[n] : 0.0f);
-    out[b * c_stride + r] = *reinterpret_cast<const uint16_t*>(&h);
+    const __nv_bfloat16 h = __float2bfloat16_rn(bias_at(p, n));
+    p.out[b * p.c_stride + r] = *reinterpret_cast<const uint16_t*>(&h);
   }
+}
+
+// FP8 output with K == 0 (y = bias) or an empty output (amax 0): one CTA
+// writes the codes, reduces max |y| and commits the output ring, so every
+// call still adds exactly one history entry.
+__global__ void __launch_bounds__(256) mm_out8_small_kernel(const MmParams p, int64_t M, int64_t N, int64_t batch) {
+  __shared__ float warp_max[8];
+  pdl_launch_dependents();
+  pdl_wait_prior_grid();
+  const float s = *p.r_scale;
+  const int64_t total = batch * M * N;
+  float amax = 0.0f;
+  for (int64_t i = threadIdx.x; i < total; i += blockDim.x) {
+    const int64_t b = i / (M * N), r = i - b * M * N, n = r % N;
+    const float y = bias_at(p, n);
+    amax = fmaxf(amax, fabsf(y));
+    p.out8[b * p.c_stride + r] = p.out_fmt == FP8_E5M2 ? cvt_one<FP8_E5M2>(y, s) : cvt_one<FP8_E4M3>(y, s);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  if (threadIdx.x != 0) return;
+  float a = 0.0f;
+#pragma unroll
+  for (int w = 0; w < 8; ++w) a = fmaxf(a, warp_max[w]);
+  float hist[kHistoryLen];
+#pragma unroll
+  for (int i = 0; i < kHistoryLen; ++i) hist[i] = p.r_history[i];
+  if (p.out_fmt == FP8_E5M2)
+    ring_commit<FP8_E5M2>(a, hist, *p.r_idx, p.r_history, p.r_idx, p.r_scale, p.r_scale_inv, s);
+  else
+    ring_commit<FP8_E4M3>(a, hist, *p.r_idx, p.r_history, p.r_idx, p.r_scale, p.r_scale_inv, s);
 }
 
 // ---- host side -----------------------------------------------------------------
@@ -830,6 +1005,17 @@ bool make_map_mn(CUtensorMap* m, const uint8_t* base, int64_t K, int64_t mn, int
 
 // 3-D map over the bf16 output [batch, M, N] with a 32x32 box, 64B swizzle
 // (the staging-buffer layout the epilogue writes).
+bool make_out_map(CUtensorMap* m, uint16_t* base, int64_t M, int64_t N, int64_t batch, int64_t c_stride);
+
+// 3-D map over FP8 output codes [batch, M, N] with a 32x32 box, 32B swizzle.
+bool make_out8_map(CUtensorMap* m, uint8_t* base, int64_t M, int64_t N, int64_t batch, int64_t c_stride) {
+  const uint64_t dims[3] = {uint64_t(N), uint64_t(M), uint64_t(batch)};
+  const uint64_t strides[2] = {uint64_t(N), uint64_t(batch > 1 ? c_stride : M * N)};
+  const uint32_t box[3] = {32u, 32u, 1u};
+  return encode_tiled_cached(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                             CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE);
+}
+
 bool make_out_map(CUtensorMap* m, uint16_t* base, int64_t M, int64_t N, int64_t batch, int64_t c_stride) {
   const uint64_t dims[3] = {uint64_t(N), uint64_t(M), uint64_t(batch)};
   const uint64_t strides[2] = {uint64_t(N * 2), uint64_t((batch > 1 ? c_stride : M * N) * 2)};
@@ -850,13 +1036,13 @@ int sm_count() {
   return cached[dev];
 }
 
-template <int BN, int PAIR>
+template <int BN, int PAIR, int EPI = 0>
 bool ensure_smem_attr() {
   static bool done[64] = {false};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
   if (!done[dev]) {
-    if (cudaFuncSetAttribute(mm_fp8_kernel<BN, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(mm_fp8_kernel<BN, PAIR, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg<BN, PAIR>::kSmemBytes) != cudaSuccess)
       return false;
     done[dev] = true;
@@ -884,7 +1070,7 @@ int max_pairs(int sms) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, mm_fp8_kernel<BN, 2>, &cfg) != cudaSuccess || n < 1) {
+    if (cudaOccupancyMaxActiveClusters(&n, mm_fp8_kernel<BN, 2, 0>, &cfg) != cudaSuccess || n < 1) {
       cudaGetLastError();
       n = sms / 2;
     }
@@ -918,6 +1104,7 @@ struct MmProblem {
   int64_t M, N, K, batch;
   const int64_t* strides;
   bool nothing;  // M == 0 or N == 0: no output
+  int epi;       // kEpiOut8 | kEpiBias8 bits: which epilogue variant runs
   MmParams p;
 };
 
@@ -934,7 +1121,9 @@ int prepare_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t
                           : make_map(&tb, B, K, N, bb, bb > 1 ? strides[1] : 0, BN / PAIR);
   if (!okA || !okB) return FP8_ERR_CUDA;
   memset(&tc, 0, sizeof(tc));
-  if (p.tma_store && !make_out_map(&tc, p.out, M, N, batch, p.c_stride)) return FP8_ERR_CUDA;
+  if (p.tma_store && !(p.out8 != nullptr ? make_out8_map(&tc, p.out8, M, N, batch, p.c_stride)
+                                         : make_out_map(&tc, p.out, M, N, batch, p.c_stride)))
+    return FP8_ERR_CUDA;
   p.a_bcast = ba == 1;
   p.b_bcast = bb == 1;
   p.m_tiles = int((M + kBM * PAIR - 1) / (kBM * PAIR));
@@ -953,16 +1142,27 @@ int prepare_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t
   return FP8_OK;
 }
 
-template <int BN, int PAIR>
-int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
-              const int64_t* strides, MmParams p, const MmChoice& c, void* ws, cudaStream_t st) {
+template <int BN, int PAIR, int EPI>
+int launch_mm_epi(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+                  const int64_t* strides, MmParams p, const MmChoice& c, void* ws, cudaStream_t st) {
   CUtensorMap ta, tb, tc;
   const int rc = prepare_mm<BN, PAIR>(A, B, M, N, K, batch, strides, p, c, ws, ta, tb, tc);
   if (rc != FP8_OK) return rc;
-  if (!ensure_smem_attr<BN, PAIR>()) return FP8_ERR_CUDA;
-  const cudaError_t e = launch_pdl(mm_fp8_kernel<BN, PAIR>, dim3(PAIR * std::max(1, c.grid)), dim3(kThreadsMM),
+  if (!ensure_smem_attr<BN, PAIR, EPI>()) return FP8_ERR_CUDA;
+  const cudaError_t e = launch_pdl(mm_fp8_kernel<BN, PAIR, EPI>, dim3(PAIR * std::max(1, c.grid)), dim3(kThreadsMM),
                                    Cfg<BN, PAIR>::kSmemBytes, st, PAIR, ta, tb, tc, p);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+template <int BN, int PAIR>
+int launch_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+              const int64_t* strides, const MmParams& p, int epi, const MmChoice& c, void* ws, cudaStream_t st) {
+  switch (epi) {
+    case 0: return launch_mm_epi<BN, PAIR, 0>(A, B, M, N, K, batch, strides, p, c, ws, st);
+    case kEpiOut8: return launch_mm_epi<BN, PAIR, kEpiOut8>(A, B, M, N, K, batch, strides, p, c, ws, st);
+    case kEpiBias8: return launch_mm_epi<BN, PAIR, kEpiBias8>(A, B, M, N, K, batch, strides, p, c, ws, st);
+    default: return launch_mm_epi<BN, PAIR, kEpiOut8 | kEpiBias8>(A, B, M, N, K, batch, strides, p, c, ws, st);
+  }
 }
 
 template <int BN, int PAIR>
@@ -1067,12 +1267,34 @@ using namespace fp8ds;
 namespace fp8ds {
 namespace {
 
+// fp8_mm_ex's epilogue options beyond fp8_mm's: FP8 bias codes and FP8 output.
+struct MmEpilogue {
+  const uint8_t* bias8;     // FP8 bias codes [N] (bias_scale set), else null
+  const float* bias_scale;  // their dequantisation factor (device scalar)
+  int out_kind;             // fp8_mm_out
+  uint8_t* out8;            // FP8 output codes (out_kind != FP8_MM_OUT_BF16)
+  fp8_ring ring;            // the FP8 output's ring
+};
+
 int mm_validate(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
                 const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
-                uint16_t* out_bf16, MmProblem& q) {
+                uint16_t* out_bf16, MmProblem& q, const MmEpilogue* ex = nullptr) {
   if (M < 0 || N < 0 || K < 0 || batch < 1) return FP8_ERR_INVALID_ARG;
-  if ((layout & ~(FP8_MM_A_E5M2 | FP8_MM_B_E5M2 | FP8_MM_A_MN_MAJOR | FP8_MM_B_MN_MAJOR)) != FP8_MM_NT)
+  const bool bias8 = ex != nullptr && ex->bias8 != nullptr;
+  const bool out8 = ex != nullptr && ex->out_kind != FP8_MM_OUT_BF16;
+  const int known = FP8_MM_A_E5M2 | FP8_MM_B_E5M2 | FP8_MM_A_MN_MAJOR | FP8_MM_B_MN_MAJOR |
+                    (bias8 ? FP8_MM_BIAS_E5M2 : 0);
+  if ((layout & ~known) != FP8_MM_NT) return FP8_ERR_INVALID_ARG;
+  if (ex != nullptr && ex->out_kind != FP8_MM_OUT_BF16 && ex->out_kind != FP8_MM_OUT_E4M3 &&
+      ex->out_kind != FP8_MM_OUT_E5M2)
     return FP8_ERR_INVALID_ARG;
+  if (bias8 && (ex->bias_scale == nullptr || bias != nullptr)) return FP8_ERR_INVALID_ARG;
+  if (out8) {
+    const fp8_ring& r = ex->ring;
+    if ((ex->out8 == nullptr && M > 0 && N > 0) || out_bf16 != nullptr) return FP8_ERR_INVALID_ARG;
+    if (!r.history || !r.idx || !r.scale || !r.scale_inv || !r.scratch) return FP8_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(r.scratch) % 8 != 0) return FP8_ERR_UNSUPPORTED;
+  }
   const bool a_mn = (layout & FP8_MM_A_MN_MAJOR) != 0;
   const bool b_mn = (layout & FP8_MM_B_MN_MAJOR) != 0;
   if (batch > 1 && strides == nullptr) return FP8_ERR_INVALID_ARG;
@@ -1086,31 +1308,47 @@ int mm_validate(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_
   q.batch = batch;
   q.strides = strides;
   q.nothing = M == 0 || N == 0;
-  if (q.nothing) return FP8_OK;
-  if (out_bf16 == nullptr || sinv_a == nullptr || sinv_b == nullptr) return FP8_ERR_INVALID_ARG;
+  q.epi = (out8 ? kEpiOut8 : 0) | (bias8 ? kEpiBias8 : 0);
+  MmParams& p = q.p;
+  const int64_t c_stride = batch > 1 ? strides[2] : M * N;
+  p.c_stride = c_stride;
+  if (out8) {
+    p.out_fmt = ex->out_kind == FP8_MM_OUT_E5M2 ? FP8_E5M2 : FP8_E4M3;
+    p.out8 = ex->out8;
+    p.r_history = ex->ring.history;
+    p.r_idx = ex->ring.idx;
+    p.r_scale = ex->ring.scale;
+    p.r_scale_inv = ex->ring.scale_inv;
+    p.r_scratch = ex->ring.scratch;
+  }
+  if (bias8) {
+    p.bias8 = ex->bias8;
+    p.bias_scale = ex->bias_scale;
+    p.bias_fmt = (layout & FP8_MM_BIAS_E5M2) ? FP8_E5M2 : FP8_E4M3;
+  }
+  if (q.nothing) return FP8_OK;  // nothing to compute (an FP8 output still folds amax 0)
+  if ((!out8 && out_bf16 == nullptr) || sinv_a == nullptr || sinv_b == nullptr) return FP8_ERR_INVALID_ARG;
   if (K > 0 && (A == nullptr || B == nullptr)) return FP8_ERR_INVALID_ARG;
   if (M > INT32_MAX / 2 || N > INT32_MAX / 2 || K > INT32_MAX / 2 || batch > 65535) return FP8_ERR_UNSUPPORTED;
   if (K % 16 != 0) return FP8_ERR_UNSUPPORTED;
   if ((a_mn && M % 16 != 0) || (b_mn && N % 16 != 0)) return FP8_ERR_UNSUPPORTED;  // MN-major row pitch
-  if (reinterpret_cast<uintptr_t>(out_bf16) % 2 != 0) return FP8_ERR_UNSUPPORTED;
+  if (!out8 && reinterpret_cast<uintptr_t>(out_bf16) % 2 != 0) return FP8_ERR_UNSUPPORTED;
   if (K > 0) {
     if (reinterpret_cast<uintptr_t>(A) % 16 != 0 || reinterpret_cast<uintptr_t>(B) % 16 != 0)
       return FP8_ERR_UNSUPPORTED;
     if (batch > 1 && ((strides[0] % 16) != 0 || (strides[1] % 16) != 0)) return FP8_ERR_UNSUPPORTED;
   }
-  const int64_t c_stride = batch > 1 ? strides[2] : M * N;
-  MmParams& p = q.p;
   p.M = int(M);
   p.N = int(N);
   p.K = int(K);
   p.k_blocks = int((K + kBK - 1) / kBK);
-  p.c_stride = c_stride;
   p.sinv_a = sinv_a;
   p.sinv_b = sinv_b;
   p.bias = bias;
   p.out = out_bf16;
-  p.out_vec = (reinterpret_cast<uintptr_t>(out_bf16) % 16 == 0) && (N % 8 == 0) && (c_stride % 8 == 0);
-  p.tma_store = p.out_vec;
+  p.out_vec = !out8 && (reinterpret_cast<uintptr_t>(out_bf16) % 16 == 0) && (N % 8 == 0) && (c_stride % 8 == 0);
+  p.out8_vec = out8 && (reinterpret_cast<uintptr_t>(ex->out8) % 16 == 0) && (N % 16 == 0) && (c_stride % 16 == 0);
+  p.tma_store = out8 ? p.out8_vec : p.out_vec;
   p.bias_vec = bias != nullptr && (reinterpret_cast<uintptr_t>(bias) % 16 == 0);
   const uint32_t fa = (layout & FP8_MM_A_E5M2) ? 1u : 0u;
   const uint32_t fb = (layout & FP8_MM_B_E5M2) ? 1u : 0u;
@@ -1127,12 +1365,17 @@ int mm_validate(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_
 int launch_bias_only(const MmProblem& q, cudaStream_t st) {
   const int64_t total = q.batch * q.M * q.N;
   const int grid = int(std::min<int64_t>((total + 255) / 256, 4096));
-  const cudaError_t e = launch_pdl(mm_bias_only_kernel, dim3(grid), dim3(256), 0, st, 1, q.p.out, q.p.bias, q.M, q.N,
-                                   q.batch, q.p.c_stride);
+  const cudaError_t e = launch_pdl(mm_bias_only_kernel, dim3(grid), dim3(256), 0, st, 1, q.p, q.M, q.N, q.batch);
+  return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+int launch_out8_small(const MmProblem& q, cudaStream_t st) {
+  const cudaError_t e = launch_pdl(mm_out8_small_kernel, dim3(1), dim3(256), 0, st, 1, q.p, q.M, q.N, q.batch);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
 int mm_run(MmProblem& q, void* workspace, size_t ws_bytes, cudaStream_t st) {
+  if ((q.epi & kEpiOut8) && (q.nothing || q.K == 0)) return launch_out8_small(q, st);
   if (q.nothing) return FP8_OK;
   if (q.K == 0) return launch_bias_only(q, st);
   const int sms = sm_count();
@@ -1140,11 +1383,11 @@ int mm_run(MmProblem& q, void* workspace, size_t ws_bytes, cudaStream_t st) {
   if (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP8_ERR_UNSUPPORTED;
   const MmChoice c = choose_mm(q.M, q.N, q.K, q.batch, sms, q.p.b_mn, workspace ? ws_bytes : 0);
   if (c.pair == 2) {
-    if (c.bn == 256) return launch_mm<256, 2>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, c, workspace, st);
-    return launch_mm<128, 2>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, c, workspace, st);
+    if (c.bn == 256) return launch_mm<256, 2>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
+    return launch_mm<128, 2>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
   }
-  if (c.bn == 256) return launch_mm<256, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, c, workspace, st);
-  return launch_mm<128, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, c, workspace, st);
+  if (c.bn == 256) return launch_mm<256, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
+  return launch_mm<128, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
 }
 
 }  // namespace
@@ -1171,6 +1414,20 @@ extern "C" int fp8_mm_ws(const uint8_t* A, const uint8_t* B, int64_t M, int64_t 
                          fp8_stream_t stream) {
   return mm_impl(A, B, M, N, K, batch, strides, layout, sinv_a, sinv_b, bias, out_bf16, workspace, workspace_bytes,
                  stream);
+}
+
+extern "C" int fp8_mm_ex(const fp8_mm_ex_args* a, void* workspace, size_t workspace_bytes, fp8_stream_t stream) {
+  if (a == nullptr) return FP8_ERR_INVALID_ARG;
+  const bool bias8 = a->bias_scale != nullptr;
+  const bool out8 = a->out_kind != FP8_MM_OUT_BF16;
+  MmEpilogue ex{bias8 ? static_cast<const uint8_t*>(a->bias) : nullptr, a->bias_scale, a->out_kind,
+                out8 ? static_cast<uint8_t*>(a->out) : nullptr, a->out_ring};
+  MmProblem q;
+  const int rc = mm_validate(a->A, a->B, a->M, a->N, a->K, a->batch, a->strides, a->layout, a->sinv_a, a->sinv_b,
+                             bias8 ? nullptr : static_cast<const float*>(a->bias),
+                             out8 ? nullptr : static_cast<uint16_t*>(a->out), q, &ex);
+  if (rc != FP8_OK) return rc;
+  return mm_run(q, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 extern "C" int fp8_mm_pair(const fp8_mm_args* a0, const fp8_mm_args* a1, void* workspace, size_t workspace_bytes,

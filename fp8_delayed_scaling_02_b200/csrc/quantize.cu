@@ -35,6 +35,7 @@
 #include <cstring>
 
 #include "common.cuh"
+#include "fp8_ring.cuh"
 
 namespace fp8ds {
 namespace {
@@ -185,46 +186,6 @@ __device__ __forceinline__ float absmax2_to_float(uint32_t acc) {
   return fmaxf(lo, hi);
 }
 
-// (a*s, b*s) with one packed fp32x2 multiply, each lane rounded to nearest
-// even exactly as a scalar fp32 multiply (no contraction into anything else).
-__device__ __forceinline__ void scale2(float& a, float& b, float s) {
-  asm("{\n\t.reg .b64 ra, rs, rd;\n\t"
-      "mov.b64 ra, {%0, %1};\n\t"
-      "mov.b64 rs, {%2, %2};\n\t"
-      "mul.rn.f32x2 rd, ra, rs;\n\t"
-      "mov.b64 {%0, %1}, rd;\n\t}"
-      : "+f"(a), "+f"(b)
-      : "f"(s));
-}
-
-// fp8 codes of two already-scaled values packed low byte first: the hardware
-// round-to-nearest-even conversion with saturation to the largest finite value.
-template <int FMT>
-__device__ __forceinline__ uint32_t cvt2(float lo, float hi) {
-  return uint32_t(
-      __nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, FMT == FP8_E4M3 ? __NV_E4M3 : __NV_E5M2));
-}
-
-// Codes of v[0..3] * s in one word (v[0] in the low byte).
-template <int FMT>
-__device__ __forceinline__ uint32_t cvt4(float v0, float v1, float v2, float v3, float s) {
-  scale2(v0, v1, s);
-  scale2(v2, v3, s);
-  return __byte_perm(cvt2<FMT>(v0, v1), cvt2<FMT>(v2, v3), 0x5410);
-}
-
-template <int FMT>
-__device__ __forceinline__ uint32_t cvt_pair(float lo, float hi, float s) {
-  scale2(lo, hi, s);
-  return cvt2<FMT>(lo, hi);
-}
-
-template <int FMT>
-__device__ __forceinline__ uint8_t cvt_one(float x, float s) {
-  return uint8_t(__nv_cvt_float_to_fp8(__fmul_rn(x, s), __NV_SATFINITE,
-                                       FMT == FP8_E4M3 ? __NV_E4M3 : __NV_E5M2));
-}
-
 // 4x4 byte transpose: word r holds bytes (r, 0..3); output word c holds bytes
 // (0..3, c), i.e. byte r of c_out is byte c of r_in.  Eight byte permutes.
 __device__ __forceinline__ void transpose4x4(uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3, uint32_t& c0,
@@ -315,20 +276,7 @@ __device__ __forceinline__ void amax_ticket_fold(float amax, const RingArgs& rin
         *ring.scale_inv = __frcp_rn(s_used);
         return;
       }
-      int idx = idx_s;
-      idx = ((idx % kHistoryLen) + kHistoryLen) % kHistoryLen;
-      hist_s[idx] = a;
-      float mx = 0.0f;
-#pragma unroll
-      for (int i = 0; i < kHistoryLen; ++i) mx = fmaxf(mx, hist_s[i]);
-      ring.history[idx] = a;
-      *ring.idx = (idx + 1) % kHistoryLen;
-      const float fmax = FMT == FP8_E4M3 ? kE4M3Max : kE5M2Max;
-      if (mx > 0.0f && isfinite(mx)) {
-        const float c = __fdiv_rn(fmax, mx);
-        if (isfinite(c) && c > 0.0f) *ring.scale = c;
-      }
-      *ring.scale_inv = __frcp_rn(s_used);
+      ring_commit<FMT>(a, hist_s, idx_s, ring.history, ring.idx, ring.scale, ring.scale_inv, s_used);
     }
   }
 }
@@ -1297,21 +1245,10 @@ __global__ void ring_fold_kernel(float* history, int32_t* idx_p, float* scale, f
   pdl_launch_dependents();
   pdl_wait_prior_grid();
   if (threadIdx.x != 0) return;
-  const float a = *amax;
-  const float s_used = *scale;
-  int idx = *idx_p;
-  idx = ((idx % kHistoryLen) + kHistoryLen) % kHistoryLen;
-  history[idx] = a;
-  float mx = 0.0f;
+  float hist[kHistoryLen];
 #pragma unroll
-  for (int i = 0; i < kHistoryLen; ++i) mx = fmaxf(mx, history[i]);
-  *idx_p = (idx + 1) % kHistoryLen;
-  const float fmax = FMT == FP8_E4M3 ? kE4M3Max : kE5M2Max;
-  if (mx > 0.0f && isfinite(mx)) {
-    const float c = __fdiv_rn(fmax, mx);
-    if (isfinite(c) && c > 0.0f) *scale = c;
-  }
-  *scale_inv = __frcp_rn(s_used);
+  for (int i = 0; i < kHistoryLen; ++i) hist[i] = history[i];
+  ring_commit<FMT>(*amax, hist, *idx_p, history, idx_p, scale, scale_inv, *scale);
 }
 }  // namespace
 }  // namespace fp8ds

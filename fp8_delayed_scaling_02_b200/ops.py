@@ -21,6 +21,8 @@ MM_A_MN_MAJOR = 1 << 0
 MM_B_MN_MAJOR = 1 << 1
 MM_A_E5M2 = 1 << 8
 MM_B_E5M2 = 1 << 9
+MM_BIAS_E5M2 = 1 << 10
+MM_OUT_BF16, MM_OUT_E4M3, MM_OUT_E5M2 = 0, 1, 2
 HISTORY_LEN = 16
 
 FP8_OK = 0
@@ -90,6 +92,8 @@ def lib():
         L.fp8_mm_pair.restype = i32
         L.fp8_quantize_pair.argtypes = [vp, vp, vp]
         L.fp8_quantize_pair.restype = i32
+        L.fp8_mm_ex.argtypes = [vp, vp, ctypes.c_size_t, vp]
+        L.fp8_mm_ex.restype = i32
         L.fp8_launch_count.argtypes = []
         L.fp8_launch_count.restype = ctypes.c_uint64
         _LIB = L
@@ -377,6 +381,66 @@ def mm(a, b, sinv_a, sinv_b, bias=None, fmt_a=E4M3, fmt_b=E4M3, out=None, stream
                          sinv_b.data_ptr(), _ptr(bias), out3.data_ptr(), workspace.data_ptr(),
                          workspace.numel() * workspace.element_size(), _stream(stream, a.get_device()))
     _check(rc, "fp8_mm")
+    return out
+
+
+class CMmExArgs(ctypes.Structure):
+    """Mirror of ``fp8_mm_ex_args``."""
+
+    _fields_ = [("A", ctypes.c_void_p), ("B", ctypes.c_void_p), ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("batch", ctypes.c_int64), ("strides", ctypes.c_void_p),
+                ("layout", ctypes.c_int), ("sinv_a", ctypes.c_void_p), ("sinv_b", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("bias_scale", ctypes.c_void_p), ("out_kind", ctypes.c_int),
+                ("out", ctypes.c_void_p), ("out_ring", CRing)]
+
+
+def mm_ex(a, b, sinv_a, sinv_b, bias=None, bias_scale=None, bias_fmt=E4M3, out_fmt=None, out_ring=None,
+          fmt_a=E4M3, fmt_b=E4M3, out=None, a_mn_major=False, b_mn_major=False, workspace=None, stream=None):
+    """fp8_mm_ex: ``mm`` with an FP8 bias and / or an FP8 output.
+
+    bias: float32 [N], or (with bias_scale, a one-element float32 CUDA tensor)
+    uint8 FP8 codes [N] in format bias_fmt, dequantised as code * bias_scale.
+    out_fmt: None for bf16 output, or E4M3 / E5M2 for FP8 codes of
+    y * out_ring.scale, with max |y| folded into ``out_ring`` (a Ring) in the
+    same launch.  Operands and batching as ``mm``.  Returns out.
+    """
+    if a.dtype != torch.uint8 or b.dtype != torch.uint8:
+        raise ValueError("a and b hold FP8 codes as uint8")
+    if out_fmt is not None and out_ring is None:
+        raise ValueError("an FP8 output needs out_ring")
+    if bias_scale is not None and bias is not None and bias.dtype != torch.uint8:
+        raise ValueError("with bias_scale the bias holds FP8 codes (uint8)")
+    a3 = a if a.dim() == 3 else a.unsqueeze(0)
+    b3 = b if b.dim() == 3 else b.unsqueeze(0)
+    batch = max(a3.shape[0], b3.shape[0])
+    K, M = (a3.shape[1], a3.shape[2]) if a_mn_major else (a3.shape[2], a3.shape[1])
+    Kb, N = (b3.shape[1], b3.shape[2]) if b_mn_major else (b3.shape[2], b3.shape[1])
+    if Kb != K:
+        raise ValueError("K mismatch")
+    for t in (a3, b3):
+        if t.shape[0] not in (1, batch) or (t.numel() > 0 and (t.stride(2) != 1 or (t.shape[1] > 1 and t.stride(1) != t.shape[2]))):
+            raise ValueError("operands must be contiguous in their last two dims with matching batch")
+    sa = 0 if a3.shape[0] == 1 else a3.stride(0)
+    sb = 0 if b3.shape[0] == 1 else b3.stride(0)
+    dtype = torch.bfloat16 if out_fmt is None else torch.uint8
+    two_d = a.dim() == 2 and b.dim() == 2
+    if out is None:
+        out = torch.empty((M, N) if two_d else (batch, M, N), dtype=dtype, device=a.device)
+    out3 = out if out.dim() == 3 else out.unsqueeze(0)
+    if out.dtype != dtype or not out.is_contiguous() or tuple(out3.shape) != (batch, M, N):
+        raise ValueError(f"out must be a contiguous [batch, M, N] {dtype} tensor")
+    strides = (ctypes.c_int64 * 3)(sa, sb, out3.stride(0) if batch > 1 else M * N)
+    layout = _layout(fmt_a, fmt_b, a_mn_major, b_mn_major)
+    if bias_scale is not None and bias_fmt == E5M2:
+        layout |= MM_BIAS_E5M2
+    kind = MM_OUT_BF16 if out_fmt is None else (MM_OUT_E5M2 if out_fmt == E5M2 else MM_OUT_E4M3)
+    ring = out_ring.c() if out_ring is not None else CRing()
+    args = CMmExArgs(a3.data_ptr(), b3.data_ptr(), M, N, K, batch, ctypes.cast(strides, ctypes.c_void_p), layout,
+                     sinv_a.data_ptr(), sinv_b.data_ptr(), _ptr(bias), _ptr(bias_scale), kind,
+                     out3.data_ptr(), ring)
+    ws, wsb = (workspace.data_ptr(), workspace.numel() * workspace.element_size()) if workspace is not None else (None, 0)
+    rc = (_LIB or lib()).fp8_mm_ex(ctypes.byref(args), ws, wsb, _stream(stream, a.get_device()))
+    _check(rc, "fp8_mm_ex")
     return out
 
 

@@ -11,7 +11,8 @@
  *                 fp32 bias, optional batch with stride-0 broadcast.
  *
  * Around them: fp8_quantize_pair / fp8_mm_pair (two calls in one launch),
- * fp8_mm_ws (stream-K tail through a caller workspace), fp8_quantize_current
+ * fp8_mm_ws (stream-K tail through a caller workspace), fp8_mm_ex (FP8 bias,
+ * FP8 output with delayed output scaling), fp8_quantize_current
  * (current scaling), fp8_quantize_local + fp8_ring_fold (data-parallel
  * delayed scaling), fp8_bias_grad and fp8_linear_forward / _backward (the
  * linear composites), fp8_quantize_static_scratch (no caller scratch), and
@@ -253,6 +254,7 @@ int fp8_bias_grad(const void* g, int dtype, int64_t rows, int64_t cols, float* d
 #define FP8_MM_B_MN_MAJOR (1 << 1) /* B stored [K, N]; needs N % 16 == 0 */
 #define FP8_MM_A_E5M2 (1 << 8)     /* A holds E5M2 codes (default E4M3) */
 #define FP8_MM_B_E5M2 (1 << 9)     /* B holds E5M2 codes (default E4M3) */
+#define FP8_MM_BIAS_E5M2 (1 << 10) /* fp8_mm_ex: FP8 bias codes are E5M2 (default E4M3) */
 
 /*
  * fp8_mm -- scaled FP8 GEMM with fused scale, bias and bf16 rounding.
@@ -380,6 +382,59 @@ typedef struct {
 } fp8_mm_args;
 int fp8_mm_pair(const fp8_mm_args* a0, const fp8_mm_args* a1, void* workspace, size_t workspace_bytes,
                 fp8_stream_t stream);
+
+/*
+ * fp8_mm_ex -- fp8_mm with the two epilogue variants of the pages' FP8
+ * GEMM: FP8 bias storage and FP8 output.
+ *
+ * Sources: "AstrAI commits, branch main, tests/extension" page, the
+ * bias_scale commit (the bias may be FP8 storage with a scale, dequantised
+ * in the epilogue after the operand scaling and before any output
+ * quantisation) and the FP8-in/FP8-out GEMM commit.  The pages give no
+ * formula for either; the reading here keeps every FP8 tensor on per-tensor
+ * delayed scaling.  With y the float32 epilogue value
+ *   y[b,m,n] = sinv_a * sinv_b * sum_k A[b,m,k] B[b,n,k] + bias[n]
+ * (one fused multiply-add on the float32 accumulator, as in fp8_mm):
+ *   bias      bias_scale == NULL: float32 [N] (or NULL, no bias), as fp8_mm;
+ *             bias_scale != NULL: FP8 codes [N] (E4M3, or E5M2 with
+ *             FP8_MM_BIAS_E5M2 in layout), bias[n] = fp32(decode(code) *
+ *             *bias_scale).
+ *   out       out_kind FP8_MM_OUT_BF16: bf16 [batch, M, N] = bf16_rn(y), as
+ *             fp8_mm (out_ring unused).
+ *             out_kind FP8_MM_OUT_E4M3 / _E5M2: FP8 codes [batch, M, N] =
+ *             saturate_rne_fp8(fp32(y * s)) with s = *out_ring.scale read at
+ *             launch -- the output tensor's delayed scale -- and, in the CTA
+ *             that finishes last, out_ring folds amax = max |y| over the
+ *             output (NaN ignored) exactly as fp8_quantize folds its input's
+ *             amax: next scale published, scale_inv = 1/s for the GEMM that
+ *             consumes the output.  An empty output folds amax 0; K == 0
+ *             gives y = bias.
+ * Arguments, layouts, strides (strides[2] counts output elements), the
+ * workspace and the errors are fp8_mm_ws's, plus FP8_ERR_INVALID_ARG for an
+ * unknown out_kind, FP8_MM_BIAS_E5M2 without bias_scale, or an FP8 output
+ * without out (non-empty output) or without a complete out_ring;
+ * FP8_ERR_UNSUPPORTED for an out_ring.scratch that is not 8-byte aligned.
+ * Validation happens before any CUDA call.  Codes leave through TMA stores
+ * when out is 16-byte aligned and N and the batch stride are multiples of 16,
+ * through byte stores otherwise.  One ring must not be used by two calls in
+ * flight.
+ */
+typedef enum { FP8_MM_OUT_BF16 = 0, FP8_MM_OUT_E4M3 = 1, FP8_MM_OUT_E5M2 = 2 } fp8_mm_out;
+typedef struct {
+  const uint8_t* A;
+  const uint8_t* B;
+  int64_t M, N, K, batch;
+  const int64_t* strides;
+  int layout;               /* fp8_mm's layout bits, plus FP8_MM_BIAS_E5M2 */
+  const float* sinv_a;
+  const float* sinv_b;
+  const void* bias;         /* NULL, float32 [N], or FP8 codes [N] (bias_scale set) */
+  const float* bias_scale;  /* device scalar, or NULL for a float32 bias */
+  int out_kind;             /* fp8_mm_out */
+  void* out;                /* bf16 or FP8 codes [batch, M, N] */
+  fp8_ring out_ring;        /* FP8 output: the output tensor's ring */
+} fp8_mm_ex_args;
+int fp8_mm_ex(const fp8_mm_ex_args* args, void* workspace, size_t workspace_bytes, fp8_stream_t stream);
 
 /* Number of kernels this process has launched through the library so far
  * (every entry point, every device; a host-side counter, safe to call from

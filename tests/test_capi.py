@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
         ["fp8_quantize", "fp8_mm", "fp8_status_string", "fp8_device_error", "fp8_device_info",
          "fp8_quantize_static_scratch", "fp8_quantize_current", "fp8_bias_grad", "fp8_linear_forward",
          "fp8_linear_backward", "fp8_mm_ws", "fp8_mm_workspace_bytes", "fp8_quantize_local", "fp8_ring_fold",
-         "fp8_mm_pair", "fp8_launch_count", "fp8_quantize_pair"])
+         "fp8_mm_pair", "fp8_launch_count", "fp8_quantize_pair", "fp8_mm_ex"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -108,3 +108,21 @@ def test_mm_rejects_bad_arguments_without_cuda(L):
     # Empty products are a no-op that needs no device.
     assert _mm(L, M=0) == ops.FP8_OK
     assert _mm(L, N=0, A=0, B=0) == ops.FP8_OK
+
+
+def _mm_ex(L, out_kind=ops.MM_OUT_E4M3, layout=0, bias=None, bias_scale=None, out=0x30000, ring=None, M=128):
+    args = ops.CMmExArgs(0x10000, 0x20000, M, 128, 128, 1, None, layout, 0x40000, 0x40010, bias, bias_scale,
+                         out_kind, out, ring if ring is not None else _ring())
+    return L.fp8_mm_ex(ctypes.byref(args), None, 0, None)
+
+
+def test_mm_ex_rejects_bad_arguments_without_cuda(L):
+    assert L.fp8_mm_ex(None, None, 0, None) == ops.FP8_ERR_INVALID_ARG
+    assert _mm_ex(L, out_kind=3) == ops.FP8_ERR_INVALID_ARG
+    assert _mm_ex(L, out_kind=-1) == ops.FP8_ERR_INVALID_ARG
+    assert _mm_ex(L, out=0) == ops.FP8_ERR_INVALID_ARG                      # FP8 output without codes
+    assert _mm_ex(L, ring=ops.CRing(0x1000, 0x1040, 0, 0x1048, 0x1050)) == ops.FP8_ERR_INVALID_ARG  # no scale
+    assert _mm_ex(L, ring=ops.CRing(0x1000, 0x1040, 0x1044, 0x1048, 0)) == ops.FP8_ERR_INVALID_ARG  # no scratch
+    assert _mm_ex(L, ring=ops.CRing(0x1000, 0x1040, 0x1044, 0x1048, 0x1054)) == ops.FP8_ERR_UNSUPPORTED
+    assert _mm_ex(L, layout=ops.MM_BIAS_E5M2) == ops.FP8_ERR_INVALID_ARG    # bias format bit without FP8 bias
+    assert _mm_ex(L, out_kind=ops.MM_OUT_BF16, out=0) == ops.FP8_ERR_INVALID_ARG

@@ -29,6 +29,19 @@ __device__ __forceinline__ void scale2(float& a, float& b, float s) {
       : "f"(s));
 }
 
+// (a*s + c, b*s + d) with one packed fp32x2 fused multiply-add: each lane
+// is rounded once to nearest even, exactly as fmaf.
+__device__ __forceinline__ void fma2(float& a, float& b, float s, float c, float d) {
+  asm("{\n\t.reg .b64 ra, rs, rc, rd;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rs, {%2, %2};\n\t"
+      "mov.b64 rc, {%3, %4};\n\t"
+      "fma.rn.f32x2 rd, ra, rs, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(a), "+f"(b)
+      : "f"(s), "f"(c), "f"(d));
+}
+
 // fp8 codes of two already-scaled values packed low byte first.
 template <int FMT>
 __device__ __forceinline__ uint32_t cvt2(float lo, float hi) {

@@ -716,10 +716,10 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
             bv.z = __shfl_sync(0xFFFFFFFFu, bias_l.z, src);
             bv.w = __shfl_sync(0xFFFFFFFFu, bias_l.w, src);
           }
-          const float y0 = fmaf(__uint_as_float(v[4 * j + 0]), sab, bv.x);
-          const float y1 = fmaf(__uint_as_float(v[4 * j + 1]), sab, bv.y);
-          const float y2 = fmaf(__uint_as_float(v[4 * j + 2]), sab, bv.z);
-          const float y3 = fmaf(__uint_as_float(v[4 * j + 3]), sab, bv.w);
+          float y0 = __uint_as_float(v[4 * j + 0]), y1 = __uint_as_float(v[4 * j + 1]);
+          float y2 = __uint_as_float(v[4 * j + 2]), y3 = __uint_as_float(v[4 * j + 3]);
+          fma2(y0, y1, sab, bv.x, bv.y);  // acc * sinv_a*sinv_b + bias, one rounding each
+          fma2(y2, y3, sab, bv.z, bv.w);
           if constexpr (kOut8) {
             // amax over this lane's in-range elements (NaN ignored), then the
             // codes of y * s_out.

@@ -134,8 +134,10 @@ __device__ __forceinline__ float4 bias8_4(const MmParams& p, int n, float bsc) {
 // ring's scratch word; the CTA that draws the last of gridDim.x tickets takes
 // the grid's amax, clears the scratch words and commits the ring.  The
 // acq_rel ticket orders each CTA's amax before its increment and gives the
-// last CTA every other CTA's.  Run by one thread after the CTA's epilogue.
-__device__ __noinline__ void out8_ticket_fold(const MmParams& p, const float* amax_s) {
+// last CTA every other CTA's.  ring_s holds the ring's history, idx and scale
+// as read at launch (only this fold writes them).  Run by one thread after
+// the CTA's epilogue.
+__device__ __noinline__ void out8_ticket_fold(const MmParams& p, const float* amax_s, const float* ring_s) {
   float m = 0.0f;
 #pragma unroll
   for (int w = 0; w < kEpiWarps; ++w) m = fmaxf(m, amax_s[w]);
@@ -149,12 +151,14 @@ __device__ __noinline__ void out8_ticket_fold(const MmParams& p, const float* am
   asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(p.r_scratch + 1) : "memory");
   float hist[kHistoryLen];
 #pragma unroll
-  for (int i = 0; i < kHistoryLen; ++i) hist[i] = p.r_history[i];
+  for (int i = 0; i < kHistoryLen; ++i) hist[i] = ring_s[i];
+  const int idx = __float_as_int(ring_s[kHistoryLen]);
+  const float s_used = ring_s[kHistoryLen + 1];
   const float a = __uint_as_float(bits);
   if (p.out_fmt == FP8_E5M2)
-    ring_commit<FP8_E5M2>(a, hist, *p.r_idx, p.r_history, p.r_idx, p.r_scale, p.r_scale_inv, *p.r_scale);
+    ring_commit<FP8_E5M2>(a, hist, idx, p.r_history, p.r_idx, p.r_scale, p.r_scale_inv, s_used);
   else
-    ring_commit<FP8_E4M3>(a, hist, *p.r_idx, p.r_history, p.r_idx, p.r_scale, p.r_scale_inv, *p.r_scale);
+    ring_commit<FP8_E4M3>(a, hist, idx, p.r_history, p.r_idx, p.r_scale, p.r_scale_inv, s_used);
 }
 
 // ---- PTX wrappers (written from the PTX ISA description) -----------------------
@@ -480,6 +484,13 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait_prior_grid();  // inputs, scales and the output buffer belong to earlier work until here
+  // FP8 output: lanes 0..17 of warp 1 hold the output ring's history, idx and
+  // scale from here to the fold, so the last CTA's fold waits for no loads.
+  float ring_v = 0.0f;
+  if constexpr (kOut8) {
+    if (warp == 1 && lane <= kHistoryLen + 1)
+      ring_v = lane < kHistoryLen ? p.r_history[lane] : lane == kHistoryLen ? __int_as_float(*p.r_idx) : *p.r_scale;
+  }
 
   if (warp == 0) {
     // ---------------- TMA producer (both CTAs of a pair) ----------------
@@ -723,7 +734,9 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
           if constexpr (kOut8) {
             // amax over this lane's in-range elements (NaN ignored), then the
             // codes of y * s_out.
-            if (row_ok) {
+            if (row_ok && full) {  // full: warp-uniform, so no per-column checks
+              amax = fmaxf(amax, fmaxf(fmaxf(fabsf(y0), fabsf(y1)), fmaxf(fabsf(y2), fabsf(y3))));
+            } else if (row_ok) {
               const int nn = n0 + 4 * j;
               amax = fmaxf(amax, nn < p.N ? fabsf(y0) : 0.f);
               amax = fmaxf(amax, nn + 1 < p.N ? fabsf(y1) : 0.f);
@@ -763,12 +776,30 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
             buf ^= 1;
             return;
           }
-          // Rows not 16-byte aligned: guarded byte stores of this lane's row.
-          if (!row_ok) return;
-          uint8_t* o = p.out8 + int64_t(b) * p.c_stride + int64_t(m0 + lane) * p.N + n0;
+          // Rows not 16-byte aligned: the chunk is staged in the same
+          // layout, then written row by row, lane l taking column n0 + l, so
+          // each store instruction covers 32 contiguous bytes of one row.
+          const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
+          __syncwarp();  // every lane has read this buffer's previous chunk
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t addr = sbuf + uint32_t(lane) * 32u + uint32_t((u ^ ((lane >> 2) & 1)) * 16);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(packed[4 * u]),
+                         "r"(packed[4 * u + 1]), "r"(packed[4 * u + 2]), "r"(packed[4 * u + 3])
+                         : "memory");
+          }
+          __syncwarp();
+          const bool col_ok = n0 + lane < p.N;
+          uint8_t* obase = p.out8 + int64_t(b) * p.c_stride + int64_t(m0) * p.N + n0 + lane;
 #pragma unroll 4
-          for (int k = 0; k < 32; ++k)
-            if (n0 + k < p.N) o[k] = uint8_t(packed[k >> 2] >> (8 * (k & 3)));
+          for (int rr = 0; rr < 32; ++rr) {
+            const uint32_t addr =
+                sbuf + uint32_t(rr) * 32u + uint32_t((((lane >> 4) ^ ((rr >> 2) & 1)) << 4) + (lane & 15));
+            uint16_t v16;
+            asm volatile("ld.shared.u8 %0, [%1];" : "=h"(v16) : "r"(addr) : "memory");
+            if (col_ok && m0 + rr < p.M) obase[int64_t(rr) * p.N] = uint8_t(v16);
+          }
+          buf ^= 1;
           return;
         }
         const uint32_t sbuf = stage0 + uint32_t(buf) * kStagingBytes;
@@ -899,7 +930,15 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
   tc_fence_before();
   __syncthreads();
   if constexpr (kOut8) {
-    if (threadIdx.x == 0) out8_ticket_fold(p, amax_s);
+    if (warp == 1) {
+      // The staging buffers are free: every epilogue warp waited for its
+      // stores before the barrier above.
+      float* ring_s = reinterpret_cast<float*>(smem + C::kStagingOffset);
+      if (lane <= kHistoryLen + 1) ring_s[lane] = ring_v;
+      __syncwarp();
+      if (lane == 0) out8_ticket_fold(p, amax_s, ring_s);
+      __syncwarp();
+    }
   }
   // A pair leaves together: the leader's MMAs read the peer's shared memory
   // and write the peer's TMEM until done_bar fired.

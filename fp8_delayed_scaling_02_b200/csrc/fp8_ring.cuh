@@ -1,5 +1,5 @@
-// FP8 casts and the delayed-scaling ring commit shared by the quantize and
-// GEMM kernels (sm_100a).
+// FP8 casts, packed fp32x2 arithmetic and the delayed-scaling ring commit
+// shared by the quantize and GEMM kernels (sm_100a).
 //
 // Cast: one fp32 multiply by the scale, rounded to nearest even, then the
 // hardware round-to-nearest-even conversion with saturation to the largest

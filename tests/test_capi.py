@@ -126,3 +126,22 @@ def test_mm_ex_rejects_bad_arguments_without_cuda(L):
     assert _mm_ex(L, ring=ops.CRing(0x1000, 0x1040, 0x1044, 0x1048, 0x1054)) == ops.FP8_ERR_UNSUPPORTED
     assert _mm_ex(L, layout=ops.MM_BIAS_E5M2) == ops.FP8_ERR_INVALID_ARG    # bias format bit without FP8 bias
     assert _mm_ex(L, out_kind=ops.MM_OUT_BF16, out=0) == ops.FP8_ERR_INVALID_ARG
+
+
+def test_mm_ex_binding_checks_arguments_on_the_host():
+    """ops.mm_ex refuses inconsistent arguments before it touches the library."""
+    import torch
+
+    a = torch.zeros((128, 64), dtype=torch.uint8)
+    b = torch.zeros((96, 64), dtype=torch.uint8)
+    one = torch.ones(1)
+    with pytest.raises(ValueError):
+        ops.mm_ex(a, b, one, one, out_fmt=ops.E4M3)  # FP8 output without a ring
+    with pytest.raises(ValueError):
+        ops.mm_ex(a, b, one, one, bias=torch.zeros(96), bias_scale=one)  # float32 bias with a scale
+    with pytest.raises(ValueError):
+        ops.mm_ex(a, torch.zeros((96, 32), dtype=torch.uint8), one, one)  # K mismatch
+    with pytest.raises(ValueError):
+        ops.mm_ex(a.float(), b, one, one)  # operands are uint8 codes
+    with pytest.raises(ValueError):
+        ops.mm_ex(a, b, one, one, out=torch.zeros((128, 96), dtype=torch.uint8))  # bf16 output expected

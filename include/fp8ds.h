@@ -416,7 +416,8 @@ int fp8_mm_pair(const fp8_mm_args* a0, const fp8_mm_args* a1, void* workspace, s
  * FP8_ERR_UNSUPPORTED for an out_ring.scratch that is not 8-byte aligned.
  * Validation happens before any CUDA call.  Codes leave through TMA stores
  * when out is 16-byte aligned and N and the batch stride are multiples of 16,
- * through byte stores otherwise.  One ring must not be used by two calls in
+ * otherwise through guarded stores of staged rows (32 contiguous bytes of
+ * one row per warp store).  One ring must not be used by two calls in
  * flight.
  */
 typedef enum { FP8_MM_OUT_BF16 = 0, FP8_MM_OUT_E4M3 = 1, FP8_MM_OUT_E5M2 = 2 } fp8_mm_out;

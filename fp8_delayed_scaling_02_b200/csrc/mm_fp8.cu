@@ -111,6 +111,7 @@ struct MmParams {
   float* r_scale;
   float* r_scale_inv;
   uint32_t* r_scratch;  // [0] amax bits, [1] CTA ticket; zero between calls
+  float* amax_out;      // data-parallel shard: the amax goes here, no fold
 };
 
 constexpr int kEpiOut8 = 1;   // EPI bit: FP8 output codes + output ring fold
@@ -155,6 +156,11 @@ __device__ __noinline__ void out8_ticket_fold(const MmParams& p, const float* am
   const int idx = __float_as_int(ring_s[kHistoryLen]);
   const float s_used = ring_s[kHistoryLen + 1];
   const float a = __uint_as_float(bits);
+  if (p.amax_out != nullptr) {  // shard of a data-parallel output: the fold follows a cross-rank MAX
+    *p.amax_out = a;
+    *p.r_scale_inv = __frcp_rn(s_used);
+    return;
+  }
   if (p.out_fmt == FP8_E5M2)
     ring_commit<FP8_E5M2>(a, hist, idx, p.r_history, p.r_idx, p.r_scale, p.r_scale_inv, s_used);
   else
@@ -1011,6 +1017,11 @@ __global__ void __launch_bounds__(256) mm_out8_small_kernel(const MmParams p, in
   float a = 0.0f;
 #pragma unroll
   for (int w = 0; w < 8; ++w) a = fmaxf(a, warp_max[w]);
+  if (p.amax_out != nullptr) {
+    *p.amax_out = a;
+    *p.r_scale_inv = __frcp_rn(s);
+    return;
+  }
   float hist[kHistoryLen];
 #pragma unroll
   for (int i = 0; i < kHistoryLen; ++i) hist[i] = p.r_history[i];
@@ -1313,6 +1324,7 @@ struct MmEpilogue {
   int out_kind;             // fp8_mm_out
   uint8_t* out8;            // FP8 output codes (out_kind != FP8_MM_OUT_BF16)
   fp8_ring ring;            // the FP8 output's ring
+  float* amax_out;          // data-parallel shard: amax out, no fold
 };
 
 int mm_validate(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
@@ -1334,6 +1346,7 @@ int mm_validate(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_
     if (!r.history || !r.idx || !r.scale || !r.scale_inv || !r.scratch) return FP8_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(r.scratch) % 8 != 0) return FP8_ERR_UNSUPPORTED;
   }
+  if (ex != nullptr && ex->amax_out != nullptr && !out8) return FP8_ERR_INVALID_ARG;
   const bool a_mn = (layout & FP8_MM_A_MN_MAJOR) != 0;
   const bool b_mn = (layout & FP8_MM_B_MN_MAJOR) != 0;
   if (batch > 1 && strides == nullptr) return FP8_ERR_INVALID_ARG;
@@ -1359,6 +1372,7 @@ int mm_validate(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_
     p.r_scale = ex->ring.scale;
     p.r_scale_inv = ex->ring.scale_inv;
     p.r_scratch = ex->ring.scratch;
+    p.amax_out = ex->amax_out;
   }
   if (bias8) {
     p.bias8 = ex->bias8;
@@ -1460,7 +1474,7 @@ extern "C" int fp8_mm_ex(const fp8_mm_ex_args* a, void* workspace, size_t worksp
   const bool bias8 = a->bias_scale != nullptr;
   const bool out8 = a->out_kind != FP8_MM_OUT_BF16;
   MmEpilogue ex{bias8 ? static_cast<const uint8_t*>(a->bias) : nullptr, a->bias_scale, a->out_kind,
-                out8 ? static_cast<uint8_t*>(a->out) : nullptr, a->out_ring};
+                out8 ? static_cast<uint8_t*>(a->out) : nullptr, a->out_ring, a->out_amax};
   MmProblem q;
   const int rc = mm_validate(a->A, a->B, a->M, a->N, a->K, a->batch, a->strides, a->layout, a->sinv_a, a->sinv_b,
                              bias8 ? nullptr : static_cast<const float*>(a->bias),

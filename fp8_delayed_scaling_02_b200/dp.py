@@ -16,6 +16,10 @@ quantize splits around one 4-byte collective:
 3. ``ops.ring_fold``: every rank folds the global amax into its own copy of
    the ring, so rings that start equal stay equal.
 
+The FP8-output GEMM splits the same way (``mm_fp8_out_dp``): each rank's
+``ops.mm_ex`` writes its output rows' codes with the output ring's scale and
+that shard's max |y|, the ranks MAX-reduce it, and every rank folds it.
+
 Weights are replicated across data-parallel ranks and keep the single-rank
 ``ops.quantize``.
 """
@@ -48,3 +52,22 @@ def quantize_dp(x, fmt, layout, ring, group=None, amax=None, out=None, out_t=Non
     all_reduce_amax(amax, group)
     ops.ring_fold(ring, fmt, amax)
     return out, out_t
+
+
+def mm_fp8_out_dp(a, b, sinv_a, sinv_b, out_fmt, ring, group=None, amax=None, **mm_kwargs):
+    """FP8-output GEMM of this rank's rows ``a`` with the output's ring folded
+    from the amax of the whole sharded output.
+
+    ``mm_kwargs`` are ``ops.mm_ex``'s other keyword arguments (bias,
+    bias_scale, bias_fmt, fmt_a, fmt_b, out, layouts, workspace).  Returns the
+    codes.  Every rank of ``group`` must call it for the same output in the
+    same order (it runs one collective).
+    """
+    import torch
+
+    if amax is None:
+        amax = torch.empty(1, dtype=torch.float32, device=a.device)
+    out = ops.mm_ex(a, b, sinv_a, sinv_b, out_fmt=out_fmt, out_ring=ring, out_amax=amax, **mm_kwargs)
+    all_reduce_amax(amax, group)
+    ops.ring_fold(ring, out_fmt, amax)
+    return out

@@ -391,18 +391,21 @@ class CMmExArgs(ctypes.Structure):
                 ("K", ctypes.c_int64), ("batch", ctypes.c_int64), ("strides", ctypes.c_void_p),
                 ("layout", ctypes.c_int), ("sinv_a", ctypes.c_void_p), ("sinv_b", ctypes.c_void_p),
                 ("bias", ctypes.c_void_p), ("bias_scale", ctypes.c_void_p), ("out_kind", ctypes.c_int),
-                ("out", ctypes.c_void_p), ("out_ring", CRing)]
+                ("out", ctypes.c_void_p), ("out_ring", CRing), ("out_amax", ctypes.c_void_p)]
 
 
 def mm_ex(a, b, sinv_a, sinv_b, bias=None, bias_scale=None, bias_fmt=E4M3, out_fmt=None, out_ring=None,
-          fmt_a=E4M3, fmt_b=E4M3, out=None, a_mn_major=False, b_mn_major=False, workspace=None, stream=None):
+          fmt_a=E4M3, fmt_b=E4M3, out=None, a_mn_major=False, b_mn_major=False, workspace=None, stream=None,
+          out_amax=None):
     """fp8_mm_ex: ``mm`` with an FP8 bias and / or an FP8 output.
 
     bias: float32 [N], or (with bias_scale, a one-element float32 CUDA tensor)
     uint8 FP8 codes [N] in format bias_fmt, dequantised as code * bias_scale.
     out_fmt: None for bf16 output, or E4M3 / E5M2 for FP8 codes of
     y * out_ring.scale, with max |y| folded into ``out_ring`` (a Ring) in the
-    same launch.  Operands and batching as ``mm``.  Returns out.
+    same launch -- or, with out_amax (a one-element float32 CUDA tensor), max |y|
+    written there and the fold left to ``ring_fold`` (a data-parallel shard).
+    Operands and batching as ``mm``.  Returns out.
     """
     if a.dtype != torch.uint8 or b.dtype != torch.uint8:
         raise ValueError("a and b hold FP8 codes as uint8")
@@ -437,7 +440,7 @@ def mm_ex(a, b, sinv_a, sinv_b, bias=None, bias_scale=None, bias_fmt=E4M3, out_f
     ring = out_ring.c() if out_ring is not None else CRing()
     args = CMmExArgs(a3.data_ptr(), b3.data_ptr(), M, N, K, batch, ctypes.cast(strides, ctypes.c_void_p), layout,
                      sinv_a.data_ptr(), sinv_b.data_ptr(), _ptr(bias), _ptr(bias_scale), kind,
-                     out3.data_ptr(), ring)
+                     out3.data_ptr(), ring, _ptr(out_amax))
     ws, wsb = (workspace.data_ptr(), workspace.numel() * workspace.element_size()) if workspace is not None else (None, 0)
     rc = (_LIB or lib()).fp8_mm_ex(ctypes.byref(args), ws, wsb, _stream(stream, a.get_device()))
     _check(rc, "fp8_mm_ex")

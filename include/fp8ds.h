@@ -408,7 +408,8 @@ int fp8_mm_pair(const fp8_mm_args* a0, const fp8_mm_args* a1, void* workspace, s
  *             output (NaN ignored) exactly as fp8_quantize folds its input's
  *             amax: next scale published, scale_inv = 1/s for the GEMM that
  *             consumes the output.  An empty output folds amax 0; K == 0
- *             gives y = bias.
+ *             gives y = bias.  With out_amax set (one rank's shard of a
+ *             data-parallel output) the fold is left to fp8_ring_fold.
  * Arguments, layouts, strides (strides[2] counts output elements), the
  * workspace and the errors are fp8_mm_ws's, plus FP8_ERR_INVALID_ARG for an
  * unknown out_kind, FP8_MM_BIAS_E5M2 without bias_scale, or an FP8 output
@@ -434,6 +435,13 @@ typedef struct {
   int out_kind;             /* fp8_mm_out */
   void* out;                /* bf16 or FP8 codes [batch, M, N] */
   fp8_ring out_ring;        /* FP8 output: the output tensor's ring */
+  float* out_amax;          /* FP8 output, data-parallel shard: NULL to fold
+                               out_ring in the launch; else the launch writes
+                               max |y| of this shard here (device float) and
+                               1/s to out_ring.scale_inv, and leaves the ring's
+                               history, idx and scale to fp8_ring_fold after a
+                               cross-rank MAX of the amax (as
+                               fp8_quantize_local) */
 } fp8_mm_ex_args;
 int fp8_mm_ex(const fp8_mm_ex_args* args, void* workspace, size_t workspace_bytes, fp8_stream_t stream);
 

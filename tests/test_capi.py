@@ -110,9 +110,10 @@ def test_mm_rejects_bad_arguments_without_cuda(L):
     assert _mm(L, N=0, A=0, B=0) == ops.FP8_OK
 
 
-def _mm_ex(L, out_kind=ops.MM_OUT_E4M3, layout=0, bias=None, bias_scale=None, out=0x30000, ring=None, M=128):
+def _mm_ex(L, out_kind=ops.MM_OUT_E4M3, layout=0, bias=None, bias_scale=None, out=0x30000, ring=None, M=128,
+           amax=None):
     args = ops.CMmExArgs(0x10000, 0x20000, M, 128, 128, 1, None, layout, 0x40000, 0x40010, bias, bias_scale,
-                         out_kind, out, ring if ring is not None else _ring())
+                         out_kind, out, ring if ring is not None else _ring(), amax)
     return L.fp8_mm_ex(ctypes.byref(args), None, 0, None)
 
 
@@ -126,6 +127,7 @@ def test_mm_ex_rejects_bad_arguments_without_cuda(L):
     assert _mm_ex(L, ring=ops.CRing(0x1000, 0x1040, 0x1044, 0x1048, 0x1054)) == ops.FP8_ERR_UNSUPPORTED
     assert _mm_ex(L, layout=ops.MM_BIAS_E5M2) == ops.FP8_ERR_INVALID_ARG    # bias format bit without FP8 bias
     assert _mm_ex(L, out_kind=ops.MM_OUT_BF16, out=0) == ops.FP8_ERR_INVALID_ARG
+    assert _mm_ex(L, out_kind=ops.MM_OUT_BF16, amax=0x50000) == ops.FP8_ERR_INVALID_ARG  # shard amax needs FP8 out
 
 
 def test_mm_ex_binding_checks_arguments_on_the_host():

@@ -164,3 +164,45 @@ def test_fp8_output_rejects_bad_arguments():
         ops.mm_ex(a, b, one, one, out_fmt=ops.E4M3)  # no ring
     with pytest.raises(ValueError):
         ops.mm_ex(a, b, one, one, bias=torch.zeros(128, device="cuda"), bias_scale=one)  # float32 bias with a scale
+
+
+def test_data_parallel_shards_fold_the_global_amax():
+    """Two row shards of one FP8 output (two data-parallel ranks emulated on
+    one GPU): each shard's launch casts with the shared ring's scale, reports
+    its own max |y| and leaves history, idx and scale alone; the MAX of the
+    two, folded with fp8_ring_fold, gives the oracle's fold of that amax, and
+    that amax is within the bound of the whole output's exact amax."""
+    from fp8_delayed_scaling_02_b200 import dp
+
+    M, N, K = 1000, 768, 1024
+    a, b = _inputs(M, N, K, seed=21)
+    bias, _, bias_ref = _bias(N, "f32", seed=4)
+    ref, S_ = OG.mm_fp8(a.numpy(), b.numpy(), ops.E4M3, ops.E4M3, 2.0 ** -7, 0.5, bias_ref)
+    ad, bd = a.cuda(), b.cuda()
+    ring = ops.Ring()
+    shards = (slice(0, 384), slice(384, M))
+    for step in range(3):
+        before = oracle_ring_from(ring)
+        amax = torch.zeros(2, dtype=torch.float32, device="cuda")
+        codes = []
+        for i, rows in enumerate(shards):
+            codes.append(ops.mm_ex(ad[rows], bd, _scalar(2.0 ** -7), _scalar(0.5), bias=bias, out_fmt=ops.E4M3,
+                                   out_ring=ring, out_amax=amax[i:i + 1]))
+        torch.cuda.synchronize()
+        hist, idx, scale, scale_inv, scratch = ring.state()
+        assert np.array_equal(hist.numpy(), before.history) and idx == before.idx  # no fold yet
+        assert np.float32(scale) == before.scale
+        assert np.float32(scale_inv) == np.float32(np.float32(1.0) / before.scale)
+        assert all(int(v) == 0 for v in scratch)
+        lo, hi = OG.out8_code_range(ref, S_, before.scale, OF.E4M3)
+        g = torch.cat(codes).cpu().numpy()
+        assert OG.codes_within(g, lo, hi, OF.E4M3).all()
+        m = amax.max().reshape(1)  # what the MAX all-reduce of the ranks computes
+        dp.all_reduce_amax(m)      # no process group here: a no-op
+        ops.ring_fold(ring, ops.E4M3, m)
+        torch.cuda.synchronize()
+        a_ref, tol = OG.amax_range(ref, S_)
+        assert abs(float(m.item()) - a_ref) <= tol
+        expect = before.copy()
+        OR.fold(expect, np.float32(m.item()), OF.E4M3)
+        assert_ring_equal(ring, expect)

@@ -112,3 +112,68 @@ def test_the_check_catches_a_local_or_summed_amax():
     summed = _ring_vector(_single_process(R.F.E4M3, lambda xf: np.float32(R.amax(xf[:ROWS]) + R.amax(xf[ROWS:])))[0])
     assert not np.array_equal(ref, local)
     assert not np.array_equal(ref, summed)
+
+
+# ---- the FP8-output GEMM's shard protocol (oracle arithmetic, gloo) ----------
+
+from oracle import gemm as OG  # noqa: E402
+
+K_GEMM, N_GEMM = 64, 48
+
+
+def _gemm_full(step):
+    a = S.fp8_codes((ROWS * WORLD, K_GEMM), seed=700 + step).numpy()
+    b = S.fp8_codes((N_GEMM, K_GEMM), seed=800).numpy()
+    return a, b
+
+
+def _gemm_worker(rank, port, results):
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=WORLD,
+                            timeout=timedelta(seconds=60))
+    try:
+        ring = R.Ring()
+        codes = []
+        for step in range(STEPS):
+            a, b = _gemm_full(step)
+            ref, _ = OG.mm_fp8(a[rank * ROWS:(rank + 1) * ROWS], b, R.F.E4M3, R.F.E4M3, 2.0 ** -6, 2.0 ** -6)
+            y = ref.astype(np.float32)  # the float64 sum is exact; every side rounds it to float32 alike
+            codes.append(R.scaled_codes(y, ring.scale, R.F.E4M3))
+            amax = torch.tensor([float(R.amax(y))], dtype=torch.float32)
+            dp.all_reduce_amax(amax)
+            R.fold(ring, np.float32(amax.item()), R.F.E4M3)
+        mine = torch.from_numpy(_ring_vector(ring))
+        rings = [torch.zeros_like(mine) for _ in range(WORLD)]
+        dist.all_gather(rings, mine)
+        results.put((rank, [r.numpy() for r in rings], np.stack(codes)))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_dp_fp8_output_rings_match_the_whole_output_fold():
+    ctx = mp.get_context("spawn")
+    results = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gemm_worker, args=(r, port, results)) for r in range(WORLD)]
+    for p in procs:
+        p.start()
+    out = {}
+    for _ in range(WORLD):
+        rank, rings, codes = results.get(timeout=180)
+        out[rank] = (rings, codes)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    ring = R.Ring()
+    ref_codes = []
+    for step in range(STEPS):
+        a, b = _gemm_full(step)
+        ref, _ = OG.mm_fp8(a, b, R.F.E4M3, R.F.E4M3, 2.0 ** -6, 2.0 ** -6)
+        y = ref.astype(np.float32)
+        ref_codes.append(R.scaled_codes(y, ring.scale, R.F.E4M3))
+        R.fold(ring, R.amax(y), R.F.E4M3)
+    ref_ring = _ring_vector(ring)
+    assert ref_ring[R.HISTORY_LEN] != 1.0  # the scale moved: the fold saw real amaxes
+    for rank, (rings, codes) in out.items():
+        for r in rings:
+            assert np.array_equal(r.astype(np.float32).view(np.uint32), ref_ring.astype(np.float32).view(np.uint32))
+        assert np.array_equal(codes, np.stack(ref_codes)[:, rank * ROWS:(rank + 1) * ROWS])

@@ -147,3 +147,30 @@ def test_mm_ex_binding_checks_arguments_on_the_host():
         ops.mm_ex(a.float(), b, one, one)  # operands are uint8 codes
     with pytest.raises(ValueError):
         ops.mm_ex(a, b, one, one, out=torch.zeros((128, 96), dtype=torch.uint8))  # bf16 output expected
+
+
+def test_paired_entry_points_reject_bad_arguments_without_cuda(L):
+    def mm_args(**kw):
+        d = dict(A=0x10000, B=0x20000, M=128, N=128, K=128, batch=1, strides=None, layout=0, sinv_a=0x40000,
+                 sinv_b=0x40010, bias=None, out_bf16=0x30000)
+        d.update(kw)
+        return ops.CMmArgs(*d.values())
+
+    good = mm_args()
+    assert L.fp8_mm_pair(None, ctypes.byref(good), None, 0, None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_mm_pair(ctypes.byref(good), ctypes.byref(mm_args(M=-1)), None, 0, None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_mm_pair(ctypes.byref(mm_args(K=24)), ctypes.byref(good), None, 0, None) == ops.FP8_ERR_UNSUPPORTED
+    assert L.fp8_mm_pair(ctypes.byref(good), ctypes.byref(mm_args(layout=1 << 10)), None, 0,
+                         None) == ops.FP8_ERR_INVALID_ARG  # the FP8-bias bit belongs to fp8_mm_ex
+
+    def q_args(**kw):
+        d = dict(inp=0x10000, dtype=0, rows=64, cols=64, layout=0, fmt=0, ring=_ring(), out=0x20000, out_t=0x30000)
+        d.update(kw)
+        return ops.CQuantArgs(*d.values())
+
+    gq = q_args()
+    assert L.fp8_quantize_pair(None, ctypes.byref(gq), None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_quantize_pair(ctypes.byref(gq), ctypes.byref(q_args(dtype=3)), None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_quantize_pair(ctypes.byref(q_args(fmt=2)), ctypes.byref(gq), None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_quantize_pair(ctypes.byref(gq), ctypes.byref(q_args(ring=ops.CRing(0, 0, 0, 0, 0))),
+                               None) == ops.FP8_ERR_INVALID_ARG

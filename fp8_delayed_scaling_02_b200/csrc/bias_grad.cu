@@ -102,7 +102,8 @@ __global__ void __cluster_dims__(kBgCluster, 1, 1) __launch_bounds__(kBgThreads)
 
 using namespace fp8ds;
 
-extern "C" int fp8_bias_grad(const void* g, int dtype, int64_t rows, int64_t cols, float* db, fp8_stream_t stream) {
+namespace fp8ds {
+int bias_grad_args_check(const void* g, int dtype, int64_t rows, int64_t cols, const float* db) {
   if (dtype < FP8_IN_BF16 || dtype > FP8_IN_FP32) return FP8_ERR_INVALID_ARG;
   if (rows < 0 || cols < 0) return FP8_ERR_INVALID_ARG;
   if (cols == 0) return FP8_OK;
@@ -112,6 +113,15 @@ extern "C" int fp8_bias_grad(const void* g, int dtype, int64_t rows, int64_t col
   if (cols > (int64_t(1) << 40) / kBgCluster || rows > (int64_t(1) << 40)) return FP8_ERR_UNSUPPORTED;
   const int64_t strips = (cols + kBgCols - 1) / kBgCols;
   if (strips * kBgCluster > INT32_MAX) return FP8_ERR_UNSUPPORTED;
+  return FP8_OK;
+}
+}  // namespace fp8ds
+
+extern "C" int fp8_bias_grad(const void* g, int dtype, int64_t rows, int64_t cols, float* db, fp8_stream_t stream) {
+  const int rc = bias_grad_args_check(g, dtype, rows, cols, db);
+  if (rc != FP8_OK) return rc;
+  if (cols == 0) return FP8_OK;
+  const int64_t strips = (cols + kBgCols - 1) / kBgCols;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const dim3 grid(unsigned(strips * kBgCluster));
   const uint8_t* gp = static_cast<const uint8_t*>(g);

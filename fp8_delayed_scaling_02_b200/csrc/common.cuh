@@ -69,6 +69,15 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 }
 __device__ __forceinline__ void pdl_wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Host-side argument checks of fp8_mm and fp8_bias_grad: the status the entry
+// point would return before launching anything (FP8_OK if it would launch).
+// The linear composites run them for every kernel they will launch before
+// they enqueue the first one, so a rejected composite changes no ring.
+int mm_args_check(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+                  const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
+                  const uint16_t* out_bf16);
+int bias_grad_args_check(const void* g, int dtype, int64_t rows, int64_t cols, const float* db);
+
 // Counts one successful kernel launch (the library-wide launch counter read
 // by fp8_launch_count).
 void note_launch();

@@ -1446,6 +1446,15 @@ int mm_run(MmProblem& q, void* workspace, size_t ws_bytes, cudaStream_t st) {
 }  // namespace
 }  // namespace fp8ds
 
+namespace fp8ds {
+int mm_args_check(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
+                  const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
+                  const uint16_t* out_bf16) {
+  MmProblem q;
+  return mm_validate(A, B, M, N, K, batch, strides, layout, sinv_a, sinv_b, bias, const_cast<uint16_t*>(out_bf16), q);
+}
+}  // namespace fp8ds
+
 static int mm_impl(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
                    const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
                    uint16_t* out_bf16, void* workspace, size_t ws_bytes, fp8_stream_t stream) {

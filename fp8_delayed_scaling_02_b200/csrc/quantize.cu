@@ -1309,11 +1309,11 @@ extern "C" int fp8_quantize_current(const void* in, int dtype, int64_t rows, int
 // plugin interfaces that hand over only input and output pointers, and
 // deployments that reserve all device memory at start-up (a cudaMalloc at run
 // time can also synchronise the device and stall other streams).  For them
-// fp8_quantize_static_scratch keeps the two scratch words that fp8_quantize
-// takes from ring.scratch (the amax bits and the block ticket) in the
-// library-owned array below instead.  Each GPU that loads the library holds
-// these 256 bytes until the process exits.  All calls on a device share the
-// array, so calls that overlap on the GPU race with each other.
+// fp8_quantize_static_scratch keeps the four scratch words that fp8_quantize
+// takes from ring.scratch (amax bits, block ticket, tile counter, spare) in
+// the library-owned array below instead.  Each GPU that loads the library
+// holds these 256 bytes until the process exits.  All calls on a device share
+// the array, so calls that overlap on the GPU race with each other.
 
 #include <mutex>
 
@@ -1328,7 +1328,9 @@ uint32_t* g_static_scratch_ptr[64] = {nullptr};
 
 // Device address of the static array on the current device, looked up once per
 // device with that device current.  Host code must not use the symbol itself:
-// on the host it is only a stand-in, not a device address.
+// on the host it is only a stand-in, not a device address.  A device reset
+// (cudaDeviceReset) unloads the module and makes the cached address stale;
+// the header says that this entry point must not be used after one.
 uint32_t* static_scratch_on_current_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
@@ -1346,20 +1348,17 @@ extern "C" int fp8_quantize_static_scratch(const void* in, int dtype, int64_t ro
                                            int fmt, fp8_ring ring, uint8_t* out, uint8_t* out_t,
                                            fp8_stream_t stream) {
   if (kQuantizeScratchWords > kStaticScratchWords) return FP8_ERR_UNSUPPORTED;
-  // The argument checks that need no device run first, so a rejected call
-  // enqueues nothing.
-  if (dtype < FP8_IN_BF16 || dtype > FP8_IN_FP32) return FP8_ERR_INVALID_ARG;
-  if (fmt != FP8_E4M3 && fmt != FP8_E5M2) return FP8_ERR_INVALID_ARG;
-  if (layout < FP8_LAYOUT_ROW || layout > FP8_LAYOUT_DUAL) return FP8_ERR_INVALID_ARG;
-  if (rows < 0 || cols < 0) return FP8_ERR_INVALID_ARG;
   if (!ring.history || !ring.idx || !ring.scale || !ring.scale_inv) return FP8_ERR_INVALID_ARG;
   uint32_t* scratch = static_scratch_on_current_device();
   if (scratch == nullptr) return FP8_ERR_CUDA;
-  // The kernel leaves both words at zero when it finishes; clearing them here
+  // Every argument check of fp8_quantize runs before the memset, so a
+  // rejected call enqueues nothing.
+  const int rc = check_quantize_args(in, dtype, rows, cols, layout, fmt, out, out_t, scratch);
+  if (rc != FP8_OK) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // The kernel leaves the words at zero when it finishes; clearing them here
   // as well means a call never depends on what an earlier call left behind.
-  if (cudaMemsetAsync(scratch, 0, kQuantizeScratchWords * sizeof(uint32_t),
-                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
-    return FP8_ERR_CUDA;
-  ring.scratch = scratch;
-  return fp8_quantize(in, dtype, rows, cols, layout, fmt, ring, out, out_t, stream);
+  if (cudaMemsetAsync(scratch, 0, kQuantizeScratchWords * sizeof(uint32_t), st) != cudaSuccess) return FP8_ERR_CUDA;
+  const RingArgs r{ring.history, ring.idx, ring.scale, ring.scale_inv, scratch};
+  return quantize_dispatch(in, dtype, rows, cols, layout, fmt, r, out, out_t, st);
 }

@@ -30,14 +30,17 @@ def _gen(seed):
     return g
 
 
-def normal_with_outliers(shape, seed, std=1.0, frac=0.0, mult=1.0, dtype="bf16"):
-    """N(0, std^2) values; a Bernoulli(frac) mask (same generator) multiplies entries by ``mult``."""
-    g = _gen(seed)
+def _normal_outliers_from(g, shape, std, frac, mult, dtype):
     x = torch.randn(shape, generator=g, dtype=torch.float32) * std
     if frac > 0:
         mask = torch.rand(shape, generator=g) < frac
         x = torch.where(mask, x * mult, x)
     return x.to(_DTYPES[dtype] if isinstance(dtype, str) else dtype)
+
+
+def normal_with_outliers(shape, seed, std=1.0, frac=0.0, mult=1.0, dtype="bf16"):
+    """N(0, std^2) values; a Bernoulli(frac) mask (same generator) multiplies entries by ``mult``."""
+    return _normal_outliers_from(_gen(seed), shape, std, frac, mult, dtype)
 
 
 def uniform(shape, seed, lo=-1.0, hi=1.0):
@@ -66,9 +69,14 @@ def fp8_codes(shape, seed, fmt=E4M3):
 # --- named workloads -------------------------------------------------------
 
 def linear_pr1_step(step):
-    """One step of the small PR1 linear: X [128,512], W [256,512] (seed = step), bias seed 0."""
-    x = normal_with_outliers((128, 512), seed=1000 + step, frac=0.01, mult=20.0)
-    w = normal_with_outliers((256, 512), seed=2000 + step, frac=0.01, mult=20.0)
+    """One step of the small PR1 linear, steps 0, 1, 2 with fresh seeds 0, 1, 2.
+
+    One generator seeded with the step draws X [128,512] and then W [256,512]
+    (values, then the outlier mask, for each); the bias comes from seed 0.
+    """
+    g = _gen(step)
+    x = _normal_outliers_from(g, (128, 512), 1.0, 0.01, 20.0, "bf16")
+    w = _normal_outliers_from(g, (256, 512), 1.0, 0.01, 20.0, "bf16")
     bias = uniform((256,), seed=0)
     return x, w, bias
 

@@ -135,13 +135,17 @@ int fp8_quantize(const void* in, int dtype, int64_t rows, int64_t cols, int layo
  *     array holds would return FP8_ERR_UNSUPPORTED.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept for the life of the
+ *     process: after a cudaDeviceReset of that device the kept address is
+ *     stale, so do not call this entry point again after a reset.
  *   - All calls on a device share the array.  Each call clears the four words
  *     on `stream` before its kernel, and the kernel leaves them at zero, but
  *     two calls that overlap on the GPU (different streams, no ordering
  *     between them) race on the array and give wrong amax and scales.
  *   - Errors are those of fp8_quantize, plus FP8_ERR_CUDA if the array's
- *     address cannot be obtained or the clearing memset fails.
+ *     address cannot be obtained or the clearing memset fails.  Every
+ *     argument check runs before the clearing memset, so a rejected call
+ *     enqueues nothing.
  */
 int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,
                                 fp8_ring ring, uint8_t* out, uint8_t* out_t, fp8_stream_t stream);
@@ -310,8 +314,11 @@ int fp8_mm(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, 
  * again in between).  dx, dw or db may be NULL to skip that output.
  * Sizes: K % 16 == 0 (forward); backward also M % 16 == 0 (dW reduces over
  * tokens) and N % 16 == 0 (MN-major row pitch).
- * Errors: those of the calls it makes; the first failure is returned and
- * the later steps are not launched.
+ * Errors: those of the calls it makes.  Every argument check of every call
+ * (the quantize, each GEMM, the bias gradient) runs on the host before the
+ * first kernel is enqueued, so a call rejected with FP8_ERR_INVALID_ARG or
+ * FP8_ERR_UNSUPPORTED launched nothing and left every ring as it was.  Only
+ * FP8_ERR_CUDA can come after earlier steps were launched.
  */
 int fp8_linear_forward(const void* x, int x_dtype, const void* w, int w_dtype, int64_t M, int64_t N, int64_t K,
                        const float* bias, fp8_ring ring_x, fp8_ring ring_w, uint8_t* xq, uint8_t* wq, uint16_t* y,

@@ -19,7 +19,11 @@ What one quantize call computes, in the pages' order:
    transpose), DUAL writes both from the same values.
 5. Ring fold ("tests/extension" page, ring commit: the last block folds amax
    into the history window and publishes the next scale):
-   ``hist[idx] = amax; idx = (idx + 1) mod 16; m = max(hist)``;
+   ``hist[idx] = amax; idx = (idx + 1) mod 16; m = max(hist)``, where
+   the maximum ignores NaN entries exactly as the amax of step 2 ignores
+   NaN elements, and is 0 when every entry is NaN (reading: the pages state
+   no NaN rule; a NaN can only reach the history through a caller-supplied
+   amax, the data-parallel fold of a MAX-reduced amax);
    ``scale' = fp32(FP8_MAX / m)`` if m is positive and finite and the
    quotient is finite, else the scale is kept (a zero history keeps the
    previous scale).
@@ -87,7 +91,8 @@ def fold(ring, a, fmt):
     s_used = np.float32(ring.scale)
     ring.history[ring.idx] = np.float32(a)
     ring.idx = (ring.idx + 1) % HISTORY_LEN
-    m = np.float32(np.max(ring.history))
+    h = ring.history[~np.isnan(ring.history)]
+    m = np.float32(np.max(h)) if h.size else np.float32(0.0)
     fmax = np.float32(F.fp8_max(fmt))
     if m > 0 and np.isfinite(m):
         with np.errstate(over="ignore"):

@@ -174,3 +174,44 @@ def test_paired_entry_points_reject_bad_arguments_without_cuda(L):
     assert L.fp8_quantize_pair(ctypes.byref(q_args(fmt=2)), ctypes.byref(gq), None) == ops.FP8_ERR_INVALID_ARG
     assert L.fp8_quantize_pair(ctypes.byref(gq), ctypes.byref(q_args(ring=ops.CRing(0, 0, 0, 0, 0))),
                                None) == ops.FP8_ERR_INVALID_ARG
+
+
+def test_linear_composites_check_every_call_before_launching(L):
+    """A linear call that one of its GEMMs (or the bias gradient) would reject
+    returns that status before any kernel is enqueued, so its rings stay as
+    they were.  With no GPU here, a quantize enqueued first would have failed
+    with FP8_ERR_CUDA instead."""
+    vp = ctypes.c_void_p
+    ring = _ring()
+
+    def fwd(M=128, N=128, K=128, xq=0x50000, wq=0x60000, y=0x70000, x=0x10000, w=0x20000):
+        return L.fp8_linear_forward(vp(x), 0, vp(w), 0, M, N, K, None, ring, _ring(0x1100), vp(xq), vp(wq), vp(y),
+                                    None)
+
+    assert fwd(K=24) == ops.FP8_ERR_UNSUPPORTED          # K % 16
+    assert fwd(y=0) == ops.FP8_ERR_INVALID_ARG           # no output
+    assert fwd(xq=0x50008) == ops.FP8_ERR_UNSUPPORTED     # FP8 operand not 16-byte aligned
+    assert fwd(y=0x70001) == ops.FP8_ERR_UNSUPPORTED      # bf16 output not 2-byte aligned
+
+    def bwd(M=128, N=128, K=128, dx=0x80000, dw=0x90000, db=0xA0000, g=0x10000, gq=0x30000, g_dtype=0):
+        return L.fp8_linear_backward(vp(g), g_dtype, M, N, K, ring, vp(0x50000), vp(0x60000), vp(0x40000),
+                                     vp(0x40010), vp(gq), vp(dx) if dx else None, vp(dw) if dw else None,
+                                     vp(db) if db else None, None)
+
+    assert bwd(M=24) == ops.FP8_ERR_UNSUPPORTED           # dW reduces over M: M % 16
+    assert bwd(N=40) == ops.FP8_ERR_UNSUPPORTED           # dX reduces over N: N % 16
+    assert bwd(N=40, dx=0) == ops.FP8_ERR_UNSUPPORTED     # dW's MN-major A needs N % 16 too
+    assert bwd(K=24, dw=0) == ops.FP8_ERR_UNSUPPORTED     # dX's MN-major B needs K % 16
+    assert bwd(gq=0x30008) == ops.FP8_ERR_UNSUPPORTED     # Gq is a GEMM operand: 16-byte aligned
+    assert bwd(g=0x10001) == ops.FP8_ERR_UNSUPPORTED      # bias gradient input alignment
+    assert bwd(g_dtype=2, g=0x10002, dx=0, dw=0) == ops.FP8_ERR_UNSUPPORTED  # fp32 G, 4-byte alignment
+
+
+def test_static_scratch_entry_point_checks_before_cuda(L):
+    """Argument errors that need no device come back before any CUDA call."""
+    f = L.fp8_quantize_static_scratch
+    vp = ctypes.c_void_p
+    f.argtypes = [vp, ctypes.c_int, ctypes.c_int64, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ops.CRing, vp, vp,
+                  vp]
+    f.restype = ctypes.c_int
+    assert f(vp(0x4000), 0, 4, 4, 0, 0, ops.CRing(0, 0, 0, 0, 0), vp(0x2000), None, None) == ops.FP8_ERR_INVALID_ARG

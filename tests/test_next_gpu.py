@@ -166,3 +166,23 @@ def test_dp_two_shards_match_the_whole_tensor():
         r_out, r_out_t, _ = OR.quantize(full, OR.F.E4M3, OR.DUAL, ref)
         assert_bytes_equal(o, r_out, "out")
     assert_ring_equal(rr, ref)
+
+
+def test_ring_fold_of_a_nan_amax_matches_the_oracle():
+    """A caller-supplied NaN amax (a data-parallel fold) is stored in its slot
+    and skipped by the window maximum on both sides; the scales stay those of
+    the finite entries.  Then a finite fold, then a ring whose only entry is
+    NaN (the scale is kept)."""
+    for fmt in (ops.E4M3, ops.E5M2):
+        ring, ref = ops.Ring(), OR.Ring()
+        for a in (3.0, float("nan"), 0.75, float("nan"), 7.5):
+            amax = torch.tensor([a], dtype=torch.float32, device="cuda")
+            ops.ring_fold(ring, fmt, amax)
+            OR.fold(ref, np.float32(a), fmt)
+            torch.cuda.synchronize()
+            assert_ring_equal(ring, ref)
+        only, ref_only = ops.Ring(scale=0.625), OR.Ring(scale=0.625)
+        ops.ring_fold(only, fmt, torch.tensor([float("nan")], dtype=torch.float32, device="cuda"))
+        OR.fold(ref_only, np.float32("nan"), fmt)
+        torch.cuda.synchronize()
+        assert_ring_equal(only, ref_only)

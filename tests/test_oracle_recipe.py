@@ -168,3 +168,55 @@ def test_no_scale_ratio_leak_across_steps():
         normal = np.abs(x * used) >= 2.0 ** -6
         sel = in_range & normal
         assert np.all(np.abs(deq[sel] - x[sel]) <= np.abs(x[sel]) * 2.0 ** -4 + 1e-30)
+
+
+def test_nan_history_entry_is_ignored_by_the_window_max():
+    """A NaN amax (only a caller-supplied amax can be one) is stored in its slot
+    and skipped by the window maximum, like NaN elements in the amax itself:
+    the scale is the one the same history without that entry gives, computed
+    here with exact rationals."""
+    for fmt, fmax in ((F.E4M3, 448), (F.E5M2, 57344)):
+        ring = R.Ring()
+        R.fold(ring, np.float32(3.0), fmt)
+        s_before = ring.scale
+        R.fold(ring, np.float32(np.nan), fmt)
+        assert np.isnan(ring.history[1]) and ring.idx == 2
+        assert _bits(ring.scale) == _bits(s_before) == _bits(_f32_rn(Fraction(fmax) / Fraction(3)))
+        R.fold(ring, np.float32(0.75), fmt)  # a smaller finite amax: the max stays 3
+        assert _bits(ring.scale) == _bits(_f32_rn(Fraction(fmax) / Fraction(3)))
+        # Only NaN in the window: the maximum is 0 and the scale is kept.
+        only = R.Ring(scale=0.625)
+        R.fold(only, np.float32(np.nan), fmt)
+        assert only.scale == np.float32(0.625) and only.scale_inv == np.float32(1.6)
+
+
+@pytest.mark.parametrize("layout", [R.ROW, R.TRANSPOSED, R.DUAL])
+@pytest.mark.parametrize("fmt", [F.E4M3, F.E5M2])
+def test_quantize_local_then_fold_equals_quantize(layout, fmt):
+    """The data-parallel split of a call: quantize_local leaves the ring alone,
+    casts with the ring's scale and returns the raw amax and 1/scale; folding
+    that amax gives the ring of one quantize call, and the codes are its codes.
+    Checked over 5 delayed steps whose amax moves by orders of magnitude, so a
+    cast with the post-fold scale or a stale scale_inv is caught."""
+    ring_a, ring_b = R.Ring(), R.Ring()
+    for step in range(5):
+        g = torch.Generator().manual_seed(step)
+        x = (torch.randn((37, 53), generator=g) * 10.0 ** (2 * (step % 3) - 2)).to(torch.bfloat16)
+        before = (ring_b.history.copy(), ring_b.idx, ring_b.scale, ring_b.scale_inv)
+        o1, t1, a1 = R.quantize(x, fmt, layout, ring_a)
+        o2, t2, a2, sinv = R.quantize_local(x, fmt, layout, ring_b)
+        assert np.array_equal(ring_b.history, before[0]) and ring_b.idx == before[1]
+        assert ring_b.scale == before[2] and ring_b.scale_inv == before[3], "quantize_local must not touch the ring"
+        assert _bits(a2) == _bits(np.max(np.abs(x.float().numpy())))
+        assert _bits(sinv) == _bits(_f32_rn(1 / Fraction(float(ring_b.scale))))
+        R.fold(ring_b, a2, fmt)
+        for u, v in ((o1, o2), (t1, t2)):
+            assert (u is None) == (v is None)
+            if u is not None:
+                assert np.array_equal(u, v)
+        assert _bits(a1) == _bits(a2)
+        assert np.array_equal(ring_a.history.view(np.uint32), ring_b.history.view(np.uint32))
+        assert ring_a.idx == ring_b.idx
+        assert _bits(ring_a.scale) == _bits(ring_b.scale) and _bits(ring_a.scale_inv) == _bits(ring_b.scale_inv)
+        assert _bits(ring_b.scale_inv) == _bits(sinv)
+    assert ring_b.scale != np.float32(1.0)

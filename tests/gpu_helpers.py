@@ -53,6 +53,34 @@ def quantize_both(x_cpu, fmt, layout, ring_gpu, misalign=False):
     return out, out_t, r_out, r_out_t, ref_ring
 
 
+def oracle_codes(x_cpu, scale, fmt):
+    """The oracle's codes encode(fp32(x * scale)) of a CPU tensor, element by element.
+
+    A bf16 or fp16 tensor holds at most 65536 distinct values, so the oracle
+    (``OR.scaled_codes``) is applied once to every 16-bit pattern and the
+    result is looked up by each element's bit pattern: the same function,
+    evaluated once per distinct input instead of once per element.  float32
+    inputs go through ``OR.scaled_codes`` directly."""
+    if x_cpu.dtype in (torch.bfloat16, torch.float16):
+        pats = torch.arange(1 << 16, dtype=torch.int32).to(torch.int16).view(x_cpu.dtype)
+        table = OR.scaled_codes(OR.to_float32(pats), np.float32(scale), fmt)
+        bits = x_cpu.contiguous().view(torch.int16).numpy().view(np.uint16)
+        return table[bits]
+    return OR.scaled_codes(OR.to_float32(x_cpu), np.float32(scale), fmt)
+
+
+def band_rows(M, seed, band=128):
+    """Output rows that hit every 128-row band of an M-row result: each band's
+    first and last row and one drawn at random inside it, so every M tile (and
+    each half of a 256-row CTA-pair tile) is compared."""
+    rng = np.random.default_rng(seed)
+    rows = []
+    for b0 in range(0, M, band):
+        b1 = min(b0 + band, M) - 1
+        rows += [b0, b1, int(rng.integers(b0, b1 + 1))]
+    return np.unique(np.array(rows, dtype=np.int64))
+
+
 def assert_bytes_equal(gpu, ref, what):
     g = gpu.cpu().numpy()
     assert g.shape == ref.shape, (what, g.shape, ref.shape)
@@ -78,4 +106,5 @@ def f32(t):
     return float(t.cpu().item())
 
 
-__all__ = ["require_gpu", "quantize_both", "assert_ring_equal", "assert_bytes_equal", "mm_check", "OF", "OG", "OR"]
+__all__ = ["require_gpu", "quantize_both", "assert_ring_equal", "assert_bytes_equal", "mm_check", "oracle_codes",
+           "band_rows", "OF", "OG", "OR"]

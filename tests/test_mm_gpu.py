@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from fp8_delayed_scaling_02_b200 import ops, synthetic as S
-from gpu_helpers import OG, OR, mm_check, require_gpu
+from gpu_helpers import OG, OR, band_rows, mm_check, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -45,16 +45,17 @@ def test_mixed_formats(fa, fb):
     _run(256, 384, 512, fmt_a=fa, fmt_b=fb, with_bias=True, sa=2.0 ** -10, sb=3.5)
 
 
-# Square sweep; full comparison up to 2048^3, sampled rows above.
+# Square sweep; full comparison up to 2048^3, above it three rows of every
+# 128-row band (each M tile and each half of a CTA-pair tile; every row spans
+# all N tiles).
 @pytest.mark.parametrize("n", [512, 1024, 1152, 2048, 3072, 4096, 8192])
 def test_square_sweep(n):
-    rows = None if n <= 2048 else np.unique(np.random.default_rng(n).integers(0, n, 24))
+    rows = None if n <= 2048 else band_rows(n, seed=n)
     _run(n, n, n, with_bias=(n % 3 == 0 or n == 1024), seed=n, rows=rows)
 
 
 def test_square_8192_scaled_with_bias():
-    rows = np.array([0, 1, 127, 128, 4095, 8191])
-    _run(8192, 8192, 8192, sa=0.37, sb=0.125, with_bias=True, seed=5, rows=rows)
+    _run(8192, 8192, 8192, sa=0.37, sb=0.125, with_bias=True, seed=5, rows=band_rows(8192, seed=5))
 
 
 def test_skinny_and_odd():
@@ -90,8 +91,8 @@ def test_batched_and_broadcast():
     y = ops.mm(a, b, sa, sb, bias.cuda())
     torch.cuda.synchronize()
     assert y.shape == (8, 1024, 2048)
-    rows = np.array([0, 5, 511, 1023])
-    for z in (0, 3, 7):
+    rows = band_rows(1024, seed=25)
+    for z in range(8):
         ref, Ssum = OG.mm_fp8_rows(a[z].cpu().numpy(), b[0].cpu().numpy(), 0, 0, sa.item(), sb.item(),
                                    bias.numpy(), rows)
         ok, ratio = OG.check(y[z].float().cpu().numpy()[rows], ref, Ssum)
@@ -162,9 +163,9 @@ def test_mn_major_backward_shapes_mixed_formats():
     dx = ops.mm(g.cuda(), w.cuda(), _scalar(0.01), _scalar(2.0), fmt_a=ops.E5M2, b_mn_major=True)
     dw = ops.mm(g.cuda(), x.cuda(), _scalar(0.01), _scalar(0.5), fmt_a=ops.E5M2, a_mn_major=True, b_mn_major=True)
     torch.cuda.synchronize()
-    rows = np.array([0, 1, 255, 511])
+    rows = band_rows(512, seed=1)
     mm_check(dx, g.numpy(), w.numpy().T.copy(), ops.E5M2, ops.E4M3, np.float32(0.01), np.float32(2.0), None, rows)
-    rows = np.array([0, 100, 4095])
+    rows = band_rows(4096, seed=2)
     mm_check(dw, g.numpy().T.copy(), x.numpy().T.copy(), ops.E5M2, ops.E4M3, np.float32(0.01), np.float32(0.5),
              None, rows)
 
@@ -210,7 +211,7 @@ def test_split_k_workspace(M, N, K, a_mn, b_mn):
     torch.cuda.synchronize()
     assert torch.equal(y1, y2), "stream-K must be deterministic"
     assert int(ws[:1024].count_nonzero()) == 0, "piece flags (the first 1024 bytes) must return to zero"
-    rows = np.unique(np.concatenate([np.random.default_rng(M).integers(0, M, 16), [0, M - 1]]))
+    rows = band_rows(M, seed=M)
     for y in (y1, y3):
         mm_check(y, a.numpy(), b.numpy(), ops.E4M3, ops.E4M3, np.float32(0.37), np.float32(0.125), bias.numpy(),
                  rows)
@@ -245,7 +246,7 @@ def test_mm_pair_matches_the_oracle(c0, c1):
     y0, y1 = ops.mm_pair(probs[0], probs[1])
     torch.cuda.synchronize()
     for y, (a, b, bias, M, i) in zip((y0, y1), refs):
-        rows = np.unique(np.concatenate([np.random.default_rng(M + i).integers(0, M, 12), [0, M - 1]]))
+        rows = band_rows(M, seed=M + i)
         mm_check(y, a.numpy(), b.numpy(), ops.E5M2 if i == 1 else ops.E4M3, ops.E4M3, np.float32(0.5 + i),
                  np.float32(0.25), None if bias is None else bias.numpy(), rows)
 

@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from fp8_delayed_scaling_02_b200 import ops, synthetic as S
-from gpu_helpers import OR, assert_bytes_equal, assert_ring_equal, quantize_both, require_gpu
+from gpu_helpers import OR, assert_bytes_equal, assert_ring_equal, oracle_codes, quantize_both, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -17,6 +17,14 @@ LAYOUTS = [ops.ROW, ops.TRANSPOSED, ops.DUAL]
 @pytest.fixture(autouse=True)
 def _gpu():
     require_gpu()
+
+
+def _dev(x, misalign):
+    if not misalign:
+        return x.cuda()
+    flat = torch.empty(x.numel() + 1, dtype=x.dtype, device="cuda")
+    flat[1:].copy_(x.reshape(-1))
+    return flat[1:].view(x.shape)
 
 
 def _run_and_compare(x, fmt, layout, ring, misalign=False):
@@ -112,43 +120,79 @@ def test_every_16bit_input_pattern(dtype, fmt, layout):
 
 
 # Full sizes of the quantize bandwidth sweep, in the launch configuration the
-# bench times; bytes compared on sampled rows, amax / ring / scales in full.
-FULL = [(128, 1536), (2048, 1536), (8192, 1536), (16384, 4096), (2048, 1537), (8192, 1537)]
+# bench times.  Every byte of out / out_t is compared with the oracle, and the
+# ring bit for bit.  Each case runs the three layouts from the same ring state
+# (one oracle evaluation serves all three) and then a second, delayed step.
+FULL = [(128, 1536), (2048, 1536), (8192, 1536), (2048, 1537), (8192, 1537)]
+VALUE_SCALES = [1.0, 1e-3, 1e3]
+
+
+def _full_case(rows, cols, dtype, fmt, misalign, vs, seed):
+    x = S.quant_sweep_input(rows, cols, dtype, vs, seed=seed)
+    xd = _dev(x, misalign)
+    rings = {lay: ops.Ring() for lay in LAYOUTS}
+    ref = OR.Ring()
+    xf = OR.to_float32(x)
+    a = OR.amax(xf)
+    for step in range(2):
+        got = {lay: ops.quantize(xd, fmt, lay, rings[lay]) for lay in LAYOUTS}
+        torch.cuda.synchronize()
+        codes = oracle_codes(x, ref.scale, fmt)
+        codes_t = np.ascontiguousarray(codes.T)
+        OR.fold(ref, a, fmt)
+        what = f"{rows}x{cols} {dtype} fmt{fmt} misalign={misalign} x{vs} step {step}"
+        for lay, (out, out_t) in got.items():
+            if out is not None:
+                assert_bytes_equal(out, codes, f"out, layout {lay}, {what}")
+            if out_t is not None:
+                assert_bytes_equal(out_t, codes_t, f"out_t, layout {lay}, {what}")
+            assert_ring_equal(rings[lay], ref)
 
 
 @pytest.mark.parametrize("shape", FULL)
-@pytest.mark.parametrize("layout", LAYOUTS)
-def test_full_size_sampled(shape, layout):
+@pytest.mark.parametrize("dtype", DTYPES)
+def test_full_size_whole_tensor(shape, dtype):
+    """The whole dtype x format x base alignment x value-scale product."""
     rows, cols = shape
-    rng = np.random.default_rng(rows + cols + layout)
-    sample = np.unique(np.concatenate([rng.integers(0, rows, 24), [0, rows - 1]]))
-    for dtype, fmt, misalign, vs in (("bf16", ops.E4M3, False, 1.0), ("fp32", ops.E5M2, True, 1e3),
-                                     ("fp16", ops.E4M3, True, 1e-3), ("fp32", ops.E4M3, False, 1.0)):
-        x = S.quant_sweep_input(rows, cols, dtype, vs, seed=rows ^ cols)
-        ring = ops.Ring()
-        for step in range(2):
-            ref_ring = OR.Ring()
-            hist, idx, sc, si, _ = ring.state()
-            ref_ring.history, ref_ring.idx = hist.numpy().astype(np.float32), idx
-            ref_ring.scale, ref_ring.scale_inv = np.float32(sc), np.float32(si)
-            if misalign:
-                flat = torch.empty(x.numel() + 1, dtype=x.dtype, device="cuda")
-                flat[1:].copy_(x.reshape(-1))
-                xd = flat[1:].view(x.shape)
-            else:
-                xd = x.cuda()
-            out, out_t = ops.quantize(xd, fmt, layout, ring)
-            torch.cuda.synchronize()
-            xf = OR.to_float32(x)
-            s_used = np.float32(ref_ring.scale)
-            ref_rows = OR.scaled_codes(xf[sample], s_used, fmt)
-            OR.fold(ref_ring, OR.amax(xf), fmt)
-            if out is not None:
-                assert_bytes_equal(out[torch.as_tensor(sample, device="cuda")], ref_rows, "out rows")
-            if out_t is not None:
-                assert_bytes_equal(out_t[:, torch.as_tensor(sample, device="cuda")].t().contiguous(), ref_rows,
-                                   "out_t columns")
-            assert_ring_equal(ring, ref_ring)
+    for fmt in FMTS:
+        for misalign in (False, True):
+            for vs in VALUE_SCALES:
+                _full_case(rows, cols, dtype, fmt, misalign, vs, seed=(rows ^ cols) + int(misalign) + 7 * fmt)
+
+
+@pytest.mark.parametrize("dtype,fmt,misalign,vs", [("bf16", ops.E4M3, False, 1.0), ("fp16", ops.E5M2, True, 1e-3),
+                                                   ("fp32", ops.E4M3, True, 1e3)])
+def test_full_size_whole_tensor_67M(dtype, fmt, misalign, vs):
+    """16384 x 4096 (67M elements: every TMA tile claim of a multi-wave launch)."""
+    _full_case(16384, 4096, dtype, fmt, misalign, vs, seed=16384 + int(misalign))
+
+
+def _fp32_rounding_boundaries():
+    """Every sign, exponent and top-12 mantissa pattern of float32 with the low
+    11 bits at 0, 1, 0x400 or 0x7FF (NaN removed): every tie between two FP8
+    neighbours of either format, one float32 ulp either side of it, and every
+    exact code, about 8.4M values."""
+    hi = np.arange(1 << 21, dtype=np.uint32) << np.uint32(11)
+    u = np.concatenate([hi | np.uint32(low) for low in (0, 1, 0x400, 0x7FF)])
+    x = u.view(np.float32)
+    x = x[~np.isnan(x)]
+    pad = (-x.size) % 2048
+    return torch.from_numpy(np.concatenate([x, np.zeros(pad, dtype=np.float32)]).reshape(-1, 2048))
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("scale", [1.0, 0.3])
+def test_fp32_rounding_boundaries(fmt, scale):
+    """The hardware cast on float32 inputs at every rounding boundary, through
+    fp8_quantize (row layout), against the oracle's encoder byte for byte."""
+    x = _fp32_rounding_boundaries()
+    ring = ops.Ring(scale=scale)
+    out, _ = ops.quantize(x.cuda(), fmt, ops.ROW, ring)
+    torch.cuda.synchronize()
+    assert_bytes_equal(out, OR.scaled_codes(x.numpy(), np.float32(scale), fmt), f"fp32 boundaries fmt{fmt} x{scale}")
+    ref = OR.Ring(scale=scale)
+    OR.fold(ref, OR.amax(x.numpy()), fmt)
+    assert_ring_equal(ring, ref)
 
 
 @pytest.mark.parametrize("dtype", DTYPES)
@@ -186,14 +230,6 @@ QPAIR = [
     (((256, 512), "bf16", 0, False), ((256, 512), "bf16", 1, False), ops.DUAL),
     (((0, 9), "bf16", 0, False), ((64, 64), "bf16", 0, False), ops.DUAL),
 ]
-
-
-def _dev(x, misalign):
-    if not misalign:
-        return x.cuda()
-    flat = torch.empty(x.numel() + 1, dtype=x.dtype, device="cuda")
-    flat[1:].copy_(x.reshape(-1))
-    return flat[1:].view(x.shape)
 
 
 @pytest.mark.parametrize("s0,s1,layout", QPAIR)

@@ -114,9 +114,23 @@ bool encode_tiled_cached(void* map, int data_type, int rank, const void* base, c
 namespace fp8ds {
 namespace {
 std::atomic<unsigned long long> g_launches{0};
+std::atomic<unsigned long long> g_wait_budget_ns{kWaitBudgetNs};
+std::atomic<uint32_t> g_stall_site{0};
 }  // namespace
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+WaitCfg wait_cfg() {
+  return WaitCfg{g_wait_budget_ns.load(std::memory_order_relaxed), g_stall_site.load(std::memory_order_relaxed)};
+}
 }  // namespace fp8ds
+
+extern "C" int fp8_debug_wait(uint64_t budget_ns, uint32_t stall_site) {
+  if (budget_ns == 0 || budget_ns > fp8ds::kWaitBudgetNs) return FP8_ERR_INVALID_ARG;
+  if (stall_site != 0 && stall_site != fp8ds::kWaitEpilogueTmemFull && stall_site != fp8ds::kWaitQuantizeTma)
+    return FP8_ERR_INVALID_ARG;
+  fp8ds::g_wait_budget_ns.store(budget_ns, std::memory_order_relaxed);
+  fp8ds::g_stall_site.store(stall_site, std::memory_order_relaxed);
+  return FP8_OK;
+}
 
 extern "C" uint64_t fp8_launch_count(void) { return fp8ds::g_launches.load(std::memory_order_relaxed); }
 

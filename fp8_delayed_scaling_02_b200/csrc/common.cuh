@@ -46,8 +46,20 @@ void* tensor_map_encoder();
 bool encode_tiled_cached(void* map, int data_type, int rank, const void* base, const uint64_t* dims,
                          const uint64_t* strides, const uint32_t* box, int swizzle, int l2_promotion);
 
-// Nanosecond budget of every bounded wait in a kernel.
+// Nanosecond budget of every bounded wait in a kernel (the default).
 constexpr unsigned long long kWaitBudgetNs = 2000000000ull;  // 2 s
+
+// What launches take for their bounded waits: the budget of every wait on
+// another role's or CTA's progress, and the one wait site (0: none) at which
+// kernels wait on a barrier that nothing completes, so that the wait runs out
+// and the kernel's timeout path runs.  Only fp8_debug_wait changes them (for
+// tests of that path); waits that drain a kernel's own copies and MMAs before
+// it frees shared memory or TMEM always keep kWaitBudgetNs.
+struct WaitCfg {
+  unsigned long long budget_ns;
+  uint32_t stall_site;
+};
+WaitCfg wait_cfg();  // defined in capi.cu
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;

@@ -66,7 +66,8 @@ struct Cfg {
   static constexpr int kBarOffset = kStagingOffset + kEpiWarps * 2 * kStagingBytes;
   static constexpr int kSmemBytes = kBarOffset + 256 + 1024;  // + barriers + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert((2 * kStages + 5) * 8 + 16 + 4 * kEpiWarps <= 256, "barrier area: barriers, TMEM slot, abort, amax");
+  static_assert((2 * kStages + 5) * 8 + 16 + 4 * kEpiWarps + 8 <= 256,
+                "barrier area: barriers, TMEM slot, abort, amax, stall barrier");
 };
 
 struct MmParams {
@@ -97,6 +98,8 @@ struct MmParams {
   int bias_vec;      // bias is 16-byte aligned
   uint32_t idesc;
   uint32_t* err;
+  unsigned long long wait_ns;  // budget of the waits on another role's progress
+  uint32_t stall;              // wait site that waits on a never-completed barrier (testing), else 0
   // Epilogue variants (kernel template EPI): an FP8 bias, dequantised as
   // fp32(code * *bias_scale), and FP8 output codes of fp32(y * *r_scale) with
   // max |y| folded into the output's ring by the CTA that finishes last.
@@ -196,14 +199,14 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
 // Bounded wait for the phase of parity `parity` to complete.  Returns false if
 // the budget ran out (error recorded, abort raised) or another role aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort, uint32_t* err,
-                                          uint32_t site) {
+                                          uint32_t site, unsigned long long budget_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitBudgetNs) {
+      if (globaltimer_ns() - t0 > budget_ns) {
         record_device_error(err, site);
         *abort = 1;
         return false;
@@ -457,6 +460,8 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * C::kStages + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * C::kStages + 2 + a); };
   const uint32_t done_bar = bar0 + 8u * (2 * C::kStages + 4);
+  // After the TMEM slot, abort flag and amax slots: never arrived on.
+  const uint32_t stall_bar = bar0 + 8u * (2 * C::kStages + 11);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -474,6 +479,7 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
       mbar_init(tempty_bar(a), kEpiWarps * PAIR);
     }
     mbar_init(done_bar, 1);
+    mbar_init(stall_bar, 1);
     *abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -515,7 +521,7 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
         const int arow = mt * kTileM + int(rank) * kBM;
         const int brow = nt * BN + int(rank) * C::kBRows;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort, p.err, kWaitProducerEmpty)) {
+          if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort, p.err, kWaitProducerEmpty, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -577,11 +583,11 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
         if (!unit_at(p, cta, ctas, i, t, kb0, kb1)) break;
         const int acc = i & 1;
         const uint32_t acc_par = (i >> 1) & 1;
-        if (!mbar_wait(tempty_bar(acc), acc_par ^ 1u, abort, p.err, kWaitMmaTmemEmpty)) break;
+        if (!mbar_wait(tempty_bar(acc), acc_par ^ 1u, abort, p.err, kWaitMmaTmemEmpty, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d = tmem_base + uint32_t(acc * BN);
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait(full_bar(stage), phase, abort, p.err, kWaitMmaFull)) {
+          if (!mbar_wait(full_bar(stage), phase, abort, p.err, kWaitMmaFull, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -654,7 +660,12 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
           finisher ? sk_owner(p, int64_t(t - p.dp_tiles) * p.k_blocks + p.k_blocks - 1) : cta;
       const int acc = i & 1;
       const uint32_t acc_par = (i >> 1) & 1;
-      if (!mbar_wait(tfull_bar(acc), acc_par, abort, p.err, kWaitEpilogueTmemFull)) break;
+      // (Testing: with the stall site set here, the wait is on a barrier that
+      // nothing completes, so it runs out and the abort path runs.)
+      const bool stall = p.stall == kWaitEpilogueTmemFull;
+      if (!mbar_wait(stall ? stall_bar : tfull_bar(acc), stall ? 0u : acc_par, abort, p.err, kWaitEpilogueTmemFull,
+                     p.wait_ns))
+        break;
       tc_fence_after();
       int b, mt, nt;
       decode_tile(p, t, b, mt, nt);
@@ -673,7 +684,7 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
           while (true) {
             asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(seen) : "l"(p.flags + q) : "memory");
             if (seen >= kPieceWarps) break;
-            if (*abort || globaltimer_ns() - w0 > kWaitBudgetNs) {
+            if (*abort || globaltimer_ns() - w0 > p.wait_ns) {
               record_device_error(p.err, kWaitSplitK);
               *abort = 1;
               break;
@@ -1362,6 +1373,9 @@ int mm_validate(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_
   q.nothing = M == 0 || N == 0;
   q.epi = (out8 ? kEpiOut8 : 0) | (bias8 ? kEpiBias8 : 0);
   MmParams& p = q.p;
+  const WaitCfg wc = wait_cfg();
+  p.wait_ns = wc.budget_ns;
+  p.stall = wc.stall_site;
   const int64_t c_stride = batch > 1 ? strides[2] : M * N;
   p.c_stride = c_stride;
   if (out8) {

@@ -84,6 +84,8 @@ def lib():
         L.fp8_linear_forward.restype = i32
         L.fp8_linear_backward.argtypes = [vp, i32, i64, i64, i64, CRing, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.fp8_linear_backward.restype = i32
+        L.fp8_debug_wait.argtypes = [ctypes.c_uint64, ctypes.c_uint32]
+        L.fp8_debug_wait.restype = i32
         L.fp8_quantize_local.argtypes = [vp, i32, i64, i64, i32, i32, CRing, vp, vp, vp, vp]
         L.fp8_quantize_local.restype = i32
         L.fp8_ring_fold.argtypes = [CRing, i32, vp, vp]
@@ -547,6 +549,17 @@ class Linear:
             _ptr(db), _stream(stream, g.get_device()))
         _check(rc, "fp8_linear_backward")
         return dx, dw, db
+
+
+WAIT_BUDGET_DEFAULT_NS = 2_000_000_000
+SITE_EPILOGUE_TMEM_FULL = 4   # fp8_mm: the epilogue's wait for an accumulator
+SITE_QUANTIZE_TMA = 6         # fp8_quantize: the producer / consumer waits
+
+
+def debug_wait(budget_ns=WAIT_BUDGET_DEFAULT_NS, stall_site=0):
+    """fp8_debug_wait (testing only): the budget of the kernels' bounded waits and
+    a wait site at which later launches wait on a barrier nothing completes."""
+    _check((_LIB or lib()).fp8_debug_wait(int(budget_ns), int(stall_site)), "fp8_debug_wait")
 
 
 def device_error(clear=True):

@@ -471,6 +471,34 @@ int fp8_device_error(int clear, uint32_t* where_out);
 /* Number of SMs and the library's build architecture string, for reports. */
 int fp8_device_info(int* sm_count, const char** arch);
 
+/*
+ * fp8_debug_wait -- testing only: shorten the bounded waits and make one run out.
+ *
+ * No page counterpart: this exists so tests can exercise the timeout path of
+ * the kernels without faulting or hanging a GPU.  It sets, for every launch
+ * made afterwards by this process (all threads, all devices):
+ *   budget_ns   the budget of each wait on another role's progress (the
+ *               producer / consumer / MMA / epilogue handshakes), in
+ *               nanoseconds, 1 .. 2e9; 2e9 is the default.  Waits that drain
+ *               a kernel's own TMA copies and MMAs before it frees shared
+ *               memory or TMEM keep 2 s whatever this says, so a kernel that
+ *               gives up never releases memory still being written.
+ *   stall_site  0 (default: no stall), or one wait site code at which the
+ *               kernels wait on a barrier that nothing completes, so that the
+ *               wait runs out after budget_ns:
+ *                 4  fp8_mm family: the epilogue's wait for an accumulator;
+ *                 6  fp8_quantize family, transposed and dual layouts of
+ *                    inputs whose rows are 16-byte aligned (the TMA tile
+ *                    kernel): the consumers' wait for a staged input tile.
+ *                    The row layout's kernel has no waits to shorten.
+ * A wait that runs out records its site code in the device error word
+ * (fp8_device_error), the kernel stops early and returns; its outputs are
+ * undefined and the ring of a stalled quantize has folded an amax of 0.
+ * Restore the defaults with fp8_debug_wait(2000000000, 0).
+ * Errors: FP8_ERR_INVALID_ARG for a budget of 0 or above 2e9, or another site.
+ */
+int fp8_debug_wait(uint64_t budget_ns, uint32_t stall_site);
+
 #ifdef __cplusplus
 }
 #endif

@@ -29,7 +29,7 @@ def test_header_declares_the_boundary():
         ["fp8_quantize", "fp8_mm", "fp8_status_string", "fp8_device_error", "fp8_device_info",
          "fp8_quantize_static_scratch", "fp8_quantize_current", "fp8_bias_grad", "fp8_linear_forward",
          "fp8_linear_backward", "fp8_mm_ws", "fp8_mm_workspace_bytes", "fp8_quantize_local", "fp8_ring_fold",
-         "fp8_mm_pair", "fp8_launch_count", "fp8_quantize_pair", "fp8_mm_ex"])
+         "fp8_mm_pair", "fp8_launch_count", "fp8_quantize_pair", "fp8_mm_ex", "fp8_debug_wait"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -215,3 +215,11 @@ def test_static_scratch_entry_point_checks_before_cuda(L):
                   vp]
     f.restype = ctypes.c_int
     assert f(vp(0x4000), 0, 4, 4, 0, 0, ops.CRing(0, 0, 0, 0, 0), vp(0x2000), None, None) == ops.FP8_ERR_INVALID_ARG
+
+
+def test_debug_wait_checks_its_arguments(L):
+    assert L.fp8_debug_wait(0, 0) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_debug_wait(2_000_000_001, 0) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_debug_wait(1000, 5) == ops.FP8_ERR_INVALID_ARG   # only sites 4 and 6 can stall
+    assert L.fp8_debug_wait(1000, 4) == ops.FP8_OK
+    assert L.fp8_debug_wait(2_000_000_000, 0) == ops.FP8_OK      # back to the defaults

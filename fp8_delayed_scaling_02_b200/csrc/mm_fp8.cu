@@ -233,7 +233,10 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* tm, uint32_t src
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Every bulk store of this thread has finished reading shared memory (its
+// global writes may still be in flight: the grid's completion orders them
+// before any later kernel's reads).
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* tm) {
@@ -940,7 +943,9 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
       if (lane == 0) amax_s[ew] = amax;
     }
-    if (p.tma_store && lane == 0) bulk_wait_all();
+    // The staging buffers are released once the stores have read them; waiting
+    // for the global writes too kept every CTA alive ~0.4 us longer.
+    if (p.tma_store && lane == 0) bulk_wait_read_all();
     __syncwarp();
   }
 
@@ -1268,7 +1273,12 @@ int launch_pair(MmProblem& q0, const MmChoice& c0, MmProblem& q1, const MmChoice
 //     for a 128 x 256 float32 partial: about 4 us to write it, fence and
 //     flag it, and about 5 us per extra piece for the finisher's wait and
 //     read (half that for BN = 128).  So stream-K pays off only where a part
-//     of a wave idles for well over 10 us: small outputs with long K.
+//     of a wave idles for well over 10 us: small outputs with long K;
+//   * the epilogue of a CTA's last tile is not hidden behind a mainloop:
+//     about 0.4 us per 32 output columns of an epilogue warp (a warp holds
+//     half of the tile's columns), measured with a %globaltimer timeline on
+//     B200 -- so a single-wave problem prefers the narrower tile when the
+//     k-blocks cost the same.
 MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool b_mn, size_t ws_limit) {
   struct Opt {
     int bn, pair;
@@ -1288,7 +1298,8 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool
     const int64_t tiles = ((M + kBM * o.pair - 1) / (kBM * o.pair)) * ((N + o.bn - 1) / o.bn) * batch;
     const double t_kb = 0.45 * (o.bn / 256.0) / o.eff;
     const double t_write = 4.0 * (o.bn / 256.0), t_read = 5.0 * (o.bn / 256.0);
-    const double dp_cost = double((tiles + slots - 1) / slots) * double(kb) * t_kb;
+    const double t_epi = 0.4 * (o.bn / 64.0);  // the last tile's epilogue: (BN / 2) / 32 chunks per warp
+    const double dp_cost = double((tiles + slots - 1) / slots) * double(kb) * t_kb + t_epi;
     if (dp_cost < best_cost) {
       best_cost = dp_cost;
       best = MmChoice{o.bn, o.pair, int(std::min<int64_t>(tiles, slots)), int(tiles), 0, 0, dp_cost};
@@ -1308,7 +1319,7 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool
       const int64_t iters = (W + pieces - 1) / pieces;
       const int64_t span = std::min<int64_t>(pieces, (kb - 1 + L - 1) / L + 1);  // pieces a tile can touch
       const double cost = double(dp / slots) * double(kb) * t_kb + double(iters) * t_kb + t_write +
-                          double(span - 1) * t_read;
+                          double(span - 1) * t_read + t_epi;
       const size_t wsb = sk_ws_bytes(int(pieces), o.bn, o.pair);
       if (wsb > ws_limit) continue;
       if (cost < best_cost) {
@@ -1543,7 +1554,8 @@ extern "C" int fp8_mm_pair(const fp8_mm_args* a0, const fp8_mm_args* a1, void* w
     else break;
   }
   const double t_kb = 0.45 / (pair == 2 ? 1.0 : 0.85);
-  const double paired = double(std::max(span(t0, c0, kb0), span(t1, c1, kb1))) * t_kb;
+  // Both problems' last epilogues run at once on different CTAs: one 256-wide epilogue.
+  const double paired = double(std::max(span(t0, c0, kb0), span(t1, c1, kb1))) * t_kb + 0.4 * (256.0 / 64.0);
   const size_t wl = workspace ? workspace_bytes : 0;
   const double apart = choose_mm(q0.M, q0.N, q0.K, q0.batch, sms, q0.p.b_mn, wl).cost +
                        choose_mm(q1.M, q1.N, q1.K, q1.batch, sms, q1.p.b_mn, wl).cost;

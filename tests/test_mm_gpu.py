@@ -190,7 +190,7 @@ def test_mn_major_batched_broadcast():
 # N), a tiny output cut four ways per tile, and ragged ones on 128-wide pair
 # tiles.  Checked against the oracle, deterministic across runs, flags left
 # at zero, and an undersized workspace falls back to whole tiles.
-@pytest.mark.parametrize("M,N,K,a_mn,b_mn", [(1536, 1536, 8192, False, False), (4096, 1536, 8192, True, True),
+@pytest.mark.parametrize("M,N,K,a_mn,b_mn", [(1536, 1536, 16384, False, False), (4096, 1536, 8192, True, True),
                                              (1536, 1536, 8192, True, True), (512, 19200, 4096, False, False),
                                              (500, 19199, 4096, False, False), (128, 256, 8192, False, False),
                                              (1000, 1537, 8192, False, False), (130, 700, 8192, False, False)])
@@ -254,9 +254,9 @@ def test_mm_pair_matches_the_oracle(c0, c1):
 def test_mm_pair_equals_separate_calls_when_the_shapes_match():
     """With one launch shape for both (256-wide CTA pairs, whole tiles) the
     paired results equal the single calls bit for bit."""
-    # 24 long tiles (K = 8192) beside 256 short ones (K = 1024): paired, and
+    # 48 long tiles (K = 8192) beside 256 short ones (K = 1024): paired, and
     # each alone also runs 256-wide CTA pairs over whole tiles.
-    a0, b0 = S.fp8_codes((1024, 8192), seed=1).cuda(), S.fp8_codes((1536, 8192), seed=2).cuda()
+    a0, b0 = S.fp8_codes((2048, 8192), seed=1).cuda(), S.fp8_codes((1536, 8192), seed=2).cuda()
     a1, b1 = S.fp8_codes((8192, 1024), seed=3).cuda(), S.fp8_codes((2048, 1024), seed=4).cuda()
     s = _scalar(1.0)
     y0, y1 = ops.mm_pair(dict(a=a0, b=b0, sinv_a=s, sinv_b=s), dict(a=a1, b=b1, sinv_a=s, sinv_b=s))

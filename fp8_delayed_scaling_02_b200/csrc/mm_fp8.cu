@@ -136,19 +136,24 @@ __device__ __forceinline__ float4 bias8_4(const MmParams& p, int n, float bsc) {
 
 // FP8 output: this CTA's max |y| (per epilogue warp in amax_s) joins the
 // ring's scratch word; the CTA that draws the last of gridDim.x tickets takes
-// the grid's amax, clears the scratch words and commits the ring.  The
-// acq_rel ticket orders each CTA's amax before its increment and gives the
-// last CTA every other CTA's.  ring_s holds the ring's history, idx and scale
-// as read at launch (only this fold writes them).  Run by one thread after
-// the CTA's epilogue.
+// the grid's amax, clears the scratch words and commits the ring.  ring_s
+// holds the ring's history, idx and scale as read at launch (only this fold
+// writes them).  Run by one thread after the CTA's epilogue.
 __device__ __noinline__ void out8_ticket_fold(const MmParams& p, const float* amax_s, const float* ring_s) {
   float m = 0.0f;
 #pragma unroll
   for (int w = 0; w < kEpiWarps; ++w) m = fmaxf(m, amax_s[w]);
-  if (m > 0.0f)
-    asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(p.r_scratch), "r"(__float_as_uint(m)) : "memory");
-  unsigned t;
-  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.r_scratch + 1) : "memory");
+  // The CTA's amax goes in with an atom.max whose return value the ticket's
+  // address depends on (bit 31 of a non-negative float: 0 at run time,
+  // opaque to the compiler), so the ticket is issued only once the amax is
+  // in L2; the CTA with the last ticket exchanges the word only after that
+  // ticket returned, i.e. after every CTA's amax was performed there.  No
+  // fence: a release-ordered ticket would wait for the CTA's output stores.
+  uint32_t old, dep, t;
+  asm volatile("atom.relaxed.gpu.global.max.u32 %0, [%1], %2;" : "=r"(old) : "l"(p.r_scratch), "r"(__float_as_uint(m))
+               : "memory");
+  asm volatile("shr.u32 %0, %1, 31;" : "=r"(dep) : "r"(old));
+  asm volatile("atom.relaxed.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(p.r_scratch + 1 + dep) : "memory");
   if (t != gridDim.x - 1) return;
   uint32_t bits;
   asm volatile("atom.relaxed.gpu.global.exch.b32 %0, [%1], 0;" : "=r"(bits) : "l"(p.r_scratch) : "memory");

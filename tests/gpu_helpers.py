@@ -63,7 +63,8 @@ def oracle_codes(x_cpu, scale, fmt):
     inputs go through ``OR.scaled_codes`` directly."""
     if x_cpu.dtype in (torch.bfloat16, torch.float16):
         pats = torch.arange(1 << 16, dtype=torch.int32).to(torch.int16).view(x_cpu.dtype)
-        table = OR.scaled_codes(OR.to_float32(pats), np.float32(scale), fmt)
+        with np.errstate(over="ignore", invalid="ignore"):  # the table spans inf, NaN and huge patterns
+            table = OR.scaled_codes(OR.to_float32(pats), np.float32(scale), fmt)
         bits = x_cpu.contiguous().view(torch.int16).numpy().view(np.uint16)
         return table[bits]
     return OR.scaled_codes(OR.to_float32(x_cpu), np.float32(scale), fmt)

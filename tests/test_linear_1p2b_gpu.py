@@ -1,10 +1,13 @@
 """GPU parity of the 1.2B-model linear workload over 16 delayed-scaling steps, M in {512, 2048, 8192}.
 
 Per step and per linear shape (W1 [1536,1536], W2 [4096,1536]), in the launch
-configuration the bench times: X and W dual E4M3 in one fp8_quantize_pair
-launch, G dual E5M2, then fwd Y = Xq.Wq^T + b (fp8_mm with the stream-K
-workspace) and dX = Gq.(W^T)q^T, dW = (G^T)q.(X^T)q^T in one fp8_mm_pair
-launch, each GEMM with its rings' scale_inv.  The three rings are checked
+configurations the bench times: X and W E4M3 in one fp8_quantize_pair launch,
+G E5M2, then fwd Y = Xq.Wq^T + b (fp8_mm with the stream-K workspace) and
+dX = Gq.Wq, dW = Gq^T.Xq in one fp8_mm_pair launch, each GEMM with its rings'
+scale_inv -- either with dual quantizes and NT backward GEMMs on the
+transposed copies (the headline step), or with row quantizes only and the
+backward GEMMs reading the row copies as MN-major operands (the layout-tag
+step).  The three rings are checked
 against the oracle after every step (bit-exact: amax history, idx, scale,
 scale_inv).  At the first and the last step every byte of the six quantized
 tensors is compared, and the three GEMM outputs on three rows of every
@@ -46,7 +49,8 @@ def _check_gemm(y, a_codes, b_codes, fmt_a, sinv_a, sinv_b, bias, rows, what):
 
 @pytest.mark.parametrize("M", [512, 2048, 8192])
 @pytest.mark.parametrize("which", [0, 1])
-def test_linear_1p2b_sixteen_delayed_steps(M, which):
+@pytest.mark.parametrize("layout_tag", [False, True])
+def test_linear_1p2b_sixteen_delayed_steps(M, which, layout_tag):
     (w1, b1), (w2, b2) = S.linear_1p2b_weights()
     w, bias = (w1, b1) if which == 0 else (w2, b2)
     n_out = w.shape[0]
@@ -64,13 +68,20 @@ def test_linear_1p2b_sixteen_delayed_steps(M, which):
     for step in range(STEPS):
         x, g = S.linear_1p2b_step(M, n_out, step)
         sx, sw, sg = ox.scale, ow.scale, og.scale  # scales this step's quantizes use
-        ops.quantize_pair(dict(x=x.cuda(), fmt=ops.E4M3, layout=ops.DUAL, ring=rx, out=xq, out_t=xq_t),
-                          dict(x=wd, fmt=ops.E4M3, layout=ops.DUAL, ring=rw, out=wq, out_t=wq_t))
-        ops.quantize(g.cuda(), ops.E5M2, ops.DUAL, rg, gq, gq_t)
+        lay = ops.ROW if layout_tag else ops.DUAL
+        ops.quantize_pair(dict(x=x.cuda(), fmt=ops.E4M3, layout=lay, ring=rx, out=xq, out_t=xq_t),
+                          dict(x=wd, fmt=ops.E4M3, layout=lay, ring=rw, out=wq, out_t=wq_t))
+        ops.quantize(g.cuda(), ops.E5M2, lay, rg, gq, gq_t)
         ops.mm(xq, wq, rx.scale_inv, rw.scale_inv, bd, out=y, workspace=ws)
-        ops.mm_pair(dict(a=gq, b=wq_t, sinv_a=rg.scale_inv, sinv_b=rw.scale_inv, fmt_a=ops.E5M2, out=dx),
-                    dict(a=gq_t, b=xq_t, sinv_a=rg.scale_inv, sinv_b=rx.scale_inv, fmt_a=ops.E5M2, out=dw),
-                    workspace=ws)
+        if layout_tag:
+            ops.mm_pair(dict(a=gq, b=wq, sinv_a=rg.scale_inv, sinv_b=rw.scale_inv, fmt_a=ops.E5M2, out=dx,
+                             b_mn_major=True),
+                        dict(a=gq, b=xq, sinv_a=rg.scale_inv, sinv_b=rx.scale_inv, fmt_a=ops.E5M2, out=dw,
+                             a_mn_major=True, b_mn_major=True), workspace=ws)
+        else:
+            ops.mm_pair(dict(a=gq, b=wq_t, sinv_a=rg.scale_inv, sinv_b=rw.scale_inv, fmt_a=ops.E5M2, out=dx),
+                        dict(a=gq_t, b=xq_t, sinv_a=rg.scale_inv, sinv_b=rx.scale_inv, fmt_a=ops.E5M2, out=dw),
+                        workspace=ws)
         torch.cuda.synchronize()
         OR.fold(ox, OR.amax(OR.to_float32(x)), OR.F.E4M3)
         OR.fold(ow, w_amax, OR.F.E4M3)
@@ -80,13 +91,14 @@ def test_linear_1p2b_sixteen_delayed_steps(M, which):
         assert_ring_equal(rg, og)
         if step not in (0, STEPS - 1):
             continue
-        what = f"M={M} N={n_out} step {step}"
+        what = f"M={M} N={n_out} step {step} {'layout tag' if layout_tag else 'dual'}"
         x_all, w_all, g_all = oracle_codes(x, sx, OR.F.E4M3), oracle_codes(w, sw, OR.F.E4M3), \
             oracle_codes(g, sg, OR.F.E5M2)
         for got, ref, name in ((xq, x_all, "xq"), (wq, w_all, "wq"), (gq, g_all, "gq")):
             assert_bytes_equal(got, ref, f"{name} {what}")
-        for got, ref, name in ((xq_t, x_all, "xq_t"), (wq_t, w_all, "wq_t"), (gq_t, g_all, "gq_t")):
-            assert_bytes_equal(got, np.ascontiguousarray(ref.T), f"{name} {what}")
+        if not layout_tag:
+            for got, ref, name in ((xq_t, x_all, "xq_t"), (wq_t, w_all, "wq_t"), (gq_t, g_all, "gq_t")):
+                assert_bytes_equal(got, np.ascontiguousarray(ref.T), f"{name} {what}")
         sinv_x, sinv_w, sinv_g = ox.scale_inv, ow.scale_inv, og.scale_inv
         rows_m, rows_n = band_rows(M, seed=M + step), band_rows(n_out, seed=n_out + step)
         _check_gemm(y, x_all, w_all, 0, sinv_x, sinv_w, bias.numpy(), rows_m, f"fwd {what}")

@@ -875,7 +875,7 @@ __device__ __forceinline__ void mm_body(const CUtensorMap* tmA, const CUtensorMa
 #pragma unroll 1
       for (int c = 0; c < kChunks; c += 2) {
         if (nbase + c * 32 >= p.N) break;  // warp-uniform: the rest of this half is beyond N
-        const bool two = nbase + (c + 1) * 32 < p.N;
+        const bool two = c + 1 < kChunks && nbase + (c + 1) * 32 < p.N;
         const bool last_pair = c + 2 >= kChunks || nbase + (c + 2) * 32 >= p.N;
         if (finisher) {
           // Per chunk: the next piece's partial is requested (8 independent
@@ -1267,31 +1267,31 @@ int launch_pair(MmProblem& q0, const MmChoice& c0, MmProblem& q1, const MmChoice
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-// Launch-shape choice by a time model in microseconds, over {one CTA, CTA
-// pair} x {BN 256, 128} and, given a workspace, a stream-K tail:
-//   * one k-block of a 128 x 256 tile takes about 0.45 us on one SM (pairs
-//     and single CTAs alike; relative efficiencies below);
-//   * whole tiles run in waves of `slots`;
+// Launch-shape choice by a time model in microseconds, over 256-wide tiles
+// on CTA pairs or single CTAs, single CTAs with 128- and 64-wide tiles and,
+// given a workspace, a stream-K tail.  (128-wide tiles on CTA pairs run the
+// same waves as on single CTAs and were never faster.)  Fitted to graph-timed B200 runs of every shape at square
+// sizes 512-2048 and the 1.2B-model linears (M 512-8192):
+//   * whole tiles run in waves of `slots`; one k-block of one wave takes
+//     `s` (0.35 us for 128 x 64 tiles up to 0.41-0.44 us for 256-wide ones:
+//     the mainloop is bound by operand traffic into the SM, so wider tiles
+//     do more work per byte), and a launch costs a fixed `I` (set-up, first
+//     loads, the last tile's epilogue: more columns, more epilogue);
 //   * stream-K (data-parallel + two-tile stream-K): all but the last full
 //     wave stay whole tiles; the k-blocks of the rest are dealt evenly to the
 //     pieces.  A piece costs its k-blocks plus the fix-up measured on B200
 //     for a 128 x 256 float32 partial: about 4 us to write it, fence and
 //     flag it, and about 5 us per extra piece for the finisher's wait and
-//     read (half that for BN = 128).  So stream-K pays off only where a part
-//     of a wave idles for well over 10 us: small outputs with long K;
-//   * the epilogue of a CTA's last tile is not hidden behind a mainloop:
-//     about 0.4 us per 32 output columns of an epilogue warp (a warp holds
-//     half of the tile's columns), measured with a %globaltimer timeline on
-//     B200 -- so a single-wave problem prefers the narrower tile when the
-//     k-blocks cost the same.
+//     read (half that for 128-wide and narrower tiles: the waits and fences
+//     do not shrink with a 64-wide partial).  So stream-K pays off only
+//     where a part of a wave idles for well over 10 us: small outputs with
+//     long K.
 MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool b_mn, size_t ws_limit) {
   struct Opt {
     int bn, pair;
-    double eff;
+    double s, fixed;  // us per k-block of a wave; us per launch
   };
-  // A 128-wide MMA issues at about the rate of a 256-wide one, so BN = 128
-  // does half the work per instruction whether or not the CTAs are paired.
-  const Opt opts[4] = {{256, 2, 1.0}, {256, 1, 0.85}, {128, 2, 0.5}, {128, 1, 0.45}};
+  const Opt opts[4] = {{256, 2, 0.41, 5.1}, {256, 1, 0.44, 4.6}, {128, 1, 0.37, 3.5}, {64, 1, 0.35, 3.3}};
   constexpr int kMinIters = 4;  // k-blocks per piece, at least
   const int64_t kb = (K + kBK - 1) / kBK;
   MmChoice best{256, 1, 1, 0, 0, 0, 0.0};
@@ -1299,12 +1299,10 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool
   for (const Opt& o : opts) {
     if (o.pair == 2 && M <= kBM) continue;  // the second CTA would hold no rows
     if (b_mn && o.bn / o.pair < 128) continue;
-    const int slots = o.pair == 2 ? (o.bn == 256 ? max_pairs<256>(sms) : max_pairs<128>(sms)) : sms;
+    const int slots = o.pair == 2 ? max_pairs<256>(sms) : sms;
     const int64_t tiles = ((M + kBM * o.pair - 1) / (kBM * o.pair)) * ((N + o.bn - 1) / o.bn) * batch;
-    const double t_kb = 0.45 * (o.bn / 256.0) / o.eff;
-    const double t_write = 4.0 * (o.bn / 256.0), t_read = 5.0 * (o.bn / 256.0);
-    const double t_epi = 0.4 * (o.bn / 64.0);  // the last tile's epilogue: (BN / 2) / 32 chunks per warp
-    const double dp_cost = double((tiles + slots - 1) / slots) * double(kb) * t_kb + t_epi;
+    const double t_write = 4.0 * (std::max(o.bn, 128) / 256.0), t_read = 5.0 * (std::max(o.bn, 128) / 256.0);
+    const double dp_cost = o.fixed + double((tiles + slots - 1) / slots) * double(kb) * o.s;
     if (dp_cost < best_cost) {
       best_cost = dp_cost;
       best = MmChoice{o.bn, o.pair, int(std::min<int64_t>(tiles, slots)), int(tiles), 0, 0, dp_cost};
@@ -1323,8 +1321,8 @@ MmChoice choose_mm(int64_t M, int64_t N, int64_t K, int64_t batch, int sms, bool
       if (W % pieces == 0 && L % kb == 0) continue;  // every piece whole tiles: the data-parallel case
       const int64_t iters = (W + pieces - 1) / pieces;
       const int64_t span = std::min<int64_t>(pieces, (kb - 1 + L - 1) / L + 1);  // pieces a tile can touch
-      const double cost = double(dp / slots) * double(kb) * t_kb + double(iters) * t_kb + t_write +
-                          double(span - 1) * t_read + t_epi;
+      const double cost = o.fixed + double(dp / slots) * double(kb) * o.s + double(iters) * o.s + t_write +
+                          double(span - 1) * t_read;
       const size_t wsb = sk_ws_bytes(int(pieces), o.bn, o.pair);
       if (wsb > ws_limit) continue;
       if (cost < best_cost) {
@@ -1465,12 +1463,10 @@ int mm_run(MmProblem& q, void* workspace, size_t ws_bytes, cudaStream_t st) {
   if (sms <= 0) return FP8_ERR_CUDA;
   if (workspace != nullptr && reinterpret_cast<uintptr_t>(workspace) % 256 != 0) return FP8_ERR_UNSUPPORTED;
   const MmChoice c = choose_mm(q.M, q.N, q.K, q.batch, sms, q.p.b_mn, workspace ? ws_bytes : 0);
-  if (c.pair == 2) {
-    if (c.bn == 256) return launch_mm<256, 2>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
-    return launch_mm<128, 2>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
-  }
+  if (c.pair == 2) return launch_mm<256, 2>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
   if (c.bn == 256) return launch_mm<256, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
-  return launch_mm<128, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
+  if (c.bn == 128) return launch_mm<128, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
+  return launch_mm<64, 1>(q.A, q.B, q.M, q.N, q.K, q.batch, q.strides, q.p, q.epi, c, workspace, st);
 }
 
 }  // namespace
@@ -1558,9 +1554,9 @@ extern "C" int fp8_mm_pair(const fp8_mm_args* a0, const fp8_mm_args* a1, void* w
     else if (c1 < t1) ++c1;
     else break;
   }
-  const double t_kb = 0.45 / (pair == 2 ? 1.0 : 0.85);
-  // Both problems' last epilogues run at once on different CTAs: one 256-wide epilogue.
-  const double paired = double(std::max(span(t0, c0, kb0), span(t1, c1, kb1))) * t_kb + 0.4 * (256.0 / 64.0);
+  // The same time model as choose_mm: one launch's fixed cost, 256-wide tiles.
+  const double paired = (pair == 2 ? 5.1 : 4.6) +
+                        double(std::max(span(t0, c0, kb0), span(t1, c1, kb1))) * (pair == 2 ? 0.41 : 0.44);
   const size_t wl = workspace ? workspace_bytes : 0;
   const double apart = choose_mm(q0.M, q0.N, q0.K, q0.batch, sms, q0.p.b_mn, wl).cost +
                        choose_mm(q1.M, q1.N, q1.K, q1.batch, sms, q1.p.b_mn, wl).cost;
@@ -1568,6 +1564,19 @@ extern "C" int fp8_mm_pair(const fp8_mm_args* a0, const fp8_mm_args* a1, void* w
   const MmChoice ch0{256, pair, int(c0), int(t0), 0, 0, 0.0};
   const MmChoice ch1{256, pair, int(c1), int(t1), 0, 0, 0.0};
   return pair == 2 ? launch_pair<256, 2>(q0, ch0, q1, ch1, st) : launch_pair<256, 1>(q0, ch0, q1, ch1, st);
+}
+
+extern "C" int fp8_mm_launch_shape(int64_t M, int64_t N, int64_t K, int64_t batch, int layout,
+                                   size_t workspace_bytes, int32_t* shape) {
+  if (shape == nullptr || M <= 0 || N <= 0 || K <= 0 || batch < 1) return FP8_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return FP8_ERR_CUDA;
+  const MmChoice c = choose_mm(M, N, K, batch, sms, (layout & FP8_MM_B_MN_MAJOR) != 0, workspace_bytes);
+  shape[0] = c.bn;
+  shape[1] = c.pair;
+  shape[2] = c.grid * c.pair;
+  shape[3] = c.sk_ctas;
+  return FP8_OK;
 }
 
 extern "C" size_t fp8_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t batch, int layout) {

@@ -80,6 +80,8 @@ def lib():
         L.fp8_mm_ws.restype = i32
         L.fp8_mm_workspace_bytes.argtypes = [i64, i64, i64, i64, i32]
         L.fp8_mm_workspace_bytes.restype = ctypes.c_size_t
+        L.fp8_mm_launch_shape.argtypes = [i64, i64, i64, i64, i32, ctypes.c_size_t, ctypes.POINTER(ctypes.c_int32)]
+        L.fp8_mm_launch_shape.restype = i32
         L.fp8_linear_forward.argtypes = [vp, i32, vp, i32, i64, i64, i64, vp, CRing, CRing, vp, vp, vp, vp]
         L.fp8_linear_forward.restype = i32
         L.fp8_linear_backward.argtypes = [vp, i32, i64, i64, i64, CRing, vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -272,6 +274,15 @@ def mm_workspace_bytes(M, N, K, batch=1, a_mn_major=False, b_mn_major=False):
     """Bytes of workspace fp8_mm_ws would use (0 when whole tiles are as fast)."""
     layout = (MM_A_MN_MAJOR if a_mn_major else 0) | (MM_B_MN_MAJOR if b_mn_major else 0)
     return int((_LIB or lib()).fp8_mm_workspace_bytes(M, N, K, batch, layout))
+
+
+def mm_launch_shape(M, N, K, batch=1, a_mn_major=False, b_mn_major=False, workspace_bytes=0):
+    """The launch shape fp8_mm / fp8_mm_ws picks: dict(bn, cluster, ctas, stream_k_pieces)."""
+    layout = (MM_A_MN_MAJOR if a_mn_major else 0) | (MM_B_MN_MAJOR if b_mn_major else 0)
+    shape = (ctypes.c_int32 * 4)()
+    rc = (_LIB or lib()).fp8_mm_launch_shape(M, N, K, batch, layout, workspace_bytes, shape)
+    _check(rc, "fp8_mm_launch_shape")
+    return dict(bn=shape[0], cluster=shape[1], ctas=shape[2], stream_k_pieces=shape[3])
 
 
 def _shape2d(a, b, a_mn_major, b_mn_major, out):

@@ -353,11 +353,24 @@ int fp8_linear_backward(const void* g, int g_dtype, int64_t M, int64_t N, int64_
  * fp8_mm_workspace_bytes -- the workspace size fp8_mm_ws would use for this
  * problem on the current device (0 when whole tiles are as fast); at most
  * 1024 + 148 x 128 x 256 x 4 bytes (about 19.4 MB) on a 148-SM B200.
+ *
+ * fp8_mm_launch_shape -- the launch shape fp8_mm (workspace_bytes 0) or
+ * fp8_mm_ws (a workspace of workspace_bytes) picks for an M x N x K problem
+ * with this layout on the current device, by the library's time model.
+ * Writes shape[0] = output tile width BN (256, 128 or 64; tiles are 128
+ * rows per CTA), shape[1] = CTAs per cluster (2: a CTA pair runs 256-row
+ * tiles, 1: single CTAs), shape[2] = CTAs launched, shape[3] = stream-K
+ * pieces (0: whole tiles only).  fp8_mm_pair has its own shared launch and
+ * is not described by this.  Host-only: launches nothing.  Errors:
+ * FP8_ERR_INVALID_ARG for a null shape or M, N, K < 1 or batch < 1;
+ * FP8_ERR_CUDA when no device can be queried.  The pages have no counterpart.
  */
 int fp8_mm_ws(const uint8_t* A, const uint8_t* B, int64_t M, int64_t N, int64_t K, int64_t batch,
               const int64_t* strides, int layout, const float* sinv_a, const float* sinv_b, const float* bias,
               uint16_t* out_bf16, void* workspace, size_t workspace_bytes, fp8_stream_t stream);
 size_t fp8_mm_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t batch, int layout);
+int fp8_mm_launch_shape(int64_t M, int64_t N, int64_t K, int64_t batch, int layout, size_t workspace_bytes,
+                        int32_t* shape);
 
 /*
  * fp8_mm_pair -- two independent GEMMs (each exactly an fp8_mm call) in one

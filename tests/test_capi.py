@@ -29,7 +29,8 @@ def test_header_declares_the_boundary():
         ["fp8_quantize", "fp8_mm", "fp8_status_string", "fp8_device_error", "fp8_device_info",
          "fp8_quantize_static_scratch", "fp8_quantize_current", "fp8_bias_grad", "fp8_linear_forward",
          "fp8_linear_backward", "fp8_mm_ws", "fp8_mm_workspace_bytes", "fp8_quantize_local", "fp8_ring_fold",
-         "fp8_mm_pair", "fp8_launch_count", "fp8_quantize_pair", "fp8_mm_ex", "fp8_debug_wait"])
+         "fp8_mm_pair", "fp8_launch_count", "fp8_quantize_pair", "fp8_mm_ex", "fp8_debug_wait",
+         "fp8_mm_launch_shape"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -223,3 +224,11 @@ def test_debug_wait_checks_its_arguments(L):
     assert L.fp8_debug_wait(1000, 5) == ops.FP8_ERR_INVALID_ARG   # only sites 4 and 6 can stall
     assert L.fp8_debug_wait(1000, 4) == ops.FP8_OK
     assert L.fp8_debug_wait(2_000_000_000, 0) == ops.FP8_OK      # back to the defaults
+
+
+def test_launch_shape_query_checks_its_arguments(L):
+    """Argument errors come before any device query, so they show on a CPU host too."""
+    shape = (ctypes.c_int32 * 4)()
+    assert L.fp8_mm_launch_shape(128, 128, 128, 1, 0, 0, None) == ops.FP8_ERR_INVALID_ARG
+    for M, N, K, batch in ((0, 128, 128, 1), (128, -1, 128, 1), (128, 128, 0, 1), (128, 128, 128, 0)):
+        assert L.fp8_mm_launch_shape(M, N, K, batch, 0, 0, shape) == ops.FP8_ERR_INVALID_ARG

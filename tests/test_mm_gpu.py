@@ -185,13 +185,13 @@ def test_mn_major_batched_broadcast():
 # Stream-K through a caller workspace (fp8_mm_ws): the k-blocks of the last
 # waves' tiles are dealt evenly to the CTAs, and pieces that start inside a
 # tile hand float32 partials to the CTA holding the tile's first k-block.
-# Shapes: the linear's dW GEMMs (fewer tiles than CTA pairs), wide outputs
+# Shapes: dW GEMMs of the linears with long K (fewer tiles than CTA pairs), wide outputs
 # with a wave of whole tiles before the stream-K tail (one ragged in M and
 # N), a tiny output cut four ways per tile, and ragged ones on 128-wide pair
 # tiles.  Checked against the oracle, deterministic across runs, flags left
 # at zero, and an undersized workspace falls back to whole tiles.
 @pytest.mark.parametrize("M,N,K,a_mn,b_mn", [(1536, 1536, 16384, False, False), (4096, 1536, 8192, True, True),
-                                             (1536, 1536, 8192, True, True), (512, 19200, 4096, False, False),
+                                             (1536, 1536, 16384, True, True), (512, 19200, 4096, False, False),
                                              (500, 19199, 4096, False, False), (128, 256, 8192, False, False),
                                              (1000, 1537, 8192, False, False), (130, 700, 8192, False, False)])
 def test_split_k_workspace(M, N, K, a_mn, b_mn):

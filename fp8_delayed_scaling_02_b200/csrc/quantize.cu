@@ -644,9 +644,17 @@ __device__ __forceinline__ void tile_tma_body(const CUtensorMap* tmIn, const Tma
       // ahead take more (CTAs progress at unequal rates: a static deal of
       // all tiles made a 67M-element DUAL call 20% slower).  Two claims are
       // kept in flight, the first issued two tiles before it is needed.
+      // When the static tiles cover the tensor (ntiles <= S * nblk, e.g. a
+      // 1536x1536 weight) nothing is claimed: a claim's round trip to L2
+      // delayed the static loads that follow it (1536x1536 bf16 T: 6.6 ->
+      // 6.0 us without claims on B200).  Issuing all static tiles before
+      // any claim was measured too: faster for fp32 (two stages) but 1.4 us
+      // slower for 12.6M-element bf16 T, where the three rounds requested
+      // at once are 87% of the input and every block's first tile lands late.
       uint32_t* ctr = a.ring.scratch + 2;
       const uint32_t rounds = min(uint32_t(S), (ntiles + nblk - 1) / nblk);
       const uint32_t dyn0 = rounds * nblk;
+      const bool dyn = dyn0 < ntiles;
       uint32_t c0 = 0, c1 = 0;  // claims in flight (c0 the older), valid from iteration rounds - 2 on
       for (uint32_t k = 0;; ++k) {
         if (!bar_wait_bounded(empty0 + 8u * stage, phase ^ 1u, args.wait_ns)) {
@@ -658,15 +666,17 @@ __device__ __forceinline__ void tile_tma_body(const CUtensorMap* tmIn, const Tma
         uint32_t t;
         if (k < rounds) {
           t = blk + k * nblk;
-          if (k + 2 == rounds) c0 = atomicAdd(ctr, 1u);
-          if (k + 1 == rounds) {
+          if (dyn && k + 2 == rounds) c0 = atomicAdd(ctr, 1u);
+          if (dyn && k + 1 == rounds) {
             if (rounds == 1) c0 = atomicAdd(ctr, 1u);
             c1 = atomicAdd(ctr, 1u);
           }
-        } else {
+        } else if (dyn) {
           t = dyn0 + c0;
           c0 = c1;
           c1 = atomicAdd(ctr, 1u);
+        } else {
+          t = kNoTile;
         }
         if (t < ntiles) {
           tile_id[stage] = t;

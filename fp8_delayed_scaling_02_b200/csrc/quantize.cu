@@ -510,11 +510,16 @@ constexpr int kConsumerWarps = 8;
 constexpr int kWsThreads = 32 * (kConsumerWarps + 1);
 constexpr uint32_t kNoTile = 0xFFFFFFFFu;
 
-template <int DT>
+// kShift: an input base that is only element-aligned, rows a multiple of 16
+// bytes (see tile_tma_body): each tile row is staged as 64 + 16 / in_bytes
+// elements (the tile's columns plus the slack of rounding the box start down
+// to 16 bytes), unswizzled.
+template <int DT, bool kShift = false>
 struct TmaTile {
   static constexpr int kBoxes = In<DT>::kBytes == 4 ? 2 : 1;  // 128-byte-wide boxes per 64-column tile
   static constexpr int kBoxBytes = kTileR * 128;
-  static constexpr int kStageBytes = kBoxes * kBoxBytes;
+  static constexpr int kSRowBytes = (kTileC + 16 / In<DT>::kBytes) * In<DT>::kBytes;  // 144 / 272
+  static constexpr int kStageBytes = kShift ? kTileR * kSRowBytes : kBoxes * kBoxBytes;
   static constexpr int kStages = DT == FP8_IN_FP32 ? 2 : 3;
   static constexpr int kTBytes = kTileC * kTileR;  // one transpose buffer: 64 rows of 128 bytes
   static constexpr int kBarOff = kStages * kStageBytes + 2 * kTBytes;
@@ -526,6 +531,9 @@ struct TmaTileArgs {
   uint32_t* err;
   unsigned long long wait_ns;  // budget of the producer's and consumers' waits on each other
   uint32_t stall;              // kWaitQuantizeTma: consumers wait on a never-completed barrier (testing)
+  // kShift only: the map starts off_e elements before the input base (at the
+  // base rounded down to 16 bytes), so input column c is map column off_e + c.
+  int off_e;
 };
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
@@ -556,6 +564,17 @@ __device__ __forceinline__ bool bar_wait_bounded(uint32_t bar, uint32_t parity,
 
 __device__ __forceinline__ void bar_arrive_local(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// mbarrier arrive issued only once `dep` is available: the predicate that
+// guards it is computed from dep, and no value of dep makes it false.
+__device__ __forceinline__ void bar_arrive_after(uint32_t bar, uint32_t dep) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 d;\n\t"
+      "and.b32 d, %1, 0x7FFFFFFF;\n\t"
+      "setp.ne.u32 p, d, 0xFFFFFFFF;\n\t"
+      "@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(bar), "r"(dep)
+      : "memory");
 }
 
 // OR-reduction barrier over the consumer warps only (named barrier 1).
@@ -592,15 +611,60 @@ __device__ __forceinline__ void issue_tile_load(const CUtensorMap* tm, uint32_t 
   }
 }
 
+// Shifted base: the tile's box starts at map column off_e + c0 rounded down
+// to 16 bytes and is 64 + 16 / in_bytes columns wide, so it holds the tile's
+// 64 columns whatever the base's offset inside its 16-byte granule.
+template <int DT>
+__device__ __forceinline__ void issue_tile_load_shift(const CUtensorMap* tm, uint32_t dst, uint32_t bar, uint32_t t,
+                                                      uint32_t tiles_c, int off_e) {
+  constexpr int kAlign = 16 / In<DT>::kBytes;
+  const uint32_t tr = t / tiles_c;
+  const int r0 = int(tr * kTileR);
+  const int x = (off_e + int(t - tr * tiles_c) * kTileC) & ~(kAlign - 1);
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+               "r"(uint32_t(TmaTile<DT, true>::kStageBytes))
+               : "memory");
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(tm)), "r"(x), "r"(r0), "r"(bar)
+      : "memory");
+}
+
+// Eight bytes (lo, hi) to an address of any alignment with the widest
+// aligned stores it allows.
+__device__ __forceinline__ void store8_any(uint8_t* o, uint32_t lo, uint32_t hi) {
+  const int m = int(reinterpret_cast<uintptr_t>(o) & 7);
+  if (m == 0) {
+    *reinterpret_cast<uint2*>(o) = make_uint2(lo, hi);
+  } else if (m == 4) {
+    reinterpret_cast<uint32_t*>(o)[0] = lo;
+    reinterpret_cast<uint32_t*>(o)[1] = hi;
+  } else if ((m & 1) == 0) {
+    uint16_t* h = reinterpret_cast<uint16_t*>(o);
+    h[0] = uint16_t(lo);
+    h[1] = uint16_t(lo >> 16);
+    h[2] = uint16_t(hi);
+    h[3] = uint16_t(hi >> 16);
+  } else {
+    o[0] = uint8_t(lo);
+    uint16_t* h = reinterpret_cast<uint16_t*>(o + 1);
+    h[0] = uint16_t(__byte_perm(lo, 0, 0x0021));
+    h[1] = uint16_t(__byte_perm(lo, hi, 0x0043));
+    h[2] = uint16_t(__byte_perm(hi, 0, 0x0021));
+    o[7] = uint8_t(hi >> 24);
+  }
+}
+
 // Byte offset of 16-byte unit v of transpose-buffer row c (rows of 128 bytes;
 // the unit index is XOR-swizzled by the column group so that the column-word
 // writes and the row reads are both free of bank conflicts).
 __device__ __forceinline__ int tbuf_unit(int c, int v) { return c * 128 + ((v ^ ((c >> 2) & 6)) << 4); }
 
-template <int DT, int FMT, bool kDual>
+template <int DT, int FMT, bool kDual, bool kShift = false>
 __device__ __forceinline__ void tile_tma_body(const CUtensorMap* tmIn, const TmaTileArgs& args, const unsigned blk,
                                               const unsigned nblk) {
-  using TT = TmaTile<DT>;
+  using TT = TmaTile<DT, kShift>;
   constexpr int kB = In<DT>::kBytes;
   constexpr int S = TT::kStages;
   const TileArgs& a = args.t;
@@ -680,7 +744,11 @@ __device__ __forceinline__ void tile_tma_body(const CUtensorMap* tmIn, const Tma
         }
         if (t < ntiles) {
           tile_id[stage] = t;
-          issue_tile_load<DT>(tmIn, sbase + uint32_t(stage * TT::kStageBytes), full0 + 8u * stage, t, tiles_c);
+          if constexpr (kShift)
+            issue_tile_load_shift<DT>(tmIn, sbase + uint32_t(stage * TT::kStageBytes), full0 + 8u * stage, t, tiles_c,
+                                      args.off_e);
+          else
+            issue_tile_load<DT>(tmIn, sbase + uint32_t(stage * TT::kStageBytes), full0 + 8u * stage, t, tiles_c);
           armed |= 1u << stage;
           armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
         } else {
@@ -725,36 +793,88 @@ __device__ __forceinline__ void tile_tma_body(const CUtensorMap* tmIn, const Tma
       uint32_t q[4][2];
       if (!stop) {
         const uint8_t* st = smem + stage * TT::kStageBytes;
+        if constexpr (kShift) {
+          // Staged row rl holds input row r0 + rl from column c0 - d on, where
+          // d = (off_e + c0) mod (16 / in_bytes); elements past the last column
+          // (zero-filled or the next row's) are set to zero before the amax.
+          // Rows 4 apart are 576 bytes apart, so a quarter-warp's loads split
+          // over two 64-byte halves of the banks (4-way conflicts).
+          constexpr int kAlign = 16 / kB;
+          const uint32_t tr = t / tiles_c;
+          const int64_t gc = int64_t(t - tr * tiles_c) * kTileC + lc0;  // this lane's first column
+          const int d = int((args.off_e + gc - lc0) & (kAlign - 1));
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int r = lr0 + i;
-          float v[8];
-          if constexpr (kB == 2) {
-            const int chunk = (lc0 >> 3) ^ (r & 7);
-            const uint4 w = *reinterpret_cast<const uint4*>(st + r * 128 + chunk * 16);
-            amax2 = absmax2<DT>(absmax2<DT>(amax2, w.x), absmax2<DT>(w.y, absmax2<DT>(w.z, w.w)));
-            unpack2<DT>(w.x, v[0], v[1]);
-            unpack2<DT>(w.y, v[2], v[3]);
-            unpack2<DT>(w.z, v[4], v[5]);
-            unpack2<DT>(w.w, v[6], v[7]);
-          } else {
-            const int box = lc0 >> 5;
-            const int ch = (lc0 & 31) >> 2;
-            const uint8_t* rowp = st + box * TT::kBoxBytes + r * 128;
-            const float4 f0 = *reinterpret_cast<const float4*>(rowp + ((ch ^ (r & 7)) * 16));
-            const float4 f1 = *reinterpret_cast<const float4*>(rowp + (((ch + 1) ^ (r & 7)) * 16));
-            v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
-            v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+          for (int i = 0; i < 4; ++i) {
+            const int off = (lr0 + i) * TT::kSRowBytes + (d + lc0) * kB;
+            const uint8_t* g16 = st + (off & ~15);
+            const int ph = off & 15;
+            float v[8];
+            if constexpr (kB == 2) {
+              uint32_t W[8], D[4];
+              const uint4 w0 = *reinterpret_cast<const uint4*>(g16);
+              const uint4 w1 = *reinterpret_cast<const uint4*>(g16 + 16);
+              W[0] = w0.x; W[1] = w0.y; W[2] = w0.z; W[3] = w0.w;
+              W[4] = w1.x; W[5] = w1.y; W[6] = w1.z; W[7] = w1.w;
+              realign<4>(W, ph, D);
 #pragma unroll
-            for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+              for (int e = 0; e < 4; ++e) unpack2<DT>(D[e], v[2 * e], v[2 * e + 1]);
+            } else {
+              uint32_t W[12], D[8];
+              const uint4 w0 = *reinterpret_cast<const uint4*>(g16);
+              const uint4 w1 = *reinterpret_cast<const uint4*>(g16 + 16);
+              const uint4 w2 = ph != 0 ? *reinterpret_cast<const uint4*>(g16 + 32) : make_uint4(0u, 0u, 0u, 0u);
+              W[0] = w0.x; W[1] = w0.y; W[2] = w0.z; W[3] = w0.w;
+              W[4] = w1.x; W[5] = w1.y; W[6] = w1.z; W[7] = w1.w;
+              W[8] = w2.x; W[9] = w2.y; W[10] = w2.z; W[11] = w2.w;
+              realign<8>(W, ph, D);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(D[e]);
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              if (gc + e >= a.cols) v[e] = 0.0f;
+              amax = fmaxf(amax, fabsf(v[e]));
+            }
+            q[i][0] = cvt4<FMT>(v[0], v[1], v[2], v[3], s);
+            q[i][1] = cvt4<FMT>(v[4], v[5], v[6], v[7], s);
           }
-          q[i][0] = cvt4<FMT>(v[0], v[1], v[2], v[3], s);
-          q[i][1] = cvt4<FMT>(v[4], v[5], v[6], v[7], s);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int r = lr0 + i;
+            float v[8];
+            if constexpr (kB == 2) {
+              const int chunk = (lc0 >> 3) ^ (r & 7);
+              const uint4 w = *reinterpret_cast<const uint4*>(st + r * 128 + chunk * 16);
+              amax2 = absmax2<DT>(absmax2<DT>(amax2, w.x), absmax2<DT>(w.y, absmax2<DT>(w.z, w.w)));
+              unpack2<DT>(w.x, v[0], v[1]);
+              unpack2<DT>(w.y, v[2], v[3]);
+              unpack2<DT>(w.z, v[4], v[5]);
+              unpack2<DT>(w.w, v[6], v[7]);
+            } else {
+              const int box = lc0 >> 5;
+              const int ch = (lc0 & 31) >> 2;
+              const uint8_t* rowp = st + box * TT::kBoxBytes + r * 128;
+              const float4 f0 = *reinterpret_cast<const float4*>(rowp + ((ch ^ (r & 7)) * 16));
+              const float4 f1 = *reinterpret_cast<const float4*>(rowp + (((ch + 1) ^ (r & 7)) * 16));
+              v[0] = f0.x; v[1] = f0.y; v[2] = f0.z; v[3] = f0.w;
+              v[4] = f1.x; v[5] = f1.y; v[6] = f1.z; v[7] = f1.w;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) amax = fmaxf(amax, fabsf(v[j]));
+            }
+            q[i][0] = cvt4<FMT>(v[0], v[1], v[2], v[3], s);
+            q[i][1] = cvt4<FMT>(v[4], v[5], v[6], v[7], s);
+          }
         }
       }
       // This warp is done reading the stage: let the producer refill it.
-      __syncwarp();
-      if (lane == 0) bar_arrive_local(empty0 + 8u * stage);
+      // Every loaded value went into the amax, and the release is predicated
+      // on the warp-wide OR of the lanes' maxima, so no lane's shared-memory
+      // load can still be in flight when the next copy lands in the stage.
+      {
+        const uint32_t dep = __reduce_or_sync(0xFFFFFFFFu, amax2 | __float_as_uint(amax));
+        if (lane == 0) bar_arrive_after(empty0 + 8u * stage, dep);
+      }
       int64_t r0 = 0, c0 = 0;
       if (!stop) {
         const uint32_t tr = t / tiles_c;
@@ -769,6 +889,8 @@ __device__ __forceinline__ void tile_tma_body(const CUtensorMap* tmIn, const Tma
             uint8_t* o = a.out + r * a.cols + c;
             if (interior && a.out8) {
               *reinterpret_cast<uint2*>(o) = make_uint2(q[i][0], q[i][1]);
+            } else if (interior) {
+              store8_any(o, q[i][0], q[i][1]);
             } else if (r < a.rows) {
 #pragma unroll
               for (int j = 0; j < 8; ++j)
@@ -826,10 +948,10 @@ __device__ __forceinline__ void tile_tma_body(const CUtensorMap* tmIn, const Tma
   amax_ticket_fold<FMT, kWsThreads>(amax, a.ring, s, rc, nblk);
 }
 
-template <int DT, int FMT, bool kDual>
+template <int DT, int FMT, bool kDual, bool kShift = false>
 __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __grid_constant__ CUtensorMap tmIn,
                                                                         const __grid_constant__ TmaTileArgs args) {
-  tile_tma_body<DT, FMT, kDual>(&tmIn, args, blockIdx.x, gridDim.x);
+  tile_tma_body<DT, FMT, kDual, kShift>(&tmIn, args, blockIdx.x, gridDim.x);
 }
 
 // Two tensors in one launch (a linear's X and W): blocks [0, split) work on
@@ -1001,41 +1123,67 @@ bool make_input_map(CUtensorMap* m, const void* in, int dtype, int64_t rows, int
                              dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
 }
 
+// Shifted-base 2-D map: rows a multiple of 16 bytes but an input base that
+// is only element-aligned.  The map starts at the base rounded down to 16
+// bytes (off_e elements earlier, inside the same 16-byte granule) and its rows
+// are cols + off_e elements long, so it ends where the tensor ends.  Boxes are
+// 64 + 16 / in_bytes elements by 128 rows, unswizzled.  (Rows that are not a
+// multiple of 16 bytes were tried through a map whose rows are g consecutive
+// input rows: slower than the register tile kernel at 8192x1537.)
+bool make_shifted_map(CUtensorMap* m, const void* in, int dtype, int64_t rows, int64_t cols, int off_e) {
+  const int eb = dtype == FP8_IN_FP32 ? 4 : 2;
+  const uint8_t* base = static_cast<const uint8_t*>(in) - off_e * eb;
+  const uint64_t dims[2] = {uint64_t(cols + off_e), uint64_t(rows)};
+  const uint64_t strides[1] = {uint64_t(cols * eb)};
+  const uint32_t box[2] = {uint32_t(kTileC + 16 / eb), uint32_t(kTileR)};
+  return encode_tiled_cached(m, eb == 4 ? CU_TENSOR_MAP_DATA_TYPE_UINT32 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base,
+                             dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+}
+
 // Resident blocks per SM of a TMA tile kernel instantiation (cached per device).
-template <int DT, int FMT, bool kDual>
+template <int DT, int FMT, bool kDual, bool kShift>
 int tma_blocks_per_sm() {
   static int cached[64] = {0};
+  constexpr int kSmem = TmaTile<DT, kShift>::kSmem;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
   if (cached[dev] == 0) {
-    auto kern = quantize_tile_tma_kernel<DT, FMT, kDual>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TmaTile<DT>::kSmem) != cudaSuccess)
-      return -1;
+    auto kern = quantize_tile_tma_kernel<DT, FMT, kDual, kShift>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem) != cudaSuccess) return -1;
     int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kWsThreads, TmaTile<DT>::kSmem) != cudaSuccess || n < 1)
-      return -1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kWsThreads, kSmem) != cudaSuccess || n < 1) return -1;
     cached[dev] = n;
   }
   return cached[dev];
 }
 
-template <int DT, int FMT>
-int launch_tile_tma(const TileArgs& t, const CUtensorMap& map, int sms, cudaStream_t st, bool dual) {
+template <int DT, int FMT, bool kDual, bool kShift>
+int launch_tile_tma1(const TileArgs& t, const CUtensorMap& map, int off_e, int sms, cudaStream_t st) {
   const WaitCfg wc = wait_cfg();
-  TmaTileArgs a{t, error_word_ptr(), wc.budget_ns, wc.stall_site};
-  const int bps = dual ? tma_blocks_per_sm<DT, FMT, true>() : tma_blocks_per_sm<DT, FMT, false>();
+  TmaTileArgs a{t, error_word_ptr(), wc.budget_ns, wc.stall_site, off_e};
+  const int bps = tma_blocks_per_sm<DT, FMT, kDual, kShift>();
   if (bps <= 0) return FP8_ERR_CUDA;
   const int grid = int(std::max<int64_t>(1, std::min<int64_t>(t.ntiles, int64_t(bps) * sms)));
-  const cudaError_t e =
-      dual ? launch_pdl(quantize_tile_tma_kernel<DT, FMT, true>, grid, kWsThreads, TmaTile<DT>::kSmem, st, 1, map, a)
-           : launch_pdl(quantize_tile_tma_kernel<DT, FMT, false>, grid, kWsThreads, TmaTile<DT>::kSmem, st, 1, map, a);
+  const cudaError_t e = launch_pdl(quantize_tile_tma_kernel<DT, FMT, kDual, kShift>, grid, kWsThreads,
+                                   TmaTile<DT, kShift>::kSmem, st, 1, map, a);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
+// off_e < 0: the 16-byte aligned kernel; otherwise the shifted-base kernel.
+template <int DT, int FMT>
+int launch_tile_tma(const TileArgs& t, const CUtensorMap& map, int off_e, int sms, cudaStream_t st, bool dual) {
+  if (off_e >= 0)
+    return dual ? launch_tile_tma1<DT, FMT, true, true>(t, map, off_e, sms, st)
+                : launch_tile_tma1<DT, FMT, false, true>(t, map, off_e, sms, st);
+  return dual ? launch_tile_tma1<DT, FMT, true, false>(t, map, 0, sms, st)
+              : launch_tile_tma1<DT, FMT, false, false>(t, map, 0, sms, st);
+}
+
 template <int DT>
-int dispatch_fmt_tile_tma(int fmt, const TileArgs& a, const CUtensorMap& map, int sms, cudaStream_t st, bool dual) {
-  return fmt == FP8_E4M3 ? launch_tile_tma<DT, FP8_E4M3>(a, map, sms, st, dual)
-                         : launch_tile_tma<DT, FP8_E5M2>(a, map, sms, st, dual);
+int dispatch_fmt_tile_tma(int fmt, const TileArgs& a, const CUtensorMap& map, int off_e, int sms, cudaStream_t st,
+                          bool dual) {
+  return fmt == FP8_E4M3 ? launch_tile_tma<DT, FP8_E4M3>(a, map, off_e, sms, st, dual)
+                         : launch_tile_tma<DT, FP8_E5M2>(a, map, off_e, sms, st, dual);
 }
 
 }  // namespace
@@ -1049,12 +1197,13 @@ namespace {
 // is null).  Arguments are already validated.
 // One quantize call resolved to its kernel: ROW, TMA tiles (16-byte aligned
 // rows) or element-aligned tiles, with the kernel arguments.
-enum QKind { kQRow = 0, kQTma = 1, kQTile = 2 };
+enum QKind { kQRow = 0, kQTma = 1, kQTile = 2, kQShift = 3 };
 struct QPlan {
   int kind, dtype, fmt, layout;
   bool aligned;  // ROW: chunks start 16-byte aligned in the input
   RowArgs ra;
   TileArgs ta;
+  int off_e;     // kQShift: element offset of the input base inside its 16-byte granule
   CUtensorMap map;
 };
 
@@ -1094,6 +1243,11 @@ int quantize_plan(const void* in, int dtype, int64_t rows, int64_t cols, int lay
       rows < (int64_t(1) << 30) && cols < (int64_t(1) << 30)) {
     if (!make_input_map(&q.map, in, dtype, rows, cols)) return FP8_ERR_CUDA;
     q.kind = kQTma;
+  } else if (n > 0 && (cols * eb) % 16 == 0 && a.ntiles < (int64_t(1) << 30) && rows < (int64_t(1) << 30) &&
+             cols < (int64_t(1) << 30)) {
+    q.off_e = int((reinterpret_cast<uintptr_t>(in) & 15) / uintptr_t(eb));
+    if (!make_shifted_map(&q.map, in, dtype, rows, cols, q.off_e)) return FP8_ERR_CUDA;
+    q.kind = kQShift;
   } else {
     q.kind = kQTile;
   }
@@ -1109,11 +1263,12 @@ int quantize_launch(const QPlan& q, int sms, cudaStream_t st) {
       default: return dispatch_fmt_row<FP8_IN_FP32>(q.fmt, q.ra, sms, st, q.aligned);
     }
   }
-  if (q.kind == kQTma) {
+  if (q.kind == kQTma || q.kind == kQShift) {
+    const int off_e = q.kind == kQShift ? q.off_e : -1;
     switch (q.dtype) {
-      case FP8_IN_BF16: return dispatch_fmt_tile_tma<FP8_IN_BF16>(q.fmt, q.ta, q.map, sms, st, dual);
-      case FP8_IN_FP16: return dispatch_fmt_tile_tma<FP8_IN_FP16>(q.fmt, q.ta, q.map, sms, st, dual);
-      default: return dispatch_fmt_tile_tma<FP8_IN_FP32>(q.fmt, q.ta, q.map, sms, st, dual);
+      case FP8_IN_BF16: return dispatch_fmt_tile_tma<FP8_IN_BF16>(q.fmt, q.ta, q.map, off_e, sms, st, dual);
+      case FP8_IN_FP16: return dispatch_fmt_tile_tma<FP8_IN_FP16>(q.fmt, q.ta, q.map, off_e, sms, st, dual);
+      default: return dispatch_fmt_tile_tma<FP8_IN_FP32>(q.fmt, q.ta, q.map, off_e, sms, st, dual);
     }
   }
   switch (q.dtype) {

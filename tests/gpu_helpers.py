@@ -39,12 +39,15 @@ def assert_ring_equal(ring_gpu, ring_ref):
 
 def quantize_both(x_cpu, fmt, layout, ring_gpu, misalign=False):
     """Run one quantize on the GPU (through the C ABI) and on the oracle from the same
-    ring state.  Returns (gpu_out, gpu_out_t, ref_out, ref_out_t, ref_ring)."""
+    ring state.  Returns (gpu_out, gpu_out_t, ref_out, ref_out_t, ref_ring).
+    ``misalign``: False, True (one element past a 256-byte aligned base) or an
+    element offset."""
     ref_ring = oracle_ring_from(ring_gpu)
     if misalign:
-        flat = torch.empty(x_cpu.numel() + 1, dtype=x_cpu.dtype, device="cuda")
-        flat[1:].copy_(x_cpu.reshape(-1))
-        x_dev = flat[1:].view(x_cpu.shape)
+        k = int(misalign)
+        flat = torch.empty(x_cpu.numel() + k, dtype=x_cpu.dtype, device="cuda")
+        flat[k:].copy_(x_cpu.reshape(-1))
+        x_dev = flat[k:].view(x_cpu.shape)
     else:
         x_dev = x_cpu.to("cuda")
     out, out_t = ops.quantize(x_dev, fmt, layout, ring_gpu)

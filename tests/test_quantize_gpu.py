@@ -28,6 +28,7 @@ def _dev(x, misalign):
 
 
 def _run_and_compare(x, fmt, layout, ring, misalign=False):
+    # misalign: False, True (one element) or an element offset of the input base
     out, out_t, r_out, r_out_t, r_ring = quantize_both(x, fmt, layout, ring, misalign)
     if layout in (ops.ROW, ops.DUAL):
         assert_bytes_equal(out, r_out, "out")
@@ -52,6 +53,26 @@ def test_small_shapes_two_calls(dtype, fmt, layout, misalign):
         for step in range(2):  # second call uses the delayed scale published by the first
             x = S.quant_sweep_input(r, c, dtype, vs, seed=31 * i + step)
             _run_and_compare(x, fmt, layout, ring, misalign)
+
+
+# Transposed / dual inputs whose rows are a multiple of 16 bytes but whose base
+# is only element-aligned go through a 2-D map that starts at the base rounded
+# down to 16 bytes (the shifted-base kernel); other element-aligned inputs go
+# through the register tile kernel.  Every element offset of the base inside
+# its 16-byte granule, ragged rows and columns, both kernels.
+BASE_OFFSET_SHAPES = [(8, 8), (130, 64), (129, 72), (257, 1536), (9, 37), (255, 1001)]
+
+
+@pytest.mark.parametrize("dtype", DTYPES)
+@pytest.mark.parametrize("layout", [ops.TRANSPOSED, ops.DUAL])
+def test_every_base_offset(dtype, layout):
+    per = 16 // (4 if dtype == "fp32" else 2)
+    for i, (r, c) in enumerate(BASE_OFFSET_SHAPES):
+        for off in range(per):
+            ring = ops.Ring()
+            for step in range(2):
+                x = S.quant_sweep_input(r, c, dtype, [1.0, 1e-3][step], seed=97 * i + 7 * off + step)
+                _run_and_compare(x, ops.E4M3 if (i + off) % 2 else ops.E5M2, layout, ring, off)
 
 
 def test_pr1_linear_three_delayed_steps():

@@ -44,11 +44,18 @@ def _stalled(site, fn):
     assert rc == ops.FP8_ERR_DEVICE_TIMEOUT and where == site, (rc, where)
 
 
+@pytest.mark.parametrize("shifted", [False, True])
 @pytest.mark.parametrize("layout", [ops.TRANSPOSED, ops.DUAL])
-def test_quantize_wait_runs_out_then_the_next_call_is_exact(layout):
-    """The TMA tile kernel (transposed / dual of 16-byte aligned rows)."""
+def test_quantize_wait_runs_out_then_the_next_call_is_exact(layout, shifted):
+    """The TMA tile kernels (transposed / dual of rows that are a multiple of
+    16 bytes): 16-byte aligned base, and a base one element past 16 bytes."""
     x = S.quant_sweep_input(2048, 1536, "bf16", 1.0, seed=9)
-    xd = x.cuda()
+    if shifted:
+        flat = torch.empty(x.numel() + 1, dtype=x.dtype, device="cuda")
+        flat[1:].copy_(x.reshape(-1))
+        xd = flat[1:].view(x.shape)
+    else:
+        xd = x.cuda()
     failed = ops.Ring()
     _stalled(ops.SITE_QUANTIZE_TMA, lambda: ops.quantize(xd, ops.E4M3, layout, failed))
     assert all(int(v) == 0 for v in failed.state()[4]), "the stopped call still clears the scratch words"

@@ -155,8 +155,8 @@ int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t
  * launch, such as a linear's X and W before its forward GEMM.
  *
  * When both resolve to the same kernel (same dtype, fmt and layout; ROW
- * inputs with the same 16-byte alignment, or T/DUAL inputs with 16-byte rows
- * on TMA) and neither is empty, one grid is split between them in proportion
+ * inputs with the same 16-byte alignment, or T/DUAL inputs with 16-byte
+ * aligned bases and rows that are a multiple of 16 bytes) and neither is empty, one grid is split between them in proportion
  * to their sizes; each set of blocks has its own amax ticket and folds its
  * own ring.  Otherwise the two run one after the other on `stream`.  Each
  * result (codes, ring, scales) is exactly that of the fp8_quantize call with
@@ -501,9 +501,11 @@ int fp8_device_info(int* sm_count, const char** arch);
  *               wait runs out after budget_ns:
  *                 4  fp8_mm family: the epilogue's wait for an accumulator;
  *                 6  fp8_quantize family, transposed and dual layouts of
- *                    inputs whose rows are 16-byte aligned (the TMA tile
- *                    kernel): the consumers' wait for a staged input tile.
- *                    The row layout's kernel has no waits to shorten.
+ *                    inputs whose rows are a multiple of 16 bytes (the TMA
+ *                    tile kernels, 16-byte aligned or element-aligned base):
+ *                    the consumers' wait for a staged input tile.  The row
+ *                    layout's kernel and the transposed / dual kernel of
+ *                    other row widths (plain loads) have no waits to shorten.
  * A wait that runs out records its site code in the device error word
  * (fp8_device_error), the kernel stops early and returns; its outputs are
  * undefined and the ring of a stalled quantize has folded an amax of 0.

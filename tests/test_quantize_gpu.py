@@ -75,6 +75,27 @@ def test_every_base_offset(dtype, layout):
                 _run_and_compare(x, ops.E4M3 if (i + off) % 2 else ops.E5M2, layout, ring, off)
 
 
+@pytest.mark.parametrize("dtype,shape", [("bf16", (257, 1536)), ("fp32", (130, 68)), ("bf16", (9, 37))])
+def test_dual_row_output_at_every_byte_offset(dtype, shape):
+    """DUAL's row-layout output written at every byte offset of an 8-byte word:
+    interior tile rows take the widest aligned stores each offset allows
+    (8, 4, 2 and 1 bytes)."""
+    r, c = shape
+    for off in range(8):
+        ring = ops.Ring()
+        ref = OR.Ring()
+        x = S.quant_sweep_input(r, c, dtype, 1.0, seed=300 + off)
+        flat = torch.empty(r * c + 8, dtype=torch.uint8, device="cuda")
+        out = flat[off:off + r * c].view(r, c)
+        out_t = torch.empty((c, r), dtype=torch.uint8, device="cuda")
+        ops.quantize(x.cuda(), ops.E4M3, ops.DUAL, ring, out, out_t)
+        torch.cuda.synchronize()
+        r_out, r_out_t, _ = OR.quantize(x, ops.E4M3, ops.DUAL, ref)
+        assert_bytes_equal(out, r_out, f"out (byte offset {off})")
+        assert_bytes_equal(out_t, r_out_t, f"out_t (byte offset {off})")
+        assert_ring_equal(ring, ref)
+
+
 def test_pr1_linear_three_delayed_steps():
     """X [128,512] row and W [256,512] dual, E4M3, rings carried over 3 steps."""
     rx, rw = ops.Ring(), ops.Ring()

@@ -8,10 +8,10 @@ workload (hidden 1536, FFN 4096) at M = 8192 tokens, for both linear shapes
   fwd  Y  = Xq . Wq^T * sx*sw + b      (M x N x 1536)
   dX   = Gq . (W^T)q^T * sg*sw          (M x 1536 x N, A = E5M2)
   dW   = (G^T)q . (X^T)q^T * sg*sx      (N x 1536 x M, A = E5M2)
-X and W of a linear go through fp8_quantize_pair and its dX and dW through
-fp8_mm_pair (one launch each when the library pairs them), so a step is 8 to
-12 kernel launches, counted with fp8_launch_count while the step's graph is
-captured.  The device-timed steps
+X, W and G of a linear go through fp8_quantize_multi and its dX and dW
+through fp8_mm_pair (one launch each when the library fuses them), so a step
+is 6 to 12 kernel launches, counted with fp8_launch_count while the step's
+graph is captured.  The device-timed steps
 replay a CUDA graph of the step; the end-to-end figure calls the C ABI
 directly every step with host copies in and out.
 
@@ -222,7 +222,13 @@ class Linear:
         self.ws = None  # stream-K workspace shared by the step's GEMMs (set by build_workload)
 
     def quantize(self, ops, x, g, ev=None):
-        # X and W (both needed by the forward GEMM) in one fp8_quantize_pair launch.
+        # X, W (E4M3) and G (E5M2) in one fp8_quantize_multi launch.
+        ops.quantize_multi([dict(x=x, fmt=ops.E4M3, layout=ops.DUAL, ring=self.rx, out=self.xq, out_t=self.xq_t),
+                            dict(x=self.w, fmt=ops.E4M3, layout=ops.DUAL, ring=self.rw, out=self.wq, out_t=self.wq_t),
+                            dict(x=g, fmt=ops.E5M2, layout=ops.DUAL, ring=self.rg, out=self.gq, out_t=self.gq_t)])
+
+    def quantize_paired(self, ops, x, g):
+        # The previous schedule: X and W in one fp8_quantize_pair launch, G alone.
         ops.quantize_pair(dict(x=x, fmt=ops.E4M3, layout=ops.DUAL, ring=self.rx, out=self.xq, out_t=self.xq_t),
                           dict(x=self.w, fmt=ops.E4M3, layout=ops.DUAL, ring=self.rw, out=self.wq, out_t=self.wq_t))
         ops.quantize(g, ops.E5M2, ops.DUAL, self.rg, self.gq, self.gq_t)

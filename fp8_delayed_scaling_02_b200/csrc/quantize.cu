@@ -954,16 +954,28 @@ __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __g
   tile_tma_body<DT, FMT, kDual, kShift>(&tmIn, args, blockIdx.x, gridDim.x);
 }
 
-// Two tensors in one launch (a linear's X and W): blocks [0, split) work on
-// tensor 0, the rest on tensor 1, each set with its own ring, ticket and
-// tile counter.
-template <int DT, int FMT, bool kDual>
-__global__ void __launch_bounds__(kWsThreads)
-    quantize_tile_tma_pair_kernel(const __grid_constant__ CUtensorMap tm0, const __grid_constant__ TmaTileArgs a0,
-                                  const __grid_constant__ CUtensorMap tm1, const __grid_constant__ TmaTileArgs a1,
-                                  const unsigned split) {
-  if (blockIdx.x < split) tile_tma_body<DT, FMT, kDual>(&tm0, a0, blockIdx.x, split);
-  else tile_tma_body<DT, FMT, kDual>(&tm1, a1, blockIdx.x - split, gridDim.x - split);
+// Several tensors in one launch (a linear's X, W and G): blocks
+// [split[s], split[s+1]) work on tensor s, each set with its own ring, amax
+// ticket and tile counter, so each tensor's result is exactly that of its
+// own launch.  The tensors share the dtype and layout (one instantiation of
+// the tile body per format, chosen per block).
+constexpr int kMaxMulti = 8;
+
+struct TmaMultiArgs {
+  CUtensorMap maps[kMaxMulti];
+  TmaTileArgs a[kMaxMulti];
+  int fmt[kMaxMulti];
+  unsigned split[kMaxMulti + 1];
+  int n;
+};
+
+template <int DT, bool kDual>
+__global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_multi_kernel(const __grid_constant__ TmaMultiArgs m) {
+  int s = 0;
+  while (s + 1 < m.n && blockIdx.x >= m.split[s + 1]) ++s;
+  const unsigned blk = blockIdx.x - m.split[s], nblk = m.split[s + 1] - m.split[s];
+  if (m.fmt[s] == FP8_E5M2) tile_tma_body<DT, FP8_E5M2, kDual>(&m.maps[s], m.a[s], blk, nblk);
+  else tile_tma_body<DT, FP8_E4M3, kDual>(&m.maps[s], m.a[s], blk, nblk);
 }
 
 // ---- current scaling: amax pass ---------------------------------------------------
@@ -1317,64 +1329,99 @@ int launch_row_pair1(const RowArgs& a0, const RowArgs& a1, int sms, cudaStream_t
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
-template <int DT, int FMT, bool kDual>
-int launch_tile_tma_pair1(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
+// One launch for n TMA-tile quantize plans with the same dtype and layout,
+// each non-empty and each on its own ring: the wave of resident blocks is
+// split between the tensors in proportion to their tiles (at least one block
+// each, never more blocks than tiles).
+template <int DT, bool kDual>
+int launch_tile_tma_multi1(const QPlan* const* qs, int n, int sms, cudaStream_t st) {
   static int cached[64] = {0};
-  auto kern = quantize_tile_tma_pair_kernel<DT, FMT, kDual>;
+  auto kern = quantize_tile_tma_multi_kernel<DT, kDual>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return FP8_ERR_CUDA;
   if (cached[dev] == 0) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, TmaTile<DT>::kSmem) != cudaSuccess)
       return FP8_ERR_CUDA;
-    int n = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, kWsThreads, TmaTile<DT>::kSmem) != cudaSuccess || n < 1)
+    int b = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, kern, kWsThreads, TmaTile<DT>::kSmem) != cudaSuccess || b < 1)
       return FP8_ERR_CUDA;
-    cached[dev] = n;
+    cached[dev] = b;
   }
   const int64_t G = int64_t(cached[dev]) * sms;
-  const int64_t t0 = q0.ta.ntiles, t1 = q1.ta.ntiles;
-  const int64_t g0 = std::min<int64_t>(share0(G, t0, t1), t0);
-  const int64_t g1 = std::min<int64_t>(G - g0, t1);
+  int64_t T = 0;
+  for (int i = 0; i < n; ++i) T += qs[i]->ta.ntiles;
   const WaitCfg wc = wait_cfg();
-  const TmaTileArgs a0{q0.ta, error_word_ptr(), wc.budget_ns, wc.stall_site};
-  const TmaTileArgs a1{q1.ta, error_word_ptr(), wc.budget_ns, wc.stall_site};
-  const cudaError_t e = launch_pdl(kern, dim3(unsigned(g0 + g1)), kWsThreads, TmaTile<DT>::kSmem, st, 1, q0.map, a0,
-                                   q1.map, a1, unsigned(g0));
+  TmaMultiArgs m;
+  std::memset(&m, 0, sizeof(m));
+  m.n = n;
+  m.split[0] = 0;
+  for (int i = 0; i < n; ++i) {
+    const int64_t t = qs[i]->ta.ntiles;
+    const int64_t g = std::min<int64_t>(t, std::max<int64_t>(1, (G - n) * t / T));
+    m.split[i + 1] = m.split[i] + unsigned(g);
+    m.maps[i] = qs[i]->map;
+    m.a[i] = TmaTileArgs{qs[i]->ta, error_word_ptr(), wc.budget_ns, wc.stall_site, 0};
+    m.fmt[i] = qs[i]->fmt;
+  }
+  const cudaError_t e = launch_pdl(kern, dim3(m.split[n]), kWsThreads, TmaTile<DT>::kSmem, st, 1, m);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
 }
 
+int launch_tile_tma_multi(const QPlan* const* qs, int n, int sms, cudaStream_t st) {
+  const bool dual = qs[0]->layout == FP8_LAYOUT_DUAL;
+  switch (qs[0]->dtype) {
+    case FP8_IN_BF16:
+      return dual ? launch_tile_tma_multi1<FP8_IN_BF16, true>(qs, n, sms, st)
+                  : launch_tile_tma_multi1<FP8_IN_BF16, false>(qs, n, sms, st);
+    case FP8_IN_FP16:
+      return dual ? launch_tile_tma_multi1<FP8_IN_FP16, true>(qs, n, sms, st)
+                  : launch_tile_tma_multi1<FP8_IN_FP16, false>(qs, n, sms, st);
+    default:
+      return dual ? launch_tile_tma_multi1<FP8_IN_FP32, true>(qs, n, sms, st)
+                  : launch_tile_tma_multi1<FP8_IN_FP32, false>(qs, n, sms, st);
+  }
+}
+
+// TMA-tile plans that can share one launch: same dtype and layout, each
+// non-empty (formats may differ).
+bool tma_fusable(const QPlan* const* qs, int n) {
+  for (int i = 0; i < n; ++i) {
+    if (qs[i]->kind != kQTma || qs[i]->ta.ntiles <= 0) return false;
+    if (qs[i]->dtype != qs[0]->dtype || qs[i]->layout != qs[0]->layout) return false;
+  }
+  return true;
+}
+
 template <int DT, int FMT>
-int launch_pair_dt_fmt(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
-  if (q0.kind == kQRow)
-    return q0.aligned ? launch_row_pair1<DT, FMT, true>(q0.ra, q1.ra, sms, st)
-                      : launch_row_pair1<DT, FMT, false>(q0.ra, q1.ra, sms, st);
-  return q0.layout == FP8_LAYOUT_DUAL ? launch_tile_tma_pair1<DT, FMT, true>(q0, q1, sms, st)
-                                      : launch_tile_tma_pair1<DT, FMT, false>(q0, q1, sms, st);
+int launch_row_pair_dt_fmt(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
+  return q0.aligned ? launch_row_pair1<DT, FMT, true>(q0.ra, q1.ra, sms, st)
+                    : launch_row_pair1<DT, FMT, false>(q0.ra, q1.ra, sms, st);
 }
 
 template <int DT>
-int launch_pair_dt(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
-  return q0.fmt == FP8_E4M3 ? launch_pair_dt_fmt<DT, FP8_E4M3>(q0, q1, sms, st)
-                            : launch_pair_dt_fmt<DT, FP8_E5M2>(q0, q1, sms, st);
+int launch_row_pair_dt(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
+  return q0.fmt == FP8_E4M3 ? launch_row_pair_dt_fmt<DT, FP8_E4M3>(q0, q1, sms, st)
+                            : launch_row_pair_dt_fmt<DT, FP8_E5M2>(q0, q1, sms, st);
 }
 
 // Both calls in one launch when they resolve to the same kernel (ROW with
-// the same alignment, or TMA tiles with the same layout) and neither is
-// empty; otherwise one launch each, in order.
+// the same alignment and format, or TMA tiles with the same layout) and
+// neither is empty; otherwise one launch each, in order.
 int quantize_pair_dispatch(QPlan& q0, QPlan& q1, cudaStream_t st) {
   const int sms = sm_count_current();
   if (sms <= 0) return FP8_ERR_CUDA;
-  const bool same = q0.kind == q1.kind && q0.dtype == q1.dtype && q0.fmt == q1.fmt && q0.layout == q1.layout &&
-                    (q0.kind == kQTma || (q0.kind == kQRow && q0.aligned == q1.aligned));
-  const bool nonempty = q0.kind == kQRow ? (q0.ra.n > 0 && q1.ra.n > 0) : (q0.ta.ntiles > 0 && q1.ta.ntiles > 0);
-  if (!same || !nonempty) {
+  const QPlan* qs[2] = {&q0, &q1};
+  if (tma_fusable(qs, 2)) return launch_tile_tma_multi(qs, 2, sms, st);
+  const bool rows = q0.kind == kQRow && q1.kind == kQRow && q0.dtype == q1.dtype && q0.fmt == q1.fmt &&
+                    q0.aligned == q1.aligned && q0.ra.n > 0 && q1.ra.n > 0;
+  if (!rows) {
     const int rc = quantize_launch(q0, sms, st);
     return rc != FP8_OK ? rc : quantize_launch(q1, sms, st);
   }
   switch (q0.dtype) {
-    case FP8_IN_BF16: return launch_pair_dt<FP8_IN_BF16>(q0, q1, sms, st);
-    case FP8_IN_FP16: return launch_pair_dt<FP8_IN_FP16>(q0, q1, sms, st);
-    default: return launch_pair_dt<FP8_IN_FP32>(q0, q1, sms, st);
+    case FP8_IN_BF16: return launch_row_pair_dt<FP8_IN_BF16>(q0, q1, sms, st);
+    case FP8_IN_FP16: return launch_row_pair_dt<FP8_IN_FP16>(q0, q1, sms, st);
+    default: return launch_row_pair_dt<FP8_IN_FP32>(q0, q1, sms, st);
   }
 }
 
@@ -1437,6 +1484,41 @@ extern "C" int fp8_quantize_pair(const fp8_quantize_args* q0, const fp8_quantize
     return rc != FP8_OK ? rc : quantize_launch(p[1], sms, st);
   }
   return quantize_pair_dispatch(p[0], p[1], st);
+}
+
+extern "C" int fp8_quantize_multi(const fp8_quantize_args* qs, int n, fp8_stream_t stream) {
+  if (qs == nullptr || n < 1 || n > kMaxMulti) return FP8_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    const fp8_ring& ring = qs[i].ring;
+    if (!ring.history || !ring.idx || !ring.scale || !ring.scale_inv || !ring.scratch) return FP8_ERR_INVALID_ARG;
+    const int rc = check_quantize_args(qs[i].in, qs[i].dtype, qs[i].rows, qs[i].cols, qs[i].layout, qs[i].fmt,
+                                       qs[i].out, qs[i].out_t, ring.scratch);
+    if (rc != FP8_OK) return rc;
+  }
+  QPlan p[kMaxMulti];
+  const QPlan* ptrs[kMaxMulti];
+  for (int i = 0; i < n; ++i) {
+    const fp8_ring& ring = qs[i].ring;
+    const RingArgs r{ring.history, ring.idx, ring.scale, ring.scale_inv, ring.scratch};
+    const int rc = quantize_plan(qs[i].in, qs[i].dtype, qs[i].rows, qs[i].cols, qs[i].layout, qs[i].fmt, r,
+                                 qs[i].out, qs[i].out_t, p[i]);
+    if (rc != FP8_OK) return rc;
+    ptrs[i] = &p[i];
+  }
+  bool distinct = true;  // a ring cannot serve two calls of one launch
+  for (int i = 0; i < n; ++i)
+    for (int j = i + 1; j < n; ++j)
+      if (qs[i].ring.scratch == qs[j].ring.scratch || qs[i].ring.history == qs[j].ring.history) distinct = false;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = sm_count_current();
+  if (sms <= 0) return FP8_ERR_CUDA;
+  if (distinct && n > 1 && tma_fusable(ptrs, n)) return launch_tile_tma_multi(ptrs, n, sms, st);
+  if (distinct && n == 2) return quantize_pair_dispatch(p[0], p[1], st);
+  for (int i = 0; i < n; ++i) {
+    const int rc = quantize_launch(p[i], sms, st);
+    if (rc != FP8_OK) return rc;
+  }
+  return FP8_OK;
 }
 
 extern "C" int fp8_quantize_local(const void* in, int dtype, int64_t rows, int64_t cols, int layout, int fmt,

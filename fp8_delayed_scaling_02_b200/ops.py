@@ -96,6 +96,8 @@ def lib():
         L.fp8_mm_pair.restype = i32
         L.fp8_quantize_pair.argtypes = [vp, vp, vp]
         L.fp8_quantize_pair.restype = i32
+        L.fp8_quantize_multi.argtypes = [vp, i32, vp]
+        L.fp8_quantize_multi.restype = i32
         L.fp8_mm_ex.argtypes = [vp, vp, ctypes.c_size_t, vp]
         L.fp8_mm_ex.restype = i32
         L.fp8_launch_count.argtypes = []
@@ -206,14 +208,10 @@ class CQuantArgs(ctypes.Structure):
                 ("out_t", ctypes.c_void_p)]
 
 
-def quantize_pair(q0, q1, stream=None):
-    """fp8_quantize_pair: two quantize calls (own rings) in one launch, e.g. a linear's X and W.
-
-    q0, q1: dicts of ``quantize`` arguments (x, fmt, layout, ring and
-    optionally out, out_t).  Returns ((out0, out_t0), (out1, out_t1)).
-    """
+def _quant_args(qs):
+    """CQuantArgs and (out, out_t) for a sequence of ``quantize`` argument dicts."""
     args, res = [], []
-    for q in (q0, q1):
+    for q in qs:
         x, layout = q["x"], q["layout"]
         if x.dim() != 2 or not x.is_contiguous():
             raise ValueError("x must be a contiguous 2-D tensor")
@@ -228,10 +226,36 @@ def quantize_pair(q0, q1, stream=None):
         args.append(CQuantArgs(x.data_ptr(), IN_DTYPE[x.dtype], rows, cols, layout, q["fmt"], q["ring"].c(),
                                _ptr(out), _ptr(out_t)))
         res.append((out, out_t))
+    return args, res
+
+
+def quantize_pair(q0, q1, stream=None):
+    """fp8_quantize_pair: two quantize calls (own rings) in one launch, e.g. a linear's X and W.
+
+    q0, q1: dicts of ``quantize`` arguments (x, fmt, layout, ring and
+    optionally out, out_t).  Returns ((out0, out_t0), (out1, out_t1)).
+    """
+    args, res = _quant_args((q0, q1))
     rc = (_LIB or lib()).fp8_quantize_pair(ctypes.byref(args[0]), ctypes.byref(args[1]),
                                            _stream(stream, q0["x"].get_device()))
     _check(rc, "fp8_quantize_pair")
     return res[0], res[1]
+
+
+def quantize_multi(qs, stream=None):
+    """fp8_quantize_multi: up to 8 quantize calls (own rings) in one launch, e.g. a linear's X, W and G.
+
+    qs: a sequence of dicts of ``quantize`` arguments (x, fmt, layout, ring and
+    optionally out, out_t).  Returns a list of (out, out_t).
+    """
+    qs = list(qs)
+    if not qs:
+        raise ValueError("quantize_multi needs at least one call")
+    args, res = _quant_args(qs)
+    arr = (CQuantArgs * len(args))(*args)
+    rc = (_LIB or lib()).fp8_quantize_multi(arr, len(args), _stream(stream, qs[0]["x"].get_device()))
+    _check(rc, "fp8_quantize_multi")
+    return res
 
 
 def quantize_local(x, fmt, layout, ring, amax=None, out=None, out_t=None, stream=None):

@@ -11,6 +11,7 @@
  *                 fp32 bias, optional batch with stride-0 broadcast.
  *
  * Around them: fp8_quantize_pair / fp8_mm_pair (two calls in one launch),
+ * fp8_quantize_multi (up to eight quantize calls in one launch),
  * fp8_mm_ws (stream-K tail through a caller workspace), fp8_mm_ex (FP8 bias,
  * FP8 output with delayed output scaling), fp8_quantize_current
  * (current scaling), fp8_quantize_local + fp8_ring_fold (data-parallel
@@ -154,11 +155,12 @@ int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t
  * fp8_quantize_pair -- two fp8_quantize calls (each on its own ring) in one
  * launch, such as a linear's X and W before its forward GEMM.
  *
- * When both resolve to the same kernel (same dtype, fmt and layout; ROW
- * inputs with the same 16-byte alignment, or T/DUAL inputs with 16-byte
- * aligned bases and rows that are a multiple of 16 bytes) and neither is empty, one grid is split between them in proportion
- * to their sizes; each set of blocks has its own amax ticket and folds its
- * own ring.  Otherwise the two run one after the other on `stream`.  Each
+ * When both resolve to the same kernel (ROW inputs with the same dtype,
+ * fmt and 16-byte alignment; or T/DUAL inputs with the same dtype and layout,
+ * 16-byte aligned bases and rows that are a multiple of 16 bytes, formats free)
+ * and neither is empty, one grid is split between them in proportion to
+ * their sizes; each set of blocks has its own amax ticket and folds its own
+ * ring.  Otherwise the two run one after the other on `stream`.  Each
  * result (codes, ring, scales) is exactly that of the fp8_quantize call with
  * the same arguments.  If both name the same ring the two calls run in order
  * (a ring cannot serve two calls at once).
@@ -176,6 +178,30 @@ typedef struct {
   uint8_t* out_t;
 } fp8_quantize_args;
 int fp8_quantize_pair(const fp8_quantize_args* q0, const fp8_quantize_args* q1, fp8_stream_t stream);
+
+/*
+ * fp8_quantize_multi -- n fp8_quantize calls (each on its own ring) in one
+ * launch, such as a linear's X, W and G before its GEMMs.
+ *
+ * When every call is transposed or dual with the same dtype and layout, a
+ * 16-byte aligned base, rows that are a multiple of 16 bytes and a
+ * non-empty input (the formats may differ), and no ring is named twice, one
+ * grid is split between them in proportion to their tiles: each tensor's
+ * blocks claim its own tiles, reduce its own amax and fold its own ring, so
+ * the launch's start-up and end costs are paid once instead of n times.
+ * Otherwise the calls run in order on `stream` (two calls as
+ * fp8_quantize_pair).  Each result (codes, ring, scales) is exactly that of
+ * the fp8_quantize call with the same arguments.
+ *   qs      host array of n structs; each field as the fp8_quantize argument
+ *           of that name.
+ *   n       1 .. 8.
+ * Errors: FP8_ERR_INVALID_ARG for a null qs or n outside 1 .. 8; otherwise as
+ * fp8_quantize, every call checked (in order) before anything is launched.
+ * FP8_ERR_CUDA from a launch of the in-order fallback leaves the earlier
+ * calls enqueued.  The pages have no counterpart (a B200 scheduling
+ * addition).
+ */
+int fp8_quantize_multi(const fp8_quantize_args* qs, int n, fp8_stream_t stream);
 
 /*
  * fp8_quantize_local / fp8_ring_fold -- delayed scaling of a tensor sharded

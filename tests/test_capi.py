@@ -30,7 +30,7 @@ def test_header_declares_the_boundary():
          "fp8_quantize_static_scratch", "fp8_quantize_current", "fp8_bias_grad", "fp8_linear_forward",
          "fp8_linear_backward", "fp8_mm_ws", "fp8_mm_workspace_bytes", "fp8_quantize_local", "fp8_ring_fold",
          "fp8_mm_pair", "fp8_launch_count", "fp8_quantize_pair", "fp8_mm_ex", "fp8_debug_wait",
-         "fp8_mm_launch_shape"])
+         "fp8_mm_launch_shape", "fp8_quantize_multi"])
 
 
 def test_library_exports_every_declared_symbol(L):
@@ -175,6 +175,18 @@ def test_paired_entry_points_reject_bad_arguments_without_cuda(L):
     assert L.fp8_quantize_pair(ctypes.byref(q_args(fmt=2)), ctypes.byref(gq), None) == ops.FP8_ERR_INVALID_ARG
     assert L.fp8_quantize_pair(ctypes.byref(gq), ctypes.byref(q_args(ring=ops.CRing(0, 0, 0, 0, 0))),
                                None) == ops.FP8_ERR_INVALID_ARG
+
+    def arr(*qs):
+        return (ops.CQuantArgs * len(qs))(*qs)
+
+    assert L.fp8_quantize_multi(None, 1, None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_quantize_multi(arr(gq), 0, None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_quantize_multi(arr(*([gq] * 9)), 9, None) == ops.FP8_ERR_INVALID_ARG
+    # Every call is checked before anything launches: a bad third call
+    # returns its own status (here, with no GPU, a launch would give FP8_ERR_CUDA).
+    assert L.fp8_quantize_multi(arr(gq, gq, q_args(layout=3)), 3, None) == ops.FP8_ERR_INVALID_ARG
+    assert L.fp8_quantize_multi(arr(gq, q_args(inp=0x10001), gq), 3, None) == ops.FP8_ERR_UNSUPPORTED
+    assert L.fp8_quantize_multi(arr(gq, q_args(layout=2, out_t=0)), 2, None) == ops.FP8_ERR_INVALID_ARG
 
 
 def test_linear_composites_check_every_call_before_launching(L):

@@ -295,6 +295,77 @@ def test_quantize_pair_equals_two_calls(s0, s1, layout):
             assert torch.equal(r.buf, e.buf)
 
 
+QMULTI = [
+    # A 1.2B-model linear's X, W and G (one launch: same dtype and layout, formats differ).
+    [((8192, 1536), "bf16", 0), ((4096, 1536), "bf16", 0), ((8192, 4096), "bf16", 1)],
+    # Eight tensors of very different sizes, one launch.
+    [((2048, 1536), "fp32", 1), ((128, 64), "fp32", 0), ((130, 64), "fp32", 1), ((1, 4), "fp32", 0),
+     ((64, 4), "fp32", 0), ((300, 68), "fp32", 1), ((1000, 128), "fp32", 0), ((129, 8), "fp32", 1)],
+    # Not fusable (an odd width, an empty input): calls in order.
+    [((256, 512), "bf16", 0), ((300, 1537), "bf16", 1), ((0, 64), "bf16", 0)],
+    [((777, 512), "fp16", 1)],
+]
+
+
+@pytest.mark.parametrize("layout", [ops.TRANSPOSED, ops.DUAL])
+@pytest.mark.parametrize("case", range(len(QMULTI)))
+def test_quantize_multi_equals_the_single_calls(case, layout):
+    specs = QMULTI[case]
+    rings = [ops.Ring() for _ in specs]
+    refs = [ops.Ring() for _ in specs]
+    for step in range(3):
+        qs, expect = [], []
+        for i, ((rows, cols), dt, fmt) in enumerate(specs):
+            x = S.quant_sweep_input(rows, cols, dt, [1.0, 1e3, 1e-3][step], seed=700 + 10 * step + i).cuda()
+            qs.append(dict(x=x, fmt=fmt, layout=layout, ring=rings[i]))
+            expect.append(ops.quantize(x, fmt, layout, refs[i]))
+        got = ops.quantize_multi(qs)
+        torch.cuda.synchronize()
+        for (o, t), (eo, et) in zip(got, expect):
+            for a, b in ((o, eo), (t, et)):
+                assert (a is None) == (b is None)
+                if a is not None:
+                    assert torch.equal(a, b)
+        for r, e in zip(rings, refs):
+            assert torch.equal(r.buf, e.buf)
+
+
+def test_quantize_multi_linear_matches_the_oracle():
+    """X, W (E4M3) and G (E5M2) of the 1.2B-model FFN linear at M = 2048, dual
+    layout, one launch per step over 3 delayed steps: every byte and ring
+    against the oracle."""
+    shapes = [((2048, 1536), ops.E4M3), ((4096, 1536), ops.E4M3), ((2048, 4096), ops.E5M2)]
+    rings = [ops.Ring() for _ in shapes]
+    refs = [OR.Ring() for _ in shapes]
+    for step in range(3):
+        xs = [S.quant_sweep_input(r, c, "bf16", [1.0, 30.0, 1e-3][step], seed=900 + 10 * step + i)
+              for i, ((r, c), _) in enumerate(shapes)]
+        got = ops.quantize_multi([dict(x=x.cuda(), fmt=f, layout=ops.DUAL, ring=rg)
+                                  for x, ((_, f)), rg in zip(xs, shapes, rings)])
+        torch.cuda.synchronize()
+        for x, (_, f), (o, t), ref, rg in zip(xs, shapes, got, refs, rings):
+            codes = oracle_codes(x, ref.scale, f)
+            OR.fold(ref, OR.amax(OR.to_float32(x)), f)
+            assert_bytes_equal(o, codes, "out")
+            assert_bytes_equal(t, np.ascontiguousarray(codes.T), "out_t")
+            assert_ring_equal(rg, ref)
+
+
+def test_quantize_multi_with_one_ring_twice_runs_in_order():
+    ring, other, ref, ref_other = ops.Ring(), ops.Ring(), ops.Ring(), ops.Ring()
+    xs = [S.quant_sweep_input(512, 256, "bf16", v, seed=20 + i).cuda() for i, v in enumerate((1.0, 1e3, 1e-3))]
+    got = ops.quantize_multi([dict(x=xs[0], fmt=ops.E4M3, layout=ops.DUAL, ring=ring),
+                              dict(x=xs[1], fmt=ops.E4M3, layout=ops.DUAL, ring=other),
+                              dict(x=xs[2], fmt=ops.E4M3, layout=ops.DUAL, ring=ring)])
+    e0 = ops.quantize(xs[0], ops.E4M3, ops.DUAL, ref)
+    e1 = ops.quantize(xs[1], ops.E4M3, ops.DUAL, ref_other)
+    e2 = ops.quantize(xs[2], ops.E4M3, ops.DUAL, ref)
+    torch.cuda.synchronize()
+    for (o, t), (eo, et) in zip(got, (e0, e1, e2)):
+        assert torch.equal(o, eo) and torch.equal(t, et)
+    assert torch.equal(ring.buf, ref.buf) and torch.equal(other.buf, ref_other.buf)
+
+
 def test_quantize_pair_with_one_ring_runs_in_order():
     """Naming the same ring twice is two calls in order (the second sees the
     scale the first published)."""

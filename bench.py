@@ -244,9 +244,9 @@ class Linear:
     # The same step with the layout tag: row-layout quantizes only, and the
     # backward GEMMs read W, G and X as quantized through MN-major operands.
     def quantize_row(self, ops, x, g):
-        ops.quantize_pair(dict(x=x, fmt=ops.E4M3, layout=ops.ROW, ring=self.rx, out=self.xq),
-                          dict(x=self.w, fmt=ops.E4M3, layout=ops.ROW, ring=self.rw, out=self.wq))
-        ops.quantize(g, ops.E5M2, ops.ROW, self.rg, self.gq)
+        ops.quantize_multi([dict(x=x, fmt=ops.E4M3, layout=ops.ROW, ring=self.rx, out=self.xq),
+                            dict(x=self.w, fmt=ops.E4M3, layout=ops.ROW, ring=self.rw, out=self.wq),
+                            dict(x=g, fmt=ops.E5M2, layout=ops.ROW, ring=self.rg, out=self.gq)])
 
     def gemms_mn(self, ops):
         ops.mm(self.xq, self.wq, self.rx.scale_inv, self.rw.scale_inv, self.bias, out=self.y, workspace=self.ws)

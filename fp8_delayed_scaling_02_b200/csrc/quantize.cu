@@ -362,13 +362,25 @@ __global__ void __launch_bounds__(kRowThreads) quantize_row_kernel(const __grid_
   row_body<DT, FMT, kAligned>(a, blockIdx.x, gridDim.x);
 }
 
-// Two tensors in one launch: blocks [0, split) cast a0, the rest a1.
-template <int DT, int FMT, bool kAligned>
-__global__ void __launch_bounds__(kRowThreads)
-    quantize_row_pair_kernel(const __grid_constant__ RowArgs a0, const __grid_constant__ RowArgs a1,
-                             const unsigned split) {
-  if (blockIdx.x < split) row_body<DT, FMT, kAligned>(a0, blockIdx.x, split);
-  else row_body<DT, FMT, kAligned>(a1, blockIdx.x - split, gridDim.x - split);
+// Several tensors in one launch: blocks [split[s], split[s+1]) cast tensor
+// s, each set with its own ring and ticket (one instantiation of the row body
+// per format, chosen per block).
+constexpr int kMaxMulti = 8;
+
+struct RowMultiArgs {
+  RowArgs a[kMaxMulti];
+  int fmt[kMaxMulti];
+  unsigned split[kMaxMulti + 1];
+  int n;
+};
+
+template <int DT, bool kAligned>
+__global__ void __launch_bounds__(kRowThreads) quantize_row_multi_kernel(const __grid_constant__ RowMultiArgs m) {
+  int s = 0;
+  while (s + 1 < m.n && blockIdx.x >= m.split[s + 1]) ++s;
+  const unsigned blk = blockIdx.x - m.split[s], nblk = m.split[s + 1] - m.split[s];
+  if (m.fmt[s] == FP8_E5M2) row_body<DT, FP8_E5M2, kAligned>(m.a[s], blk, nblk);
+  else row_body<DT, FP8_E4M3, kAligned>(m.a[s], blk, nblk);
 }
 
 // ---- T / DUAL layouts --------------------------------------------------------
@@ -959,7 +971,6 @@ __global__ void __launch_bounds__(kWsThreads) quantize_tile_tma_kernel(const __g
 // ticket and tile counter, so each tensor's result is exactly that of its
 // own launch.  The tensors share the dtype and layout (one instantiation of
 // the tile body per format, chosen per block).
-constexpr int kMaxMulti = 8;
 
 struct TmaMultiArgs {
   CUtensorMap maps[kMaxMulti];
@@ -1301,32 +1312,61 @@ int quantize_dispatch(const void* in, int dtype, int64_t rows, int64_t cols, int
   return rc != FP8_OK ? rc : quantize_launch(q, sms, st);
 }
 
-// ---- two tensors in one launch -----------------------------------------------
+// ---- several tensors in one launch -------------------------------------------
 
-// Blocks for side 0 out of g, in proportion to the work w0 : w1, at least one
-// each side.
-int64_t share0(int64_t g, int64_t w0, int64_t w1) {
-  const int64_t s = (g * w0 + (w0 + w1) / 2) / std::max<int64_t>(1, w0 + w1);
-  return std::min<int64_t>(std::max<int64_t>(s, 1), g - 1);
-}
-
-template <int DT, int FMT, bool kAligned>
-int launch_row_pair1(const RowArgs& a0, const RowArgs& a1, int sms, cudaStream_t st) {
+// One launch for n ROW plans with the same dtype and input alignment, each
+// non-empty and on its own ring: the wave is shared in proportion to the
+// chunks, and each tensor is sized as a single launch with its share (every
+// thread the same number of chunks, at least kRowMinChunks).
+template <int DT, bool kAligned>
+int launch_row_multi1(const QPlan* const* qs, int n, int sms, cudaStream_t st) {
   static int cached[64] = {0};
-  const int bps = resident_blocks(quantize_row_pair_kernel<DT, FMT, kAligned>, kRowThreads, cached);
+  const int bps = resident_blocks(quantize_row_multi_kernel<DT, kAligned>, kRowThreads, cached);
   if (bps <= 0) return FP8_ERR_CUDA;
   const int64_t G = int64_t(bps) * sms;
-  const int64_t g0max = share0(G, a0.nchunks + 1, a1.nchunks + 1);
-  // Each side sized as a single launch with its share of the wave.
-  auto size = [](const RowArgs& a, int64_t gmax) {
+  int64_t W = 0;
+  for (int i = 0; i < n; ++i) W += qs[i]->ra.nchunks + 1;
+  RowMultiArgs m;
+  std::memset(&m, 0, sizeof(m));
+  m.n = n;
+  m.split[0] = 0;
+  for (int i = 0; i < n; ++i) {
+    const RowArgs& a = qs[i]->ra;
+    const int64_t gmax = std::max<int64_t>(1, (G - n) * (a.nchunks + 1) / W);
     const int64_t tmax = gmax * kRowThreads;
     const int64_t per = std::max<int64_t>(kRowMinChunks, (a.nchunks + tmax - 1) / tmax);
-    return std::max<int64_t>(1, (a.nchunks + per * kRowThreads - 1) / (per * kRowThreads));
-  };
-  const int64_t g0 = size(a0, g0max), g1 = size(a1, G - g0max);
-  const cudaError_t e = launch_pdl(quantize_row_pair_kernel<DT, FMT, kAligned>, dim3(unsigned(g0 + g1)), kRowThreads, 0,
-                                   st, 1, a0, a1, unsigned(g0));
+    const int64_t g = std::max<int64_t>(1, (a.nchunks + per * kRowThreads - 1) / (per * kRowThreads));
+    m.split[i + 1] = m.split[i] + unsigned(g);
+    m.a[i] = a;
+    m.fmt[i] = qs[i]->fmt;
+  }
+  const cudaError_t e = launch_pdl(quantize_row_multi_kernel<DT, kAligned>, dim3(m.split[n]), kRowThreads, 0, st, 1, m);
   return e == cudaSuccess ? FP8_OK : FP8_ERR_CUDA;
+}
+
+int launch_row_multi(const QPlan* const* qs, int n, int sms, cudaStream_t st) {
+  const bool al = qs[0]->aligned;
+  switch (qs[0]->dtype) {
+    case FP8_IN_BF16:
+      return al ? launch_row_multi1<FP8_IN_BF16, true>(qs, n, sms, st)
+                : launch_row_multi1<FP8_IN_BF16, false>(qs, n, sms, st);
+    case FP8_IN_FP16:
+      return al ? launch_row_multi1<FP8_IN_FP16, true>(qs, n, sms, st)
+                : launch_row_multi1<FP8_IN_FP16, false>(qs, n, sms, st);
+    default:
+      return al ? launch_row_multi1<FP8_IN_FP32, true>(qs, n, sms, st)
+                : launch_row_multi1<FP8_IN_FP32, false>(qs, n, sms, st);
+  }
+}
+
+// ROW plans that can share one launch: same dtype and input alignment, each
+// non-empty (formats may differ).
+bool row_fusable(const QPlan* const* qs, int n) {
+  for (int i = 0; i < n; ++i) {
+    if (qs[i]->kind != kQRow || qs[i]->ra.n <= 0) return false;
+    if (qs[i]->dtype != qs[0]->dtype || qs[i]->aligned != qs[0]->aligned) return false;
+  }
+  return true;
 }
 
 // One launch for n TMA-tile quantize plans with the same dtype and layout,
@@ -1392,37 +1432,19 @@ bool tma_fusable(const QPlan* const* qs, int n) {
   return true;
 }
 
-template <int DT, int FMT>
-int launch_row_pair_dt_fmt(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
-  return q0.aligned ? launch_row_pair1<DT, FMT, true>(q0.ra, q1.ra, sms, st)
-                    : launch_row_pair1<DT, FMT, false>(q0.ra, q1.ra, sms, st);
-}
-
-template <int DT>
-int launch_row_pair_dt(const QPlan& q0, const QPlan& q1, int sms, cudaStream_t st) {
-  return q0.fmt == FP8_E4M3 ? launch_row_pair_dt_fmt<DT, FP8_E4M3>(q0, q1, sms, st)
-                            : launch_row_pair_dt_fmt<DT, FP8_E5M2>(q0, q1, sms, st);
-}
-
-// Both calls in one launch when they resolve to the same kernel (ROW with
-// the same alignment and format, or TMA tiles with the same layout) and
-// neither is empty; otherwise one launch each, in order.
-int quantize_pair_dispatch(QPlan& q0, QPlan& q1, cudaStream_t st) {
+// Calls (on distinct rings) in one launch when they resolve to the same
+// kernel -- ROW with the same dtype and alignment, or TMA tiles with the same
+// dtype and layout -- and none is empty; otherwise one launch each, in order.
+int quantize_multi_dispatch(const QPlan* const* qs, int n, cudaStream_t st) {
   const int sms = sm_count_current();
   if (sms <= 0) return FP8_ERR_CUDA;
-  const QPlan* qs[2] = {&q0, &q1};
-  if (tma_fusable(qs, 2)) return launch_tile_tma_multi(qs, 2, sms, st);
-  const bool rows = q0.kind == kQRow && q1.kind == kQRow && q0.dtype == q1.dtype && q0.fmt == q1.fmt &&
-                    q0.aligned == q1.aligned && q0.ra.n > 0 && q1.ra.n > 0;
-  if (!rows) {
-    const int rc = quantize_launch(q0, sms, st);
-    return rc != FP8_OK ? rc : quantize_launch(q1, sms, st);
+  if (n > 1 && tma_fusable(qs, n)) return launch_tile_tma_multi(qs, n, sms, st);
+  if (n > 1 && row_fusable(qs, n)) return launch_row_multi(qs, n, sms, st);
+  for (int i = 0; i < n; ++i) {
+    const int rc = quantize_launch(*qs[i], sms, st);
+    if (rc != FP8_OK) return rc;
   }
-  switch (q0.dtype) {
-    case FP8_IN_BF16: return launch_row_pair_dt<FP8_IN_BF16>(q0, q1, sms, st);
-    case FP8_IN_FP16: return launch_row_pair_dt<FP8_IN_FP16>(q0, q1, sms, st);
-    default: return launch_row_pair_dt<FP8_IN_FP32>(q0, q1, sms, st);
-  }
+  return FP8_OK;
 }
 
 }  // namespace
@@ -1477,13 +1499,10 @@ extern "C" int fp8_quantize_pair(const fp8_quantize_args* q0, const fp8_quantize
   }
   // One ring for both: two calls in order, as the caller wrote them.
   const bool shared = q0->ring.scratch == q1->ring.scratch || q0->ring.history == q1->ring.history;
-  if (shared) {
-    const int sms = sm_count_current();
-    if (sms <= 0) return FP8_ERR_CUDA;
-    const int rc = quantize_launch(p[0], sms, st);
-    return rc != FP8_OK ? rc : quantize_launch(p[1], sms, st);
-  }
-  return quantize_pair_dispatch(p[0], p[1], st);
+  const QPlan* ptrs[2] = {&p[0], &p[1]};
+  if (!shared) return quantize_multi_dispatch(ptrs, 2, st);
+  const int rc = quantize_multi_dispatch(ptrs, 1, st);
+  return rc != FP8_OK ? rc : quantize_multi_dispatch(ptrs + 1, 1, st);
 }
 
 extern "C" int fp8_quantize_multi(const fp8_quantize_args* qs, int n, fp8_stream_t stream) {
@@ -1510,12 +1529,9 @@ extern "C" int fp8_quantize_multi(const fp8_quantize_args* qs, int n, fp8_stream
     for (int j = i + 1; j < n; ++j)
       if (qs[i].ring.scratch == qs[j].ring.scratch || qs[i].ring.history == qs[j].ring.history) distinct = false;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const int sms = sm_count_current();
-  if (sms <= 0) return FP8_ERR_CUDA;
-  if (distinct && n > 1 && tma_fusable(ptrs, n)) return launch_tile_tma_multi(ptrs, n, sms, st);
-  if (distinct && n == 2) return quantize_pair_dispatch(p[0], p[1], st);
+  if (distinct) return quantize_multi_dispatch(ptrs, n, st);
   for (int i = 0; i < n; ++i) {
-    const int rc = quantize_launch(p[i], sms, st);
+    const int rc = quantize_multi_dispatch(ptrs + i, 1, st);
     if (rc != FP8_OK) return rc;
   }
   return FP8_OK;

@@ -155,12 +155,12 @@ int fp8_quantize_static_scratch(const void* in, int dtype, int64_t rows, int64_t
  * fp8_quantize_pair -- two fp8_quantize calls (each on its own ring) in one
  * launch, such as a linear's X and W before its forward GEMM.
  *
- * When both resolve to the same kernel (ROW inputs with the same dtype,
- * fmt and 16-byte alignment; or T/DUAL inputs with the same dtype and layout,
- * 16-byte aligned bases and rows that are a multiple of 16 bytes, formats free)
- * and neither is empty, one grid is split between them in proportion to
- * their sizes; each set of blocks has its own amax ticket and folds its own
- * ring.  Otherwise the two run one after the other on `stream`.  Each
+ * When both resolve to the same kernel (ROW inputs with the same dtype and
+ * 16-byte alignment of their data; or T/DUAL inputs with the same dtype and
+ * layout, 16-byte aligned bases and rows that are a multiple of 16 bytes;
+ * the formats may differ) and neither is empty, one grid is split between
+ * them in proportion to their sizes; each set of blocks has its own amax
+ * ticket and folds its own ring.  Otherwise the two run one after the other on `stream`.  Each
  * result (codes, ring, scales) is exactly that of the fp8_quantize call with
  * the same arguments.  If both name the same ring the two calls run in order
  * (a ring cannot serve two calls at once).
@@ -183,14 +183,15 @@ int fp8_quantize_pair(const fp8_quantize_args* q0, const fp8_quantize_args* q1, 
  * fp8_quantize_multi -- n fp8_quantize calls (each on its own ring) in one
  * launch, such as a linear's X, W and G before its GEMMs.
  *
- * When every call is transposed or dual with the same dtype and layout, a
- * 16-byte aligned base, rows that are a multiple of 16 bytes and a
- * non-empty input (the formats may differ), and no ring is named twice, one
- * grid is split between them in proportion to their tiles: each tensor's
- * blocks claim its own tiles, reduce its own amax and fold its own ring, so
- * the launch's start-up and end costs are paid once instead of n times.
- * Otherwise the calls run in order on `stream` (two calls as
- * fp8_quantize_pair).  Each result (codes, ring, scales) is exactly that of
+ * When no ring is named twice, every input is non-empty and the calls
+ * resolve to one kernel -- all ROW with the same dtype and 16-byte alignment
+ * of their data, or all transposed or all dual with the same dtype, 16-byte
+ * aligned bases and rows that are a multiple of 16 bytes (in both cases the
+ * formats may differ) -- one grid is split between them in proportion to
+ * their sizes: each tensor's blocks cast its own elements, reduce its own
+ * amax and fold its own ring, so the launch's start-up and end costs are
+ * paid once instead of n times.  Otherwise the calls run in order on
+ * `stream`.  Each result (codes, ring, scales) is exactly that of
  * the fp8_quantize call with the same arguments.
  *   qs      host array of n structs; each field as the fp8_quantize argument
  *           of that name.

@@ -3,11 +3,11 @@
 Per step and per linear shape (W1 [1536,1536], W2 [4096,1536]), in the launch
 configurations the bench times: fwd Y = Xq.Wq^T + b (fp8_mm with the
 stream-K workspace) and dX = Gq.Wq, dW = Gq^T.Xq in one fp8_mm_pair launch,
-each GEMM with its rings' scale_inv -- either with X, W (E4M3) and G (E5M2)
-dual-quantized in one fp8_quantize_multi launch and NT backward GEMMs on the
-transposed copies (the headline step), or with row quantizes only (X and W
-in one fp8_quantize_pair launch, G alone) and the backward GEMMs reading the
-row copies as MN-major operands (the layout-tag step).  The three rings are checked
+each GEMM with its rings' scale_inv, and X, W (E4M3) and G (E5M2) quantized
+in one fp8_quantize_multi launch -- either in dual layout with NT backward
+GEMMs on the transposed copies (the headline step), or in row layout only with
+the backward GEMMs reading the row copies as MN-major operands (the layout-tag
+step).  The three rings are checked
 against the oracle after every step (bit-exact: amax history, idx, scale,
 scale_inv).  At the first and the last step every byte of the six quantized
 tensors is compared, and the three GEMM outputs on three rows of every
@@ -68,14 +68,10 @@ def test_linear_1p2b_sixteen_delayed_steps(M, which, layout_tag):
     for step in range(STEPS):
         x, g = S.linear_1p2b_step(M, n_out, step)
         sx, sw, sg = ox.scale, ow.scale, og.scale  # scales this step's quantizes use
-        if layout_tag:
-            ops.quantize_pair(dict(x=x.cuda(), fmt=ops.E4M3, layout=ops.ROW, ring=rx, out=xq),
-                              dict(x=wd, fmt=ops.E4M3, layout=ops.ROW, ring=rw, out=wq))
-            ops.quantize(g.cuda(), ops.E5M2, ops.ROW, rg, gq)
-        else:
-            ops.quantize_multi([dict(x=x.cuda(), fmt=ops.E4M3, layout=ops.DUAL, ring=rx, out=xq, out_t=xq_t),
-                                dict(x=wd, fmt=ops.E4M3, layout=ops.DUAL, ring=rw, out=wq, out_t=wq_t),
-                                dict(x=g.cuda(), fmt=ops.E5M2, layout=ops.DUAL, ring=rg, out=gq, out_t=gq_t)])
+        lay = ops.ROW if layout_tag else ops.DUAL
+        ops.quantize_multi([dict(x=x.cuda(), fmt=ops.E4M3, layout=lay, ring=rx, out=xq, out_t=xq_t),
+                            dict(x=wd, fmt=ops.E4M3, layout=lay, ring=rw, out=wq, out_t=wq_t),
+                            dict(x=g.cuda(), fmt=ops.E5M2, layout=lay, ring=rg, out=gq, out_t=gq_t)])
         ops.mm(xq, wq, rx.scale_inv, rw.scale_inv, bd, out=y, workspace=ws)
         if layout_tag:
             ops.mm_pair(dict(a=gq, b=wq, sinv_a=rg.scale_inv, sinv_b=rw.scale_inv, fmt_a=ops.E5M2, out=dx,

@@ -301,13 +301,14 @@ QMULTI = [
     # Eight tensors of very different sizes, one launch.
     [((2048, 1536), "fp32", 1), ((128, 64), "fp32", 0), ((130, 64), "fp32", 1), ((1, 4), "fp32", 0),
      ((64, 4), "fp32", 0), ((300, 68), "fp32", 1), ((1000, 128), "fp32", 0), ((129, 8), "fp32", 1)],
-    # Not fusable (an odd width, an empty input): calls in order.
+    # T / DUAL: not fusable (an odd width, an empty input), calls in order;
+    # ROW: not fusable (an empty input).
     [((256, 512), "bf16", 0), ((300, 1537), "bf16", 1), ((0, 64), "bf16", 0)],
     [((777, 512), "fp16", 1)],
 ]
 
 
-@pytest.mark.parametrize("layout", [ops.TRANSPOSED, ops.DUAL])
+@pytest.mark.parametrize("layout", [ops.ROW, ops.TRANSPOSED, ops.DUAL])
 @pytest.mark.parametrize("case", range(len(QMULTI)))
 def test_quantize_multi_equals_the_single_calls(case, layout):
     specs = QMULTI[case]

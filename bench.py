@@ -66,6 +66,7 @@ def parse():
                     help="gemm sweep: output kinds to time, of bf16,e4m3,e5m2 (FP8 outputs fold an output ring)")
     ap.add_argument("--qdtypes", default="bf16,fp32", help="quantize sweep input dtypes")
     ap.add_argument("--qlayouts", default="row,T,dual", help="quantize sweep layouts")
+    ap.add_argument("--qmisalign", action="store_true", help="quantize sweep: also time a base one element past 16 B")
     return ap.parse_args()
 
 
@@ -517,23 +518,39 @@ def sweep(args):
         want = [tuple(int(v) for v in s.split("x")) for s in args.shapes.split(",")] if args.shapes else None
         for rows, cols in (QUANT_SHAPES if not want else want):
             for dt in args.qdtypes.split(","):
-                x = S.quant_sweep_input(rows, cols, dt, 1.0).cuda()
-                eb = x.element_size()
-                for layout, name in ((ops.ROW, "row"), (ops.TRANSPOSED, "T"), (ops.DUAL, "dual")):
-                    if name not in args.qlayouts.split(","):
+                x0 = S.quant_sweep_input(rows, cols, dt, 1.0).cuda()
+                eb = x0.element_size()
+                # The input at a 16-byte aligned base and one element past it.
+                flat = torch.empty(rows * cols + 1, dtype=x0.dtype, device="cuda")
+                flat[1:].copy_(x0.reshape(-1))
+                for base, x in (("aligned", x0), ("+1 element", flat[1:].view(rows, cols))):
+                    if base != "aligned" and not args.qmisalign:
                         continue
-                    ring = ops.Ring()
-                    out = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
-                    out_t = torch.empty((cols, rows), dtype=torch.uint8, device="cuda")
-                    fn = lambda: ops.quantize(x, ops.E4M3, layout, ring, out, out_t)  # noqa: E731
-                    for _ in range(3):
-                        fn()
-                    ms = _kernel_ms(fn, torch, args.iters, flush)
-                    nbytes = rows * cols * (eb + (2 if layout == ops.DUAL else 1)) + 96
-                    print(json.dumps({"kernel": "quantize", "dtype": dt, "layout": name, "rows": rows,
-                                      "cols": cols, "us": round(ms * 1e3, 2),
-                                      "gbs": round(nbytes / ms / 1e6, 1)}))
+                    for layout, name in ((ops.ROW, "row"), (ops.TRANSPOSED, "T"), (ops.DUAL, "dual")):
+                        if name not in args.qlayouts.split(","):
+                            continue
+                        ring = ops.Ring()
+                        out = torch.empty((rows, cols), dtype=torch.uint8, device="cuda")
+                        out_t = torch.empty((cols, rows), dtype=torch.uint8, device="cuda")
+                        fn = lambda: ops.quantize(x, ops.E4M3, layout, ring, out, out_t)  # noqa: E731
+                        for _ in range(3):
+                            fn()
+                        ms = _kernel_ms(fn, torch, args.iters, flush)
+                        nbytes = rows * cols * (eb + (2 if layout == ops.DUAL else 1)) + 96
+                        print(json.dumps({"kernel": "quantize", "dtype": dt, "layout": name, "rows": rows,
+                                          "cols": cols, "base": base, "us": round(ms * 1e3, 2),
+                                          "gbs": round(nbytes / ms / 1e6, 1),
+                                          "frac": round(nbytes / ms / 1e6 / hbm_peak_gbs(), 3)}))
     return 0
+
+
+def hbm_peak_gbs():
+    """The measured HBM copy bandwidth (GB/s) of this machine, else the fallback figure."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f).get("hbm_gbs", 6650.0))
+    except (OSError, ValueError):
+        return 6650.0
 
 
 def _time_rotating(torch, fns, reps):
